@@ -1,0 +1,186 @@
+/*
+ * oracle.c -- plain fp64 CPU oracle for the fused tensor-core GEMM
+ *
+ *     C = epilogue(A . B),   epilogue(x)[i,j] = GELU(x[i,j] + bias[j])  or  identity
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check of the build
+ * entry point and the CPU-baseline leg of the benchmark may load this file.
+ * The product path never calls it, never links it, and shares no code with it.
+ *
+ * What it follows:
+ *   - "Designing High-Performance GPU Kernels with TileLang" (blog retelling),
+ *     Step 4 "Tensor-Core GEMM": A_shared is (block_M, block_K), B_shared is
+ *     (block_K, block_N), so A is M x K and B is K x N, both row-major; the
+ *     accumulator fragment is float32.  Here the accumulation is done in fp64,
+ *     an exact stand-in: every product of two fp16 (or two bf16) values is
+ *     exact in fp64, so the only error left is the fp64 summation.
+ *   - TileLang GPU kernel design article, paragraph 5 (fused GEMM epilogue):
+ *     bias add, then GELU, applied to the accumulator before the one write
+ *     of the output.  Read as: per-column bias (length N), added
+ *     first; GELU in its exact form 0.5 x (1 + erf(x / sqrt 2)).
+ *
+ * Plain definition, no blocking, no reordering: for each output element the
+ * sum over k runs k = 0 .. K-1 in order, in double.  The result is kept in
+ * fp64 and is NOT rounded to the input dtype.
+ *
+ * Inputs are raw 16-bit patterns (IEEE binary16 or bfloat16), decoded here
+ * from the format definitions.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#define ORACLE_F16 0
+#define ORACLE_BF16 1
+#define ORACLE_EPI_NONE 0
+#define ORACLE_EPI_BIAS_GELU 1
+
+/* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits.
+ * Normal: (1024 + f) * 2^(e - 25).  Subnormal (e = 0): f * 2^-24.          */
+static double decode_f16(uint16_t h)
+{
+    int s = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(f + 1024), e - 25);
+    return s ? -v : v;
+}
+
+/* bfloat16: 1 sign bit, 8 exponent bits (bias 127), 7 fraction bits.
+ * Normal: (128 + f) * 2^(e - 134).  Subnormal (e = 0): f * 2^-133.         */
+static double decode_bf16(uint16_t h)
+{
+    int s = (h >> 15) & 1;
+    int e = (h >> 7) & 0xff;
+    int f = h & 0x7f;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -133);
+    else if (e == 255)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(f + 128), e - 134);
+    return s ? -v : v;
+}
+
+static double decode(uint16_t h, int dtype)
+{
+    return dtype == ORACLE_BF16 ? decode_bf16(h) : decode_f16(h);
+}
+
+/* Exact (erf) GELU: x * Phi(x) with Phi the standard normal CDF,
+ * Phi(x) = (1 + erf(x / sqrt 2)) / 2.                                       */
+double oracle_gelu(double x)
+{
+    return 0.5 * x * (1.0 + erf(x / sqrt(2.0)));
+}
+
+void oracle_gelu_array(const double *x, double *y, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        y[i] = oracle_gelu(x[i]);
+}
+
+void oracle_decode_array(const uint16_t *bits, int dtype, double *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = decode(bits[i], dtype);
+}
+
+/* Rows `rows[0..nrows)` of C, written densely to out[r * N + j].
+ * Returns 0 on success, -1 if a row index is out of range or memory runs out. */
+int oracle_gemm_rows(int64_t M, int64_t N, int64_t K,
+                     const uint16_t *A, const uint16_t *B, const uint16_t *bias,
+                     int dtype, int epi,
+                     const int64_t *rows, int64_t nrows, double *out)
+{
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= M)
+            return -1;
+    if (epi == ORACLE_EPI_BIAS_GELU && bias == NULL)
+        return -1;
+
+    /* B decoded once; every row reads all of it. */
+    double *Bd = (double *)malloc((size_t)(K * N > 0 ? K * N : 1) * sizeof(double));
+    if (!Bd)
+        return -1;
+    oracle_decode_array(B, dtype, Bd, K * N);
+
+    int64_t r;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < nrows; ++r) {
+        const int64_t i = rows[r];
+        double *c = out + r * N;
+        for (int64_t j = 0; j < N; ++j)
+            c[j] = 0.0;
+        /* c[j] = sum_{k=0}^{K-1} A[i,k] * B[k,j], k in increasing order */
+        for (int64_t k = 0; k < K; ++k) {
+            const double a = decode(A[i * K + k], dtype);
+            const double *b = Bd + k * N;
+            for (int64_t j = 0; j < N; ++j)
+                c[j] += a * b[j];
+        }
+        if (epi == ORACLE_EPI_BIAS_GELU)
+            for (int64_t j = 0; j < N; ++j)
+                c[j] = oracle_gelu(c[j] + decode(bias[j], dtype));
+    }
+    free(Bd);
+    return 0;
+}
+
+/* Whole C (M x N, row-major, fp64). */
+int oracle_gemm(int64_t M, int64_t N, int64_t K,
+                const uint16_t *A, const uint16_t *B, const uint16_t *bias,
+                int dtype, int epi, double *C)
+{
+    int64_t *rows = (int64_t *)malloc((size_t)(M > 0 ? M : 1) * sizeof(int64_t));
+    if (!rows)
+        return -1;
+    for (int64_t i = 0; i < M; ++i)
+        rows[i] = i;
+    int rc = oracle_gemm_rows(M, N, K, A, B, bias, dtype, epi, rows, M, C);
+    free(rows);
+    return rc;
+}
+
+/* Single elements C[ii[p], jj[p]] for p < npts: the same sum, same k order. */
+int oracle_gemm_points(int64_t M, int64_t N, int64_t K,
+                       const uint16_t *A, const uint16_t *B, const uint16_t *bias,
+                       int dtype, int epi,
+                       const int64_t *ii, const int64_t *jj, int64_t npts, double *out)
+{
+    for (int64_t p = 0; p < npts; ++p)
+        if (ii[p] < 0 || ii[p] >= M || jj[p] < 0 || jj[p] >= N)
+            return -1;
+    if (epi == ORACLE_EPI_BIAS_GELU && bias == NULL)
+        return -1;
+    int64_t p;
+#pragma omp parallel for schedule(static)
+    for (p = 0; p < npts; ++p) {
+        const int64_t i = ii[p], j = jj[p];
+        double s = 0.0;
+        for (int64_t k = 0; k < K; ++k)
+            s += decode(A[i * K + k], dtype) * decode(B[k * N + j], dtype);
+        if (epi == ORACLE_EPI_BIAS_GELU)
+            s = oracle_gelu(s + decode(bias[j], dtype));
+        out[p] = s;
+    }
+    return 0;
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,55 @@
+"""Plant plausible mistakes in copies of the oracle (on the CPU) and show that
+each one fails at least one pin.  The copies are built in a temporary folder;
+the oracle in oracle/ is never modified."""
+import os
+import sys
+
+import pytest
+
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+import oracle  # noqa: E402
+from oracle_pins import ALL_PINS  # noqa: E402
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+# (name, text in oracle.c, replacement).  Every replacement stays in bounds.
+MUTANTS = [
+    ("transposed_B_rows", "c[j] += a * b[j];", "c[j] += a * Bd[j * K + k];"),
+    ("transposed_B_points", "decode(B[k * N + j], dtype)", "decode(B[j * K + k], dtype)"),
+    ("dropped_first_k", "for (int64_t k = 0; k < K; ++k) {", "for (int64_t k = 1; k < K; ++k) {"),
+    ("wrong_sign", "c[j] += a * b[j];", "c[j] -= a * b[j];"),
+    ("float_accumulator", "c[j] += a * b[j];", "c[j] = (float)(c[j] + a * b[j]);"),
+    ("tanh_gelu", "return 0.5 * x * (1.0 + erf(x / sqrt(2.0)));",
+     "return 0.5 * x * (1.0 + tanh(0.7978845608028654 * (x + 0.044715 * x * x * x)));"),
+    ("gelu_wrong_scale", "erf(x / sqrt(2.0))", "erf(x / 2.0)"),
+    ("bias_after_gelu", "c[j] = oracle_gelu(c[j] + decode(bias[j], dtype));",
+     "c[j] = oracle_gelu(c[j]) + decode(bias[j], dtype);"),
+    ("bias_by_row", "c[j] = oracle_gelu(c[j] + decode(bias[j], dtype));",
+     "c[j] = oracle_gelu(c[j] + decode(bias[i % N], dtype));"),
+    ("f16_exponent_bias", "v = ldexp((double)(f + 1024), e - 25);", "v = ldexp((double)(f + 1024), e - 24);"),
+    ("f16_subnormal_as_normal", "v = ldexp((double)f, -24);", "v = ldexp((double)(f + 1024), -25);"),
+    ("bf16_exponent_bias", "v = ldexp((double)(f + 128), e - 134);", "v = ldexp((double)(f + 128), e - 133);"),
+    ("bf16_fraction_width", "int f = h & 0x7f;", "int f = h & 0x3f;"),
+    ("last_k_dropped_points", "for (int64_t k = 0; k < K; ++k)\n            s +=",
+     "for (int64_t k = 0; k + 1 < K; ++k)\n            s +="),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_fails_a_pin(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    mutated = src.replace(old, new, 1)
+    csrc = tmp_path / f"oracle_{name}.c"
+    csrc.write_text(mutated)
+    so = oracle.build(force=True, src=str(csrc), out=str(tmp_path / f"liboracle_{name}.so"))
+    orc = oracle.from_library(so)
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            failed.append(pin.__name__)
+            break
+    assert failed, f"mutant {name} passed every pin"
