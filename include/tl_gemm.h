@@ -1,0 +1,162 @@
+/*
+ * tl_gemm.h -- C ABI of the B200 (sm_100a) fused tensor-core GEMM library
+ *              (libtlgemm.so).
+ *
+ * The operation, as the TileLang pages define it:
+ *
+ *   C = epilogue(A . B)
+ *
+ *   - "Designing High-Performance GPU Kernels with TileLang" (blog retelling),
+ *     Step 4 (Tensor-Core GEMM): A is M x K, B is K x N, both row-major (the
+ *     shared tiles are block_M x block_K and block_K x block_N); the inputs
+ *     are 16-bit floats and the accumulator is float32.
+ *   - TileLang GPU kernel design article, paragraph 5 (fused GEMM epilogue):
+ *     optionally add a per-column bias and apply GELU to the float32
+ *     accumulator before the single write of C, so no intermediate reaches
+ *     global memory.  GELU is the exact form x * Phi(x) =
+ *     0.5 x (1 + erf(x / sqrt 2)).
+ *
+ * The result is rounded once, to nearest even, from float32 to the input
+ * dtype.  Sums are accumulated in float32 on the tensor cores; the order of
+ * the sum is fixed by the kernel configuration, so two calls with the same
+ * configuration give bit-identical results.
+ *
+ * All calls are host functions.  None of them allocates memory that outlives
+ * the call; a call that must re-lay out an operand (see tl_gemm) takes a
+ * stream-ordered temporary from a library-owned CUDA memory pool and returns
+ * it on the same stream.
+ */
+#ifndef TL_GEMM_H
+#define TL_GEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TL_VERSION 1000 /* major * 1000 + minor */
+
+#if defined(__GNUC__)
+#define TL_API __attribute__((visibility("default")))
+#else
+#define TL_API
+#endif
+
+typedef enum { TL_F16 = 0, TL_BF16 = 1 } tl_dtype;
+
+typedef enum {
+    TL_EPI_NONE = 0,      /* C = A.B                                   */
+    TL_EPI_BIAS_GELU = 1  /* C = GELU(A.B + bias[col]), exact erf GELU */
+} tl_epilogue;
+
+typedef enum {
+    TL_OK = 0,
+    TL_ERR_INVALID_ARG = 1,     /* null pointer, size <= 0, bad enum, missing bias */
+    TL_ERR_UNSUPPORTED = 2,     /* size beyond the 32-bit coordinate range, no sm_100 device */
+    TL_ERR_MISALIGNED = 3,      /* a pointer not aligned to its 2-byte element */
+    TL_ERR_CUDA = 4,            /* a CUDA runtime or driver call failed */
+    TL_ERR_DEVICE_TIMEOUT = 5   /* a bounded wait inside a kernel ran out (see tl_check_device) */
+} tl_status;
+
+/* A cudaStream_t, passed as an opaque pointer; NULL is the legacy default stream. */
+typedef void *tl_stream;
+
+/*
+ * tl_gemm -- C = epilogue(A . B) on the current CUDA device, asynchronously on
+ * `stream`.
+ *
+ *   A     device pointer, M x K, row-major (leading dimension K), `dtype`
+ *   B     device pointer, K x N, row-major (leading dimension N), `dtype`
+ *   bias  device pointer to N values of `dtype`; required when
+ *         epi == TL_EPI_BIAS_GELU, ignored (may be NULL) otherwise
+ *   C     device pointer, M x N, row-major (leading dimension N), `dtype`;
+ *         written, never read.  C must not overlap A, B or bias (not checked).
+ *   M, N, K   sizes, each in [1, 2^31 - 1]
+ *
+ * Layout requirements: every pointer must be aligned to 2 bytes.  Nothing
+ * else is required.  When a row stride of A or B is not a multiple of 16
+ * bytes (K or N not a multiple of 8) or its base is not 16-byte aligned, the
+ * call first copies that operand into a zero-padded temporary; when C's rows
+ * are not 16-byte aligned the epilogue stores element by element instead of
+ * through the tensor-memory-access unit.  Both are slower than the aligned
+ * path but give the same numbers.
+ *
+ * Ownership: the caller owns every buffer and must keep them alive until the
+ * work on `stream` completes.  The call does not synchronize.
+ *
+ * Returns TL_OK once the work is enqueued.  Argument errors are reported
+ * before anything is enqueued.  A fault found by the kernel itself (a bounded
+ * wait that ran out) is reported later by tl_check_device.
+ */
+TL_API tl_status tl_gemm(const void *A, const void *B, const void *bias, void *C,
+                  int64_t M, int64_t N, int64_t K,
+                  tl_dtype dtype, tl_epilogue epi, tl_stream stream);
+
+/* Options for tl_gemm_ex.  Zero-initialise, then set what you need. */
+typedef struct {
+    int32_t config;       /* 0: the library's choice for the shape; k > 0: kernel
+                             configuration k - 1 (see tl_num_configs)            */
+    int32_t inject_fault; /* test hook, 0 in production: 1 makes the copy warp
+                             skip its first stage without issuing the copy, so
+                             the consumer's bounded wait runs out and the kernel
+                             returns with TL_ERR_DEVICE_TIMEOUT recorded          */
+    uint64_t timeout_ns;  /* bound on every wait inside the kernel; 0 = 10 s     */
+} tl_gemm_options;
+
+/* tl_gemm with options (NULL options == tl_gemm).  Same arguments and errors;
+ * TL_ERR_INVALID_ARG also for a configuration index out of range.             */
+TL_API tl_status tl_gemm_ex(const void *A, const void *B, const void *bias, void *C,
+                     int64_t M, int64_t N, int64_t K,
+                     tl_dtype dtype, tl_epilogue epi, tl_stream stream,
+                     const tl_gemm_options *options);
+
+/*
+ * tl_check_device -- synchronize `stream`, then read and clear the error word
+ * the kernels of this library set on the current device when a bounded wait
+ * runs out.  Returns TL_ERR_DEVICE_TIMEOUT if it was set (the kernel stopped
+ * early, C is incomplete), TL_ERR_CUDA if the synchronization failed, TL_OK
+ * otherwise.  `detail`, if not NULL, receives the raw error word (which waits
+ * gave up: bit 0 copy warp, bit 1 MMA warp on data, bit 2 MMA warp on the
+ * accumulator, bit 3 epilogue warps, bit 4 final drain).
+ */
+TL_API tl_status tl_check_device(tl_stream stream, uint32_t *detail);
+
+/*
+ * tl_gemm_plan -- the host-side decision tl_gemm would take for these
+ * arguments, without launching anything (no GPU needed when num_sms > 0).
+ * Validation is the same as tl_gemm's and returns the same status.
+ */
+typedef struct {
+    int32_t config;          /* kernel configuration index                     */
+    int32_t block_m, block_n, block_k, stages;
+    int32_t tiles_m, tiles_n;
+    int32_t grid;            /* persistent CTAs launched                       */
+    int32_t pad_a, pad_b;    /* 1 when the operand is first copied to a padded temporary */
+    int32_t direct_store;    /* 1 when C is stored element by element          */
+    int32_t smem_bytes;      /* dynamic shared memory per CTA                  */
+    int64_t workspace_bytes; /* stream-ordered temporary the call takes        */
+} tl_plan;
+
+TL_API tl_status tl_gemm_plan(const void *A, const void *B, const void *bias, void *C,
+                       int64_t M, int64_t N, int64_t K,
+                       tl_dtype dtype, tl_epilogue epi, int32_t num_sms,
+                       const tl_gemm_options *options, tl_plan *plan);
+
+/* Number of compiled kernel configurations, and the name of configuration i
+ * ("bm128_bn256_bk64_s4" ...; NULL when i is out of range).                   */
+TL_API int32_t tl_num_configs(void);
+TL_API const char *tl_config_name(int32_t i);
+
+/* Human-readable name of a status code (never NULL). */
+TL_API const char *tl_status_string(tl_status s);
+
+/* TL_VERSION of the built library. */
+TL_API int32_t tl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TL_GEMM_H */

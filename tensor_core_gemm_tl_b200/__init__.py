@@ -1,0 +1,110 @@
+"""B200-native (sm_100a) fused tensor-core GEMM:  C = epilogue(A . B).
+
+The work runs in libtlgemm.so (hand-written tcgen05 / TMA kernels behind a C
+ABI, include/tl_gemm.h).  This package is its Python binding: the raw C-ABI
+calls (``tl_gemm``, ``tl_gemm_ex``, ``tl_check_device``, ``tl_gemm_plan`` ...)
+on device pointers, and ``gemm`` which takes torch CUDA tensors and passes
+their pointers and the current stream.  PyTorch only provides device memory
+and streams; nothing here computes.
+
+Importing the package fails if the library is not built -- there is no CPU
+or library fallback.
+"""
+from __future__ import annotations
+
+from ._binding import (  # noqa: F401
+    LIB_PATH, Options, Plan, Status, TLError, TL_BF16, TL_EPI_BIAS_GELU, TL_EPI_NONE, TL_F16,
+    SIGNATURES, tl_check_device, tl_config_name, tl_gemm, tl_gemm_ex, tl_gemm_plan, tl_num_configs,
+    tl_status_string, tl_version,
+)
+
+__all__ = [
+    "gemm", "check_device", "plan", "configs", "Options", "Plan", "Status", "TLError",
+    "tl_gemm", "tl_gemm_ex", "tl_check_device", "tl_gemm_plan", "tl_num_configs", "tl_config_name",
+    "tl_status_string", "tl_version", "TL_F16", "TL_BF16", "TL_EPI_NONE", "TL_EPI_BIAS_GELU",
+]
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float16:
+        return TL_F16
+    if t.dtype == torch.bfloat16:
+        return TL_BF16
+    raise TypeError(f"expected float16 or bfloat16, got {t.dtype}")
+
+
+def _epi_code(epilogue):
+    if epilogue in (None, "none", TL_EPI_NONE):
+        return TL_EPI_NONE
+    if epilogue in ("bias_gelu", "bias+gelu", TL_EPI_BIAS_GELU):
+        return TL_EPI_BIAS_GELU
+    raise ValueError(f"unknown epilogue {epilogue!r}")
+
+
+def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0, timeout_ns: int = 0):
+    """C = epilogue(A @ B) for row-major CUDA tensors A (M x K) and B (K x N).
+
+    ``epilogue`` is None / "none" or "bias_gelu" (``bias`` of length N is then
+    required).  ``out`` (M x N, same dtype) is written if given, else
+    allocated.  Runs asynchronously on ``stream`` (default: torch's current
+    stream).  ``config`` = k > 0 forces kernel configuration k - 1.
+    """
+    import torch
+    epi = _epi_code(epilogue if epilogue is not None else ("bias_gelu" if bias is not None else None))
+    if A.dim() != 2 or B.dim() != 2 or A.shape[1] != B.shape[0]:
+        raise ValueError(f"shapes {tuple(A.shape)} and {tuple(B.shape)} do not chain")
+    for name, t in (("A", A), ("B", B)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    dt = _dtype_code(A)
+    if B.dtype != A.dtype:
+        raise TypeError("A and B must have the same dtype")
+    M, K = A.shape
+    N = B.shape[1]
+    if epi == TL_EPI_BIAS_GELU:
+        if bias is None or bias.shape != (N,) or bias.dtype != A.dtype or not bias.is_cuda or not bias.is_contiguous():
+            raise ValueError("bias_gelu needs a contiguous CUDA bias of length N in the input dtype")
+    if out is None:
+        out = torch.empty((M, N), dtype=A.dtype, device=A.device)
+    elif out.shape != (M, N) or out.dtype != A.dtype or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous CUDA tensor of shape (M, N) and the input dtype")
+    s = stream if stream is not None else torch.cuda.current_stream(A.device)
+    with torch.cuda.device(A.device):
+        if config or timeout_ns:
+            opt = Options(config=config, inject_fault=0, timeout_ns=timeout_ns)
+            st = tl_gemm_ex(A.data_ptr(), B.data_ptr(), bias.data_ptr() if bias is not None else 0,
+                            out.data_ptr(), M, N, K, dt, epi, s.cuda_stream, opt)
+        else:
+            st = tl_gemm(A.data_ptr(), B.data_ptr(), bias.data_ptr() if bias is not None else 0,
+                         out.data_ptr(), M, N, K, dt, epi, s.cuda_stream)
+    if st != 0:
+        raise TLError(st, "tl_gemm")
+    return out
+
+
+def check_device(stream=None) -> int:
+    """Synchronize and return the device error word (0 = no wait ran out)."""
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    st, word = tl_check_device(s.cuda_stream)
+    if st not in (0, int(Status.DEVICE_TIMEOUT)):
+        raise TLError(st, "tl_check_device")
+    return word
+
+
+def plan(M, N, K, dtype=TL_F16, epilogue=None, num_sms=148, config=0, ptrs=(256, 256, 256, 256)) -> dict:
+    """The host plan for a call (no GPU needed): config, grid, padding, store path."""
+    a, b, bias, c = ptrs
+    epi = _epi_code(epilogue)
+    opt = Options(config=config) if config else None
+    st, p = tl_gemm_plan(a, b, bias if epi else 0, c, M, N, K, dtype, epi, num_sms, opt)
+    if st != 0:
+        raise TLError(st, "tl_gemm_plan")
+    d = p.as_dict()
+    d["config_name"] = tl_config_name(d["config"])
+    return d
+
+
+def configs() -> list[str]:
+    return [tl_config_name(i) for i in range(tl_num_configs())]

@@ -1,0 +1,465 @@
+// gemm_kernel.cuh -- persistent, warp-specialised sm_100a GEMM with a fused
+// bias + exact-GELU epilogue:  C = epilogue(A . B).
+//
+// What it computes follows "Designing High-Performance GPU Kernels with
+// TileLang" (blog retelling), Step 4 (tiled Tensor-Core GEMM: A tiles
+// block_M x block_K and B tiles block_K x block_N staged through shared memory
+// in a pipelined K loop, float32 accumulator) and the TileLang GPU kernel
+// design article, paragraph 5 (bias add and GELU applied to the accumulator
+// before the single store of C).  The pages' schedule (128/128/32, 2 stages,
+// register fragments, mma.sync class) targets T4/A100/L4; on sm_100a the same
+// roles map to:
+//
+//   global --TMA (128B swizzle)--> STAGES-deep shared-memory ring
+//          --tcgen05.mma (one thread)--> fp32 accumulator in Tensor Memory
+//          --tcgen05.ld--> registers: + bias, GELU, round once to fp16/bf16
+//          --st.shared (swizzled)--> TMA store --> global
+//
+// Warp roles (192 threads, one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer (one lane)
+//   warp 1      TMEM allocator + MMA issuer (one lane)
+//   warps 2..5  epilogue; warp w reads TMEM lanes 32*(w%4) .. +31
+//
+// Two TMEM accumulators (2 x BN fp32 columns) let the epilogue of tile i run
+// while the MMAs of tile i+1 accumulate.  Every wait is bounded by a
+// %globaltimer limit: on expiry the kernel records which wait gave up in a
+// device error word, lets its issued copies and MMAs land, frees TMEM and
+// returns (no trap, no hang).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "sm100.cuh"
+
+namespace tl {
+
+// Device error word, read and cleared by tl_check_device.  This header is
+// included by exactly one translation unit (tl_gemm.cu), which owns it.
+__device__ unsigned int g_device_error = 0;
+
+enum : unsigned {
+    ERR_PRODUCER = 1u,
+    ERR_MMA_DATA = 2u,
+    ERR_MMA_ACC = 4u,
+    ERR_EPILOGUE = 8u,
+    ERR_DRAIN = 16u,
+};
+
+struct GemmParams {
+    int32_t M, N, K;
+    int32_t tiles_m, tiles_n, num_tiles, num_kb;
+    int32_t group_m;         // output-tile rows per rasterisation group
+    const uint16_t *bias;    // N values of the input dtype (epilogue only)
+    int32_t bias_vec16;      // bias is 16-byte aligned: load 8 values per access
+    int32_t inject_fault;    // test hook: skip the first stage's copy
+    uint16_t *C;             // direct-store path only
+    int64_t ldc;             // direct-store path only (elements)
+    uint64_t timeout_ns;
+};
+
+// Compile-time tile configuration.  BM = 128 rows (one TMEM lane per row),
+// BK = 64 (one 128-byte swizzle row of 16-bit values), BN in {64, 128, 256}.
+template <int BN_, int STAGES_>
+struct TileConfig {
+    static constexpr int BM = 128, BN = BN_, BK = 64, STAGES = STAGES_;
+    static constexpr int A_STAGE_BYTES = BM * BK * 2;
+    static constexpr int B_BOX_BYTES = BK * 128;   // one 64-column box of B
+    static constexpr int B_STAGE_BYTES = BK * BN * 2;
+    static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+    static constexpr int EPI_WARPS = 4;
+    static constexpr int C_BOX_BYTES = 32 * 128;   // 32 rows x 64 columns of 16-bit
+    static constexpr int C_STAGING_BYTES = EPI_WARPS * 2 * C_BOX_BYTES;
+    static constexpr int ACC_COLS = BN;             // fp32 TMEM columns per accumulator
+    static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_STAGE_BYTES;
+    static constexpr int OFF_C = OFF_B + STAGES * B_STAGE_BYTES;
+    static constexpr int OFF_BAR = OFF_C + C_STAGING_BYTES;
+    static constexpr int NUM_BARS = 2 * STAGES + 5;
+    static constexpr int SMEM_USED = OFF_BAR + NUM_BARS * 8 + 16;
+    static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024
+    static constexpr int THREADS = 192;
+    static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+    static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM columns");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+// Output tile t -> (tile row, tile col), grouped so that consecutive tiles
+// share A rows within a group of `group_m` tile rows (L2 reuse).
+__device__ __forceinline__ void tile_coords(int t, const GemmParams &p, int &tm, int &tn)
+{
+    const int group_size = p.group_m * p.tiles_n;
+    const int g = t / group_size;
+    const int first_m = g * p.group_m;
+    const int rows = min(p.tiles_m - first_m, p.group_m);
+    const int r = t - g * group_size;
+    tm = first_m + r % rows;
+    tn = r / rows;
+}
+
+// Bounded wait.  Returns false when the abort flag is raised by another role
+// or when this wait runs past timeout_ns (then it raises the flag itself).
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                             uint64_t timeout_ns, unsigned code)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if (*abort_flag)
+            return false;
+        if (global_timer_ns() - t0 > timeout_ns) {
+            *abort_flag = 1;
+            atomicOr(&g_device_error, code);
+            return false;
+        }
+    }
+}
+
+// Bounded wait that ignores the abort flag (used to let in-flight work land).
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > timeout_ns) {
+            atomicOr(&g_device_error, ERR_DRAIN);
+            return false;
+        }
+    }
+    return true;
+}
+
+template <int DT>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi)
+{
+    if constexpr (DT == 1) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t *>(&v);
+    } else {
+        __half2 v = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t *>(&v);
+    }
+}
+
+template <int DT>
+__device__ __forceinline__ float to_float(uint16_t bits)
+{
+    if constexpr (DT == 1)
+        return __uint_as_float(static_cast<uint32_t>(bits) << 16);
+    else
+        return __half2float(__ushort_as_half(bits));
+}
+
+// Exact GELU on the fp32 accumulator: x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)).
+// Evaluated as 0.5 x erfc(-x / sqrt 2), the same function: for negative x the
+// form 1 + erf(.) subtracts two numbers close to 1 and loses most of its
+// float32 bits, erfc of a positive argument does not.
+__device__ __forceinline__ float gelu_erf(float x)
+{
+    return 0.5f * x * erfcf(x * -0.70710678118654752f);
+}
+
+template <class CF, int DT, int EPI, bool TMA_STORE>
+__global__ void __launch_bounds__(192, 1)
+    gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                      const __grid_constant__ CUtensorMap tmap_c, const GemmParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const uint32_t sA = smem_addr(smem + CF::OFF_A);
+    const uint32_t sB = smem_addr(smem + CF::OFF_B);
+    uint8_t *cstage = smem + CF::OFF_C;
+    const uint32_t bar0 = smem_addr(smem + CF::OFF_BAR);
+    // barrier i lives at bar0 + 8 i
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (CF::STAGES + s); };
+    auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * CF::STAGES + a); };
+    auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * CF::STAGES + 2 + a); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * CF::STAGES + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + CF::OFF_BAR + CF::NUM_BARS * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < CF::STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), CF::EPI_WARPS);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_map(&tmap_a);
+        tma_prefetch_map(&tmap_b);
+        if constexpr (TMA_STORE)
+            tma_prefetch_map(&tmap_c);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), CF::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint64_t timeout = p.timeout_ns;
+
+    // Last fill issued per stage (bit s set) and its phase parity: on an abort,
+    // every copy issued is waited for before the CTA exits.
+    uint32_t issued = 0, issued_parity = 0;
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool skip = p.inject_fault != 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+                int tm, tn;
+                tile_coords(t, p, tm, tn);
+                const int m0 = tm * CF::BM, n0 = tn * CF::BN;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, timeout, ERR_PRODUCER)) {
+                        ok = false;
+                        break;
+                    }
+                    if (skip) {
+                        skip = false;
+                    } else {
+                        const uint32_t fb = full_bar(stage);
+                        mbar_arrive_expect_tx(fb, CF::STAGE_BYTES);
+                        tma_load_2d(sA + stage * CF::A_STAGE_BYTES, &tmap_a, fb, kb * CF::BK, m0);
+#pragma unroll
+                        for (int j = 0; j < CF::BN / 64; ++j)
+                            tma_load_2d(sB + stage * CF::B_STAGE_BYTES + j * CF::B_BOX_BYTES, &tmap_b, fb,
+                                        n0 + 64 * j, kb * CF::BK);
+                        issued |= 1u << stage;
+                        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                    }
+                    if (++stage == CF::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC = mma_idesc_f16(DT, CF::BM, CF::BN, 0, 1);
+            // A: K-major, rows of 128 B, 8-row atoms 1024 B apart (SBO); LBO unused.
+            // B: N-major, 64-column boxes of BK rows (LBO = box bytes), 8-row atoms (SBO).
+            const uint64_t a_desc0 = smem_desc_sw128(sA, 16, 1024);
+            const uint64_t b_desc0 = smem_desc_sw128(sB, CF::B_BOX_BYTES, 1024);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+                if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, timeout, ERR_MMA_ACC)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * CF::ACC_COLS);
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!wait_bounded(full_bar(stage), phase, abort_flag, timeout, ERR_MMA_DATA)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint64_t a_desc = a_desc0 + ((stage * CF::A_STAGE_BYTES) >> 4);
+                    const uint64_t b_desc = b_desc0 + ((stage * CF::B_STAGE_BYTES) >> 4);
+#pragma unroll
+                    for (int k = 0; k < CF::BK / 16; ++k) {
+                        // K step of 16: +32 B inside A's swizzled row, +16 rows (2048 B) of B
+                        tc_mma_f16(d_tmem, a_desc + ((32 * k) >> 4), b_desc + ((2048 * k) >> 4), IDESC,
+                                   (kb | k) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(empty_bar(stage));
+                    if (++stage == CF::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                tc_commit(tfull_bar(acc));
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            // every MMA issued above completes before TMEM is released
+            tc_commit(drain_bar);
+            wait_drain(drain_bar, 0, timeout);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        int cbuf = 0;
+        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+            int tm, tn;
+            tile_coords(t, p, tm, tn);
+            const int m0 = tm * CF::BM, n0 = tn * CF::BN;
+            const int row0 = m0 + q * 32;  // first output row of this warp
+            if (!wait_bounded(tfull_bar(acc), acc_phase, abort_flag, timeout, ERR_EPILOGUE))
+                break;
+            tc_fence_after_sync();
+#pragma unroll 1
+            for (int c = 0; c < CF::BN / 64; ++c) {
+                uint32_t r[64];
+                const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(acc * CF::ACC_COLS + c * 64);
+                tmem_load_32cols(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+                tmem_load_32cols(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+                tmem_load_wait();
+                if (c == CF::BN / 64 - 1) {
+                    // accumulator fully read: hand it back to the MMA warp
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(tempty_bar(acc));
+                }
+                const int col0 = n0 + c * 64;
+                if (col0 >= p.N || row0 >= p.M)
+                    continue;  // nothing of this chunk lies inside C
+
+                float v[64];
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    v[j] = __uint_as_float(r[j]);
+                if constexpr (EPI == 1) {
+                    if (p.bias_vec16 && col0 + 64 <= p.N) {
+                        const uint4 *bp = reinterpret_cast<const uint4 *>(p.bias + col0);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const uint4 w = __ldg(bp + i);
+                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                v[8 * i + 2 * h] += to_float<DT>(static_cast<uint16_t>(ww[h] & 0xFFFFu));
+                                v[8 * i + 2 * h + 1] += to_float<DT>(static_cast<uint16_t>(ww[h] >> 16));
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j)
+                            if (col0 + j < p.N)
+                                v[j] += to_float<DT>(__ldg(p.bias + col0 + j));
+                    }
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        v[j] = gelu_erf(v[j]);
+                }
+                uint32_t packed[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    packed[j] = pack2<DT>(v[2 * j], v[2 * j + 1]);
+
+                if constexpr (TMA_STORE) {
+                    // staging buffer `cbuf` was last used two stores ago
+                    if (lane == 0)
+                        bulk_wait_group_read<1>();
+                    __syncwarp();
+                    uint8_t *buf = cstage + (q * 2 + cbuf) * CF::C_BOX_BYTES;
+                    // row `lane` of the 32x64 box; 16-byte chunk i lands at i ^ (lane & 7)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        uint4 w = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                        *reinterpret_cast<uint4 *>(buf + lane * 128 + ((i ^ (lane & 7)) << 4)) = w;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmap_c, smem_addr(buf), col0, row0);
+                        bulk_commit_group();
+                    }
+                    cbuf ^= 1;
+                } else {
+                    const int m = row0 + lane;
+                    if (m < p.M) {
+                        uint16_t *crow = p.C + static_cast<int64_t>(m) * p.ldc;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int n = col0 + 2 * j;
+                            if (n < p.N)
+                                crow[n] = static_cast<uint16_t>(packed[j] & 0xFFFFu);
+                            if (n + 1 < p.N)
+                                crow[n + 1] = static_cast<uint16_t>(packed[j] >> 16);
+                        }
+                    }
+                }
+            }
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if constexpr (TMA_STORE) {
+            if (lane == 0)
+                bulk_wait_group<0>();
+            __syncwarp();
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0 && lane == 0 && *abort_flag) {
+        // Some role gave up: copies it never consumed may still be landing.
+        for (int s = 0; s < CF::STAGES; ++s)
+            if (issued & (1u << s))
+                wait_drain(full_bar(s), (issued_parity >> s) & 1u, timeout);
+    }
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 1)
+        tmem_dealloc(tmem_base, CF::TMEM_COLS);
+}
+
+// Zero-padded copy of a rows x cols matrix of 16-bit values (any alignment of
+// `src`) into dst with a row length of dst_cols (a multiple of 8) and a
+// 16-byte-aligned base: each thread writes 8 values (16 bytes) at a time.
+__global__ void __launch_bounds__(256) pad_copy_kernel(const uint16_t *__restrict__ src, int64_t rows,
+                                                       int64_t cols, uint16_t *__restrict__ dst,
+                                                       int64_t dst_cols)
+{
+    const int64_t chunks_per_row = dst_cols >> 3;
+    const int64_t total = rows * chunks_per_row;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = idx / chunks_per_row;
+        const int64_t c0 = (idx - r * chunks_per_row) << 3;
+        const uint16_t *s = src + r * cols;
+        uint16_t e[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            e[i] = (c0 + i < cols) ? s[c0 + i] : static_cast<uint16_t>(0);
+        uint4 w;
+        w.x = e[0] | (static_cast<uint32_t>(e[1]) << 16);
+        w.y = e[2] | (static_cast<uint32_t>(e[3]) << 16);
+        w.z = e[4] | (static_cast<uint32_t>(e[5]) << 16);
+        w.w = e[6] | (static_cast<uint32_t>(e[7]) << 16);
+        *reinterpret_cast<uint4 *>(dst + r * dst_cols + c0) = w;
+    }
+}
+
+} // namespace tl

@@ -1,0 +1,468 @@
+// tl_gemm.cu -- host side of libtlgemm.so: argument validation, the launch
+// plan (kernel configuration, padding, store path), tensor-map encoding and
+// the launches.  The C ABI is declared in include/tl_gemm.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <unordered_map>
+
+#include "tl_gemm.h"
+#include "gemm_kernel.cuh"
+
+namespace tl {
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 10ull * 1000 * 1000 * 1000;
+
+using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
+
+struct ConfigEntry {
+    const char *name;
+    int bm, bn, bk, stages;
+    int smem_bytes;
+    KernelFn fn[2][2][2];  // [dtype][epilogue][tma_store]
+};
+
+template <class CF>
+ConfigEntry make_entry(const char *name)
+{
+    ConfigEntry e;
+    e.name = name;
+    e.bm = CF::BM;
+    e.bn = CF::BN;
+    e.bk = CF::BK;
+    e.stages = CF::STAGES;
+    e.smem_bytes = CF::SMEM_BYTES;
+    e.fn[0][0][0] = gemm_sm100_kernel<CF, 0, 0, false>;
+    e.fn[0][0][1] = gemm_sm100_kernel<CF, 0, 0, true>;
+    e.fn[0][1][0] = gemm_sm100_kernel<CF, 0, 1, false>;
+    e.fn[0][1][1] = gemm_sm100_kernel<CF, 0, 1, true>;
+    e.fn[1][0][0] = gemm_sm100_kernel<CF, 1, 0, false>;
+    e.fn[1][0][1] = gemm_sm100_kernel<CF, 1, 0, true>;
+    e.fn[1][1][0] = gemm_sm100_kernel<CF, 1, 1, false>;
+    e.fn[1][1][1] = gemm_sm100_kernel<CF, 1, 1, true>;
+    return e;
+}
+
+const ConfigEntry &config(int i);
+int num_configs();
+
+const ConfigEntry kConfigs[] = {
+    make_entry<TileConfig<256, 4>>("bm128_bn256_bk64_s4"),
+    make_entry<TileConfig<128, 6>>("bm128_bn128_bk64_s6"),
+    make_entry<TileConfig<64, 8>>("bm128_bn64_bk64_s8"),
+};
+
+int num_configs() { return static_cast<int>(sizeof(kConfigs) / sizeof(kConfigs[0])); }
+const ConfigEntry &config(int i) { return kConfigs[i]; }
+
+// Shapes measured by the offline sweep: (M, N, K, dtype, epilogue) -> config.
+struct TableRow {
+    int64_t m, n, k;
+    int dtype, epi;
+    const char *config;
+};
+const TableRow kTable[] = {
+#include "config_table.inc"
+};
+
+int config_index(const char *name)
+{
+    for (int i = 0; i < num_configs(); ++i)
+        if (std::strcmp(kConfigs[i].name, name) == 0)
+            return i;
+    return -1;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Model for shapes the sweep has not measured: time ~ waves x tile width,
+// with narrower tiles running the tensor pipe less efficiently (they read
+// more shared memory per MMA flop).
+int model_config(int64_t M, int64_t N, int num_sms)
+{
+    static const double eff[] = {1.0, 0.88, 0.6};
+    int best = 0;
+    double best_cost = 1e300;
+    for (int i = 0; i < num_configs(); ++i) {
+        const ConfigEntry &c = kConfigs[i];
+        const int64_t tiles = ceil_div(M, c.bm) * ceil_div(N, c.bn);
+        const double waves = static_cast<double>(ceil_div(tiles, num_sms));
+        const double cost = waves * c.bn / eff[i < 3 ? i : 2];
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = i;
+        }
+    }
+    return best;
+}
+
+int choose_config(int64_t M, int64_t N, int64_t K, int dtype, int epi, int num_sms)
+{
+    for (const TableRow &r : kTable) {
+        if (r.m == M && r.n == N && r.k == K && r.dtype == dtype && r.epi == epi) {
+            const int i = config_index(r.config);
+            if (i >= 0)
+                return i;
+        }
+    }
+    return model_config(M, N, num_sms);
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+struct Plan {
+    tl_plan pub;
+    int64_t lda, ldb;        // row lengths (elements) of the operands the kernel reads
+    int64_t a_ws_off, b_ws_off;
+};
+
+tl_status validate(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N,
+                   int64_t K, int dtype, int epi, const tl_gemm_options *opt)
+{
+    if (!A || !B || !C)
+        return TL_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0)
+        return TL_ERR_INVALID_ARG;
+    if (dtype != TL_F16 && dtype != TL_BF16)
+        return TL_ERR_INVALID_ARG;
+    if (epi != TL_EPI_NONE && epi != TL_EPI_BIAS_GELU)
+        return TL_ERR_INVALID_ARG;
+    if (epi == TL_EPI_BIAS_GELU && !bias)
+        return TL_ERR_INVALID_ARG;
+    if (opt && (opt->config < 0 || opt->config > num_configs()))
+        return TL_ERR_INVALID_ARG;
+    if (opt && (opt->inject_fault != 0 && opt->inject_fault != 1))
+        return TL_ERR_INVALID_ARG;
+    const int64_t lim = 0x7FFFFFFFll;
+    if (M > lim || N > lim || K > lim)
+        return TL_ERR_UNSUPPORTED;
+    if (!aligned(A, 2) || !aligned(B, 2) || !aligned(C, 2) || (epi == TL_EPI_BIAS_GELU && !aligned(bias, 2)))
+        return TL_ERR_MISALIGNED;
+    return TL_OK;
+}
+
+tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N,
+                    int64_t K, int dtype, int epi, int num_sms, const tl_gemm_options *opt, Plan *out)
+{
+    tl_status st = validate(A, B, bias, C, M, N, K, dtype, epi, opt);
+    if (st != TL_OK)
+        return st;
+    if (num_sms <= 0)
+        return TL_ERR_INVALID_ARG;
+    const int ci = (opt && opt->config > 0) ? opt->config - 1 : choose_config(M, N, K, dtype, epi, num_sms);
+    const ConfigEntry &c = kConfigs[ci];
+    Plan p{};
+    tl_plan &q = p.pub;
+    q.config = ci;
+    q.block_m = c.bm;
+    q.block_n = c.bn;
+    q.block_k = c.bk;
+    q.stages = c.stages;
+    q.tiles_m = static_cast<int32_t>(ceil_div(M, c.bm));
+    q.tiles_n = static_cast<int32_t>(ceil_div(N, c.bn));
+    const int64_t tiles = static_cast<int64_t>(q.tiles_m) * q.tiles_n;
+    if (tiles > 0x7FFFFFFFll)
+        return TL_ERR_UNSUPPORTED;
+    q.grid = static_cast<int32_t>(tiles < num_sms ? tiles : num_sms);
+    q.smem_bytes = c.smem_bytes;
+    // TMA needs a 16-byte-aligned base and row strides that are multiples of 16 bytes.
+    q.pad_a = !(aligned(A, 16) && K % 8 == 0);
+    q.pad_b = !(aligned(B, 16) && N % 8 == 0);
+    q.direct_store = !(aligned(C, 16) && N % 8 == 0);
+    p.lda = q.pad_a ? ceil_div(K, 8) * 8 : K;
+    p.ldb = q.pad_b ? ceil_div(N, 8) * 8 : N;
+    int64_t ws = 0;
+    p.a_ws_off = p.b_ws_off = -1;
+    if (q.pad_a) {
+        p.a_ws_off = ws;
+        ws += ceil_div(M * p.lda * 2, 256) * 256;
+    }
+    if (q.pad_b) {
+        p.b_ws_off = ws;
+        ws += ceil_div(K * p.ldb * 2, 256) * 256;
+    }
+    q.workspace_bytes = ws;
+    *out = p;
+    return TL_OK;
+}
+
+// ------------------------------------------------------------------ driver API
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiledFn>(nullptr);
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// 2-D row-major matrix of 16-bit values: `rows` x `cols`, row length `ld`;
+// box of box_cols (<= 64, 128 B) x box_rows, 128-byte swizzle.
+bool encode_2d(CUtensorMap *map, const void *base, int dtype, int64_t rows, int64_t cols, int64_t ld,
+               int box_cols, int box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType dt = dtype == TL_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ per-device state
+struct DeviceState {
+    int num_sms = 0;
+    int cc_major = 0;
+    cudaMemPool_t pool = nullptr;
+    std::unordered_map<const void *, bool> smem_set;  // kernels whose smem limit is raised
+};
+
+std::mutex g_mu;
+std::unordered_map<int, DeviceState> g_dev;
+
+tl_status device_state(DeviceState **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return TL_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState &d = g_dev[dev];
+    if (d.num_sms == 0) {
+        int sms = 0, major = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+            return TL_ERR_CUDA;
+        d.num_sms = sms;
+        d.cc_major = major;
+    }
+    *out = &d;
+    return TL_OK;
+}
+
+tl_status ensure_pool(DeviceState *d)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (d->pool)
+        return TL_OK;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return TL_ERR_CUDA;
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    if (cudaMemPoolCreate(&d->pool, &props) != cudaSuccess)
+        return TL_ERR_CUDA;
+    uint64_t keep = ~0ull;  // keep freed blocks for reuse by later calls
+    cudaMemPoolSetAttribute(d->pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    return TL_OK;
+}
+
+tl_status raise_smem_limit(DeviceState *d, KernelFn fn, int bytes)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = d->smem_set.find(reinterpret_cast<const void *>(fn));
+    if (it != d->smem_set.end())
+        return TL_OK;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return TL_ERR_CUDA;
+    d->smem_set[reinterpret_cast<const void *>(fn)] = true;
+    return TL_OK;
+}
+
+tl_status launch_pad(const void *src, int64_t rows, int64_t cols, void *dst, int64_t dst_cols, int num_sms,
+                     cudaStream_t stream)
+{
+    const int64_t work = rows * (dst_cols / 8);
+    int64_t blocks = ceil_div(work, 256);
+    const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+    if (blocks > cap)
+        blocks = cap;
+    if (blocks < 1)
+        blocks = 1;
+    pad_copy_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const uint16_t *>(src), rows, cols, static_cast<uint16_t *>(dst), dst_cols);
+    return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ERR_CUDA;
+}
+
+// Launch the GEMM itself with operands the kernel can read through TMA.
+tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *bias, void *C, int64_t M,
+                      int64_t N, int64_t K, int dtype, int epi, cudaStream_t stream, DeviceState *d,
+                      const tl_gemm_options *opt)
+{
+    const ConfigEntry &c = kConfigs[p.pub.config];
+    const bool tma_store = !p.pub.direct_store;
+    KernelFn fn = c.fn[dtype][epi][tma_store ? 1 : 0];
+    tl_status st = raise_smem_limit(d, fn, c.smem_bytes);
+    if (st != TL_OK)
+        return st;
+
+    CUtensorMap ta, tb, tc;
+    std::memset(&tc, 0, sizeof(tc));
+    if (!encode_2d(&ta, A, dtype, M, K, p.lda, 64, c.bm))
+        return TL_ERR_CUDA;
+    if (!encode_2d(&tb, B, dtype, K, N, p.ldb, 64, c.bk))
+        return TL_ERR_CUDA;
+    if (tma_store && !encode_2d(&tc, C, dtype, M, N, N, 64, 32))
+        return TL_ERR_CUDA;
+
+    GemmParams gp{};
+    gp.M = static_cast<int32_t>(M);
+    gp.N = static_cast<int32_t>(N);
+    gp.K = static_cast<int32_t>(K);
+    gp.tiles_m = p.pub.tiles_m;
+    gp.tiles_n = p.pub.tiles_n;
+    gp.num_tiles = p.pub.tiles_m * p.pub.tiles_n;
+    gp.num_kb = static_cast<int32_t>(ceil_div(K, c.bk));
+    gp.group_m = 8;
+    gp.bias = static_cast<const uint16_t *>(bias);
+    gp.bias_vec16 = bias && aligned(bias, 16);
+    gp.inject_fault = opt ? opt->inject_fault : 0;
+    gp.C = static_cast<uint16_t *>(C);
+    gp.ldc = N;
+    gp.timeout_ns = (opt && opt->timeout_ns) ? opt->timeout_ns : kDefaultTimeoutNs;
+
+    fn<<<p.pub.grid, 192, c.smem_bytes, stream>>>(ta, tb, tc, gp);
+    return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ERR_CUDA;
+}
+
+tl_status gemm_impl(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
+                    int dtype, int epi, cudaStream_t stream, const tl_gemm_options *opt)
+{
+    tl_status st = validate(A, B, bias, C, M, N, K, dtype, epi, opt);
+    if (st != TL_OK)
+        return st;
+    DeviceState *d = nullptr;
+    if ((st = device_state(&d)) != TL_OK)
+        return st;
+    if (d->cc_major != 10)
+        return TL_ERR_UNSUPPORTED;
+    Plan p;
+    if ((st = make_plan(A, B, bias, C, M, N, K, dtype, epi, d->num_sms, opt, &p)) != TL_OK)
+        return st;
+
+    if (p.pub.workspace_bytes == 0)
+        return launch_gemm(p, A, B, bias, C, M, N, K, dtype, epi, stream, d, opt);
+
+    if ((st = ensure_pool(d)) != TL_OK)
+        return st;
+    void *ws = nullptr;
+    if (cudaMallocFromPoolAsync(&ws, static_cast<size_t>(p.pub.workspace_bytes), d->pool, stream) != cudaSuccess)
+        return TL_ERR_CUDA;
+    const void *a_use = A, *b_use = B;
+    if (p.pub.pad_a) {
+        void *dst = static_cast<uint8_t *>(ws) + p.a_ws_off;
+        st = launch_pad(A, M, K, dst, p.lda, d->num_sms, stream);
+        a_use = dst;
+    }
+    if (st == TL_OK && p.pub.pad_b) {
+        void *dst = static_cast<uint8_t *>(ws) + p.b_ws_off;
+        st = launch_pad(B, K, N, dst, p.ldb, d->num_sms, stream);
+        b_use = dst;
+    }
+    if (st == TL_OK)
+        st = launch_gemm(p, a_use, b_use, bias, C, M, N, K, dtype, epi, stream, d, opt);
+    if (cudaFreeAsync(ws, stream) != cudaSuccess && st == TL_OK)
+        st = TL_ERR_CUDA;
+    return st;
+}
+
+} // namespace
+} // namespace tl
+
+extern "C" {
+
+tl_status tl_gemm(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
+                  tl_dtype dtype, tl_epilogue epi, tl_stream stream)
+{
+    return tl::gemm_impl(A, B, bias, C, M, N, K, dtype, epi, static_cast<cudaStream_t>(stream), nullptr);
+}
+
+tl_status tl_gemm_ex(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
+                     tl_dtype dtype, tl_epilogue epi, tl_stream stream, const tl_gemm_options *options)
+{
+    return tl::gemm_impl(A, B, bias, C, M, N, K, dtype, epi, static_cast<cudaStream_t>(stream), options);
+}
+
+tl_status tl_check_device(tl_stream stream, uint32_t *detail)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return TL_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, tl::g_device_error, sizeof(v)) != cudaSuccess)
+        return TL_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(tl::g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+        return TL_ERR_CUDA;
+    if (detail)
+        *detail = v;
+    return v ? TL_ERR_DEVICE_TIMEOUT : TL_OK;
+}
+
+tl_status tl_gemm_plan(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
+                       tl_dtype dtype, tl_epilogue epi, int32_t num_sms, const tl_gemm_options *options,
+                       tl_plan *plan)
+{
+    if (!plan)
+        return TL_ERR_INVALID_ARG;
+    tl_status st = tl::validate(A, B, bias, C, M, N, K, dtype, epi, options);
+    if (st != TL_OK)
+        return st;
+    if (num_sms <= 0) {
+        tl::DeviceState *d = nullptr;
+        if ((st = tl::device_state(&d)) != TL_OK)
+            return st;
+        num_sms = d->num_sms;
+    }
+    tl::Plan p;
+    st = tl::make_plan(A, B, bias, C, M, N, K, dtype, epi, num_sms, options, &p);
+    if (st == TL_OK)
+        *plan = p.pub;
+    return st;
+}
+
+int32_t tl_num_configs(void) { return tl::num_configs(); }
+
+const char *tl_config_name(int32_t i)
+{
+    if (i < 0 || i >= tl::num_configs())
+        return nullptr;
+    return tl::config(i).name;
+}
+
+const char *tl_status_string(tl_status s)
+{
+    switch (s) {
+    case TL_OK: return "TL_OK";
+    case TL_ERR_INVALID_ARG: return "TL_ERR_INVALID_ARG";
+    case TL_ERR_UNSUPPORTED: return "TL_ERR_UNSUPPORTED";
+    case TL_ERR_MISALIGNED: return "TL_ERR_MISALIGNED";
+    case TL_ERR_CUDA: return "TL_ERR_CUDA";
+    case TL_ERR_DEVICE_TIMEOUT: return "TL_ERR_DEVICE_TIMEOUT";
+    }
+    return "TL_ERR_UNKNOWN";
+}
+
+int32_t tl_version(void) { return TL_VERSION; }
+
+} // extern "C"

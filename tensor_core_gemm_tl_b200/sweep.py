@@ -1,0 +1,123 @@
+"""Offline tile/stage configuration sweep (needs a B200).
+
+For each shape, every compiled kernel configuration is timed through
+tl_gemm_ex on seeded inputs (rotating over input sets larger than L2, CUDA
+events, median of the launches after warm-up).  With --write, the fastest
+configuration per (M, N, K, dtype, epilogue) is written to
+csrc/config_table.inc, which the library compiles in; shapes not in the table
+use the library's wave model.  Nothing here runs at call time.
+
+    python -m tensor_core_gemm_tl_b200.sweep [--write] [--launches 50] [--shapes all|named]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+TABLE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc", "config_table.inc")
+L2_BYTES = 126 * 1024 * 1024
+
+
+def time_config(w, config, launches, warmup, seed=0):
+    import torch
+    import tensor_core_gemm_tl_b200 as tg
+    A_bits, B_bits, bias_bits = wl.make_inputs(w, seed)
+    tdt = torch.float16 if w.dtype == wl.F16 else torch.bfloat16
+
+    def dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).cuda().view(tdt)
+
+    A0, B0 = dev(A_bits), dev(B_bits)
+    bias = dev(bias_bits) if bias_bits is not None else None
+    set_bytes = 2 * (w.M * w.K + w.K * w.N + w.M * w.N)
+    nsets = max(2, int(np.ceil(3 * L2_BYTES / set_bytes)))
+    sets = [(A0 if i == 0 else A0.clone(), B0 if i == 0 else B0.clone(),
+             torch.empty((w.M, w.N), dtype=tdt, device="cuda")) for i in range(nsets)]
+    epi = "bias_gelu" if w.epi == wl.EPI_BIAS_GELU else None
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        A, B, C = sets[i % nsets]
+        tg.gemm(A, B, bias, epilogue=epi, out=C, config=config, stream=stream)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
+    for i, (s, e) in enumerate(ev):
+        A, B, C = sets[i % nsets]
+        s.record(stream)
+        tg.gemm(A, B, bias, epilogue=epi, out=C, config=config, stream=stream)
+        e.record(stream)
+    torch.cuda.synchronize()
+    if tg.check_device() != 0:
+        raise RuntimeError("device error")
+    ms = np.array([s.elapsed_time(e) for s, e in ev])
+    return float(np.median(ms)), float(ms.mean())
+
+
+def shapes(which):
+    named = list(wl.WORKLOADS.values())
+    if which == "named":
+        return named
+    extra = [wl.custom(f"square{n}_{d}", n, n, n, dt, 0) for n in (1024, 2048, 8192)
+             for d, dt in (("f16", wl.F16), ("bf16", wl.BF16))]
+    return named + extra
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--write", action="store_true")
+    ap.add_argument("--launches", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--shapes", default="named", choices=["named", "all"])
+    ap.add_argument("--only", default=None, help="comma-separated workload names")
+    a = ap.parse_args(argv)
+    import torch
+    import tensor_core_gemm_tl_b200 as tg
+    torch.cuda.set_device(0)
+    rows = []
+    todo = shapes(a.shapes)
+    if a.only:
+        keep = set(a.only.split(","))
+        todo = [w for w in todo if w.name in keep]
+    for w in todo:
+        best = None
+        for k in range(1, tg.tl_num_configs() + 1):
+            med, mean = time_config(w, k, a.launches, a.warmup)
+            tflops = w.flops / (med / 1e3) / 1e12
+            rec = {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "dtype": wl.DTYPE_NAMES[w.dtype],
+                   "epi": w.epi, "config": tg.tl_config_name(k - 1), "median_ms": round(med, 5),
+                   "mean_ms": round(mean, 5), "tflops": round(tflops, 1)}
+            print(json.dumps(rec), flush=True)
+            if best is None or med < best[0]:
+                best = (med, rec)
+        rows.append(best[1])
+    if a.write:
+        lines = ["// Kernel configuration per measured shape: {M, N, K, dtype, epilogue, config}.",
+                 "// Written by tensor_core_gemm_tl_b200/sweep.py from timings on a B200; shapes",
+                 "// not listed fall back to the wave model in tl_gemm.cu."]
+        seen = set()
+        for r in rows:
+            key = (r["M"], r["N"], r["K"], r["dtype"], r["epi"])
+            if key in seen:
+                continue
+            seen.add(key)
+            dt = 0 if r["dtype"] == "f16" else 1
+            lines.append(f'{{{r["M"]}, {r["N"]}, {r["K"]}, {dt}, {r["epi"]}, "{r["config"]}"}},'
+                         f'  // {r["tflops"]} TFLOP/s')
+        lines.append('{0, 0, 0, -1, -1, ""},  // sentinel, never matches')
+        with open(TABLE, "w") as f:
+            f.write("\n".join(lines) + "\n")
+        print("wrote", TABLE, file=sys.stderr)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,147 @@
+"""The C-ABI library on the CPU: it loads, exports every symbol the header
+declares, validates arguments before touching a GPU, and plans launches
+(configuration, grid, padding, store path) as documented."""
+import os
+import re
+
+import pytest
+
+import tensor_core_gemm_tl_b200 as tg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tl_gemm.h")
+P = 1 << 20  # a fake, 256-byte aligned "device pointer" (never dereferenced on the CPU)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"TL_API\s+[\w\s\*]+?\b(tl_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    assert {"tl_gemm", "tl_gemm_ex", "tl_check_device", "tl_gemm_plan", "tl_num_configs",
+            "tl_config_name", "tl_status_string", "tl_version"} <= set(names)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = tg._binding._lib
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in tg.SIGNATURES, f"binding lacks {name}"
+
+
+def test_version_and_strings():
+    assert tg.tl_version() == 1000
+    for s in tg.Status:
+        assert tg.tl_status_string(int(s)) == "TL_" + ("OK" if s.name == "OK" else "ERR_" + s.name)
+    assert tg.tl_status_string(99) == "TL_ERR_UNKNOWN"
+    n = tg.tl_num_configs()
+    assert n >= 3
+    names = tg.configs()
+    assert all(re.fullmatch(r"bm\d+_bn\d+_bk\d+_s\d+", x) for x in names)
+    assert tg.tl_config_name(n) is None and tg.tl_config_name(-1) is None
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(A=0), tg.Status.INVALID_ARG),
+    (dict(B=0), tg.Status.INVALID_ARG),
+    (dict(C=0), tg.Status.INVALID_ARG),
+    (dict(M=0), tg.Status.INVALID_ARG),
+    (dict(N=-1), tg.Status.INVALID_ARG),
+    (dict(K=0), tg.Status.INVALID_ARG),
+    (dict(dtype=2), tg.Status.INVALID_ARG),
+    (dict(epi=7), tg.Status.INVALID_ARG),
+    (dict(epi=1, bias=0), tg.Status.INVALID_ARG),
+    (dict(M=1 << 31), tg.Status.UNSUPPORTED),
+    (dict(K=1 << 40), tg.Status.UNSUPPORTED),
+    (dict(A=P + 1), tg.Status.MISALIGNED),
+    (dict(C=P + 3), tg.Status.MISALIGNED),
+    (dict(epi=1, bias=P + 1), tg.Status.MISALIGNED),
+])
+def test_validation_before_any_cuda_call(args, status):
+    a = dict(A=P, B=P, bias=0, C=P, M=64, N=64, K=64, dtype=0, epi=0)
+    a.update(args)
+    st = tg.tl_gemm(a["A"], a["B"], a["bias"], a["C"], a["M"], a["N"], a["K"], a["dtype"], a["epi"], 0)
+    assert st == status
+    st2, _ = tg.tl_gemm_plan(a["A"], a["B"], a["bias"], a["C"], a["M"], a["N"], a["K"], a["dtype"],
+                             a["epi"], 148)
+    assert st2 == status
+
+
+def test_options_validation():
+    bad = tg.Options(config=tg.tl_num_configs() + 1)
+    assert tg.tl_gemm_ex(P, P, 0, P, 8, 8, 8, 0, 0, 0, bad) == tg.Status.INVALID_ARG
+    bad = tg.Options(config=-1)
+    assert tg.tl_gemm_ex(P, P, 0, P, 8, 8, 8, 0, 0, 0, bad) == tg.Status.INVALID_ARG
+    bad = tg.Options(inject_fault=3)
+    assert tg.tl_gemm_ex(P, P, 0, P, 8, 8, 8, 0, 0, 0, bad) == tg.Status.INVALID_ARG
+
+
+@pytest.mark.skipif(os.environ.get("CUDA_VISIBLE_DEVICES") is None and __import__("torch").cuda.is_available(),
+                    reason="only meaningful without a GPU")
+def test_no_device_is_a_cuda_error_not_a_crash():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert tg.tl_gemm(P, P, 0, P, 64, 64, 64, 0, 0, 0) == tg.Status.CUDA
+
+
+def test_plan_aligned_headline_shape():
+    p = tg.plan(4096, 4096, 4096, tg.TL_F16, None, num_sms=148)
+    assert p["pad_a"] == 0 and p["pad_b"] == 0 and p["direct_store"] == 0
+    assert p["workspace_bytes"] == 0
+    assert p["tiles_m"] == 4096 // p["block_m"] and p["tiles_n"] == 4096 // p["block_n"]
+    assert p["grid"] == min(148, p["tiles_m"] * p["tiles_n"])
+    assert p["smem_bytes"] <= 232448
+
+
+def test_plan_grid_never_exceeds_tiles():
+    p = tg.plan(100, 60, 30, tg.TL_BF16, None, num_sms=148)
+    assert p["tiles_m"] == 1 and p["tiles_n"] == 1 and p["grid"] == 1
+
+
+def test_plan_unaligned_k_pads_A_only():
+    M, N, K = 4000, 3000, 2050
+    p = tg.plan(M, N, K, tg.TL_BF16, "bias_gelu", num_sms=148)
+    assert p["pad_a"] == 1 and p["pad_b"] == 0 and p["direct_store"] == 0
+    assert p["workspace_bytes"] == ((M * 2056 * 2 + 255) // 256) * 256
+
+
+def test_plan_unaligned_n_pads_B_and_stores_directly():
+    M, N, K = 300, 1001, 64
+    p = tg.plan(M, N, K, tg.TL_F16, None, num_sms=148)
+    assert p["pad_a"] == 0 and p["pad_b"] == 1 and p["direct_store"] == 1
+    assert p["workspace_bytes"] == ((K * 1008 * 2 + 255) // 256) * 256
+
+
+def test_plan_misaligned_bases():
+    # 2-byte aligned but not 16-byte aligned bases take the padded / direct paths
+    p = tg.plan(256, 256, 256, tg.TL_F16, None, num_sms=148, ptrs=(P + 2, P + 6, 0, P + 8))
+    assert p["pad_a"] == 1 and p["pad_b"] == 1 and p["direct_store"] == 1
+
+
+def test_plan_forced_config():
+    for k in range(1, tg.tl_num_configs() + 1):
+        p = tg.plan(4096, 4096, 4096, tg.TL_F16, None, num_sms=148, config=k)
+        assert p["config"] == k - 1
+        assert p["config_name"] == tg.tl_config_name(k - 1)
+
+
+def test_plan_skinny_prefers_narrow_tiles():
+    # 128 x 16384: a 128 x 256 tiling leaves most of 148 SMs idle
+    wide = tg.plan(128, 16384, 4096, tg.TL_BF16, None, num_sms=148, config=1)
+    chosen = tg.plan(128, 16384, 4096, tg.TL_BF16, None, num_sms=148)
+    assert wide["tiles_m"] * wide["tiles_n"] < 148
+    assert chosen["tiles_m"] * chosen["tiles_n"] > wide["tiles_m"] * wide["tiles_n"]
+
+
+def test_torch_wrapper_rejects_bad_tensors():
+    import torch
+    A = torch.zeros(4, 4, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        tg.gemm(A, A)  # CPU tensors
+    with pytest.raises(ValueError):
+        tg.gemm(A, torch.zeros(5, 4, dtype=torch.float16))
+    with pytest.raises(ValueError):
+        tg._epi_code("relu")

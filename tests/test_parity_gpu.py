@@ -1,0 +1,196 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs.  Bar: relative Frobenius error <= 2e-3 and
+|C - ref| <= 1e-2 |ref| + 1e-2 elementwise; on the small cases also at most
+the fp32-accumulation error bound plus half an ulp of the output type."""
+import os
+import sys
+
+import numpy as np
+import pytest
+
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+import oracle  # noqa: E402
+import workloads as wl  # noqa: E402
+from gpu_util import accumulation_bound, compare, run_library, to_device  # noqa: E402
+
+torch = pytest.importorskip("torch")
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+
+def tg():
+    import tensor_core_gemm_tl_b200 as m
+    return m
+
+
+def n_configs():
+    return tg().tl_num_configs()
+
+
+def inputs(M, N, K, dt, epi, seed=0):
+    w = wl.custom("t", M, N, K, dt, epi)
+    return wl.make_inputs(w, seed)
+
+
+# ------------------------------------------------------------------ layout probes
+@pytest.mark.parametrize("config", [1, 2, 3])
+@pytest.mark.parametrize("dt", [wl.F16, wl.BF16])
+def test_layout_probe_one_hot(config, dt):
+    """A has one 1 per row (row i picks k(i)); B[k, j] encodes (k, j) as a small
+    integer, so C[i, j] must equal B[k(i), j] exactly: any swizzle, descriptor
+    or TMEM lane/column mistake shows as a wrong code."""
+    M, N, K = 384, 320, 192
+    kk = (np.arange(M) * 37 + 5) % K
+    A = np.zeros((M, K), np.float32)
+    A[np.arange(M), kk] = 1.0
+    if dt == wl.F16:
+        code = (np.arange(K)[:, None] % 32) * 32 + (np.arange(N)[None, :] % 32)
+    else:
+        code = (np.arange(K)[:, None] % 16) * 16 + (np.arange(N)[None, :] % 16)
+    Ab = wl.round_to_bits(A, dt)
+    Bb = wl.round_to_bits(code.astype(np.float32), dt)
+    C = run_library(Ab, Bb, None, dt, wl.EPI_NONE, config=config)
+    got = wl.bits_to_float32(C, dt)
+    assert np.array_equal(got, code[kk, :].astype(np.float32))
+
+
+@pytest.mark.parametrize("config", [1, 2, 3])
+def test_identity_gives_B(config):
+    n, N = 256, 384
+    A = wl.round_to_bits(np.eye(n, dtype=np.float32), wl.BF16)
+    _, B, _ = inputs(n, N, n, wl.BF16, 0, seed=3)
+    C = run_library(A, B, None, wl.BF16, wl.EPI_NONE, config=config)
+    assert np.array_equal(C, B)
+
+
+# ------------------------------------------------------------------ small shapes vs the oracle
+SHAPES = [
+    (128, 256, 64),      # one tile, one k block
+    (256, 512, 256),     # several tiles, several k blocks
+    (300, 520, 200),     # ragged M, N, K tails
+    (1, 1, 1),
+    (15, 16, 63),
+    (16, 63, 64),
+    (63, 64, 65),
+    (65, 127, 128),
+    (127, 129, 255),
+    (129, 255, 257),
+    (257, 8, 16),
+    (8, 257, 129),
+    (1000, 24, 8),
+]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+@pytest.mark.parametrize("dt", [wl.F16, wl.BF16])
+@pytest.mark.parametrize("epi", [wl.EPI_NONE, wl.EPI_BIAS_GELU])
+def test_small_shapes_vs_oracle(M, N, K, dt, epi):
+    A, B, bias = inputs(M, N, K, dt, epi, seed=M * 7 + N * 3 + K)
+    ref = oracle.gemm(A, B, bias, dt, epi)
+    C = run_library(A, B, bias, dt, epi)
+    compare(C, ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
+
+
+@pytest.mark.parametrize("config", [1, 2, 3])
+@pytest.mark.parametrize("epi", [wl.EPI_NONE, wl.EPI_BIAS_GELU])
+def test_every_config_vs_oracle(config, epi):
+    M, N, K = 700, 900, 333
+    for dt in (wl.F16, wl.BF16):
+        A, B, bias = inputs(M, N, K, dt, epi, seed=config)
+        ref = oracle.gemm(A, B, bias, dt, epi)
+        C = run_library(A, B, bias, dt, epi, config=config)
+        compare(C, ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
+
+
+@pytest.mark.parametrize("offsets", [(1, 0, 0, 0), (0, 3, 0, 0), (0, 0, 1, 0), (0, 0, 0, 5), (2, 1, 3, 7)])
+def test_unaligned_bases(offsets):
+    """Bases 2-byte but not 16-byte aligned: padded operand copies, the scalar
+    bias path and the element-by-element store."""
+    M, N, K = 200, 264, 136
+    dt, epi = wl.BF16, wl.EPI_BIAS_GELU
+    A, B, bias = inputs(M, N, K, dt, epi, seed=sum(offsets))
+    ref = oracle.gemm(A, B, bias, dt, epi)
+    C = run_library(A, B, bias, dt, epi, offsets=offsets)
+    compare(C, ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
+
+
+def test_deterministic_bitwise():
+    M, N, K = 1024, 768, 1000
+    A, B, bias = inputs(M, N, K, wl.BF16, wl.EPI_BIAS_GELU, seed=42)
+    c1 = run_library(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU)
+    c2 = run_library(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU)
+    assert np.array_equal(c1, c2)
+
+
+def test_epilogue_matches_plain_plus_gelu_structure():
+    """Fused result vs the oracle's epilogue applied to the oracle's plain
+    product -- and the plain path from the same call site."""
+    M, N, K = 256, 384, 512
+    dt = wl.F16
+    A, B, bias = inputs(M, N, K, dt, wl.EPI_BIAS_GELU, seed=9)
+    plain = run_library(A, B, None, dt, wl.EPI_NONE)
+    fused = run_library(A, B, bias, dt, wl.EPI_BIAS_GELU)
+    rp = oracle.gemm(A, B, None, dt, wl.EPI_NONE)
+    rf = oracle.gemm(A, B, bias, dt, wl.EPI_BIAS_GELU)
+    compare(plain, rp, dt, accumulation_bound(A, B, None, dt, wl.EPI_NONE, rp))
+    compare(fused, rf, dt, accumulation_bound(A, B, bias, dt, wl.EPI_BIAS_GELU, rf))
+
+
+# ------------------------------------------------------------------ the named workloads
+def _sample_rows(M, n, rng):
+    rows = {0, M - 1, M // 2}
+    for t in (127, 128, 129, 255, 256):
+        if t < M:
+            rows.add(t)
+    rows.update(int(r) for r in rng.integers(0, M, n))
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("name", list(wl.WORKLOADS))
+def test_workload_sampled_vs_oracle(name):
+    """Every named workload at full size in the launch configuration the
+    benchmark times (the library's choice): whole rows of C sampled and
+    compared with the oracle's rows (the 256^3 case in full)."""
+    w = wl.WORKLOADS[name]
+    A, B, bias = wl.make_inputs(w, 0)
+    C = run_library(A, B, bias, w.dtype, w.epi)
+    if w.M * w.N * w.K <= 1 << 28:
+        ref = oracle.gemm(A, B, bias, w.dtype, w.epi)
+        compare(C, ref, w.dtype, accumulation_bound(A, B, bias, w.dtype, w.epi, ref))
+        return
+    rng = np.random.default_rng(1)
+    budget_rows = max(8, int(4e9 // (2 * w.N * w.K)))
+    rows = _sample_rows(w.M, min(48, budget_rows), rng)
+    ref = oracle.gemm(A, B, bias, w.dtype, w.epi, rows=rows)
+    compare(C[rows], ref, w.dtype, accumulation_bound(A, B, bias, w.dtype, w.epi, ref, rows=rows))
+    # and scattered single elements over the whole of C
+    ii = rng.integers(0, w.M, 2000)
+    jj = rng.integers(0, w.N, 2000)
+    refp = oracle.gemm_points(A, B, bias, w.dtype, w.epi, ii, jj)
+    compare(C[ii, jj], refp, w.dtype, accumulation_bound(A, B, bias, w.dtype, w.epi, refp, points=(ii, jj)))
+
+
+# ------------------------------------------------------------------ failure detection
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """The copy warp skips its first stage without issuing the copy: the MMA
+    warp's bounded wait runs out, the kernel records it and returns.  The
+    status is read on the host; the next call on the same context is right."""
+    import tensor_core_gemm_tl_b200 as m
+    M, N, K = 256, 256, 256
+    A, B, bias = inputs(M, N, K, wl.F16, 0, seed=5)
+    dA, dB = to_device(A, wl.F16), to_device(B, wl.F16)
+    out = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    opt = m.Options(config=0, inject_fault=1, timeout_ns=200_000_000)
+    st = m.tl_gemm_ex(dA.data_ptr(), dB.data_ptr(), 0, out.data_ptr(), M, N, K, wl.F16, 0,
+                      torch.cuda.current_stream().cuda_stream, opt)
+    assert st == 0
+    st, word = m.tl_check_device(torch.cuda.current_stream().cuda_stream)
+    assert st == int(m.Status.DEVICE_TIMEOUT)
+    assert word & 2  # the MMA warp's wait on data gave up
+    assert not (word & 16)  # and every issued copy / MMA drained in time
+    st, word = m.tl_check_device(torch.cuda.current_stream().cuda_stream)
+    assert st == 0 and word == 0  # the word was cleared
+    C = run_library(A, B, None, wl.F16, 0)
+    ref = oracle.gemm(A, B, None, wl.F16, 0)
+    compare(C, ref, wl.F16, accumulation_bound(A, B, None, wl.F16, 0, ref))

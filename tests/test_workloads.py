@@ -62,3 +62,16 @@ def test_table_of_workloads():
             (16384, 1024, 8192), (128, 16384, 4096)} <= shapes
     for w in wl.WORKLOADS.values():
         assert w.flops == 2 * w.M * w.N * w.K
+
+
+def test_test_side_rounding_matches_torch():
+    """The tests' fp64 -> fp16/bf16 rounding (used for ulp diagnostics) agrees
+    with torch's casts on float32-representable inputs."""
+    import sys, os
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    from gpu_util import round_to_dtype
+    x = _ties_and_randoms(np.random.default_rng(3), 4000)
+    x = x[np.abs(x) < 60000]
+    for dt, tdt in ((wl.F16, torch.float16), (wl.BF16, torch.bfloat16)):
+        ref = torch.from_numpy(x).to(tdt).double().numpy()
+        assert np.array_equal(round_to_dtype(x.astype(np.float64), dt), ref)
