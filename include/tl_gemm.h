@@ -132,7 +132,9 @@ typedef struct {
     int32_t config;          /* kernel configuration index                     */
     int32_t block_m, block_n, block_k, stages;
     int32_t tiles_m, tiles_n;
-    int32_t grid;            /* persistent CTAs launched                       */
+    int32_t grid;            /* persistent CTAs launched (the launch may lower it
+                                to the number of CTA pairs that fit at once)   */
+    int32_t cluster_ctas;    /* 1, or 2 when pairs of CTAs share each tile     */
     int32_t pad_a, pad_b;    /* 1 when the operand is first copied to a padded temporary */
     int32_t direct_store;    /* 1 when C is stored element by element          */
     int32_t smem_bytes;      /* dynamic shared memory per CTA                  */

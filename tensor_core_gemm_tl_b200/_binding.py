@@ -43,7 +43,8 @@ class Plan(ctypes.Structure):
     """tl_plan: the host-side decision for one call."""
     _fields_ = [("config", ctypes.c_int32), ("block_m", ctypes.c_int32), ("block_n", ctypes.c_int32),
                 ("block_k", ctypes.c_int32), ("stages", ctypes.c_int32), ("tiles_m", ctypes.c_int32),
-                ("tiles_n", ctypes.c_int32), ("grid", ctypes.c_int32), ("pad_a", ctypes.c_int32),
+                ("tiles_n", ctypes.c_int32), ("grid", ctypes.c_int32), ("cluster_ctas", ctypes.c_int32),
+                ("pad_a", ctypes.c_int32),
                 ("pad_b", ctypes.c_int32), ("direct_store", ctypes.c_int32),
                 ("smem_bytes", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64)]
 

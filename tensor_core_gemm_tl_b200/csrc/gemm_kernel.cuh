@@ -59,15 +59,25 @@ struct GemmParams {
     uint64_t timeout_ns;
 };
 
-// Compile-time tile configuration.  BM = 128 rows (one TMEM lane per row),
-// BK = 64 (one 128-byte swizzle row of 16-bit values), BN in {64, 128, 256}.
-template <int BN_, int STAGES_>
+// Compile-time tile configuration.  Each CTA owns BM = 128 output rows (one
+// TMEM lane per row) and BK = 64 (one 128-byte swizzle row of 16-bit values).
+// PAIR = false: one CTA computes a 128 x BN tile with cta_group::1 MMAs.
+// PAIR = true:  a cluster of two CTAs computes a 256 x BN tile with
+//               cta_group::2 MMAs issued by the even CTA; each CTA loads its
+//               own 128 rows of A and its own BN/2 columns of B, and holds its
+//               128 rows of the accumulator in its own TMEM.
+template <int BN_, int STAGES_, bool PAIR_ = false>
 struct TileConfig {
+    static constexpr bool PAIR = PAIR_;
+    static constexpr int CTAS = PAIR ? 2 : 1;
     static constexpr int BM = 128, BN = BN_, BK = 64, STAGES = STAGES_;
+    static constexpr int TILE_M = BM * CTAS;       // output rows per tile
+    static constexpr int BN_LOCAL = BN / CTAS;     // B columns this CTA loads
     static constexpr int A_STAGE_BYTES = BM * BK * 2;
     static constexpr int B_BOX_BYTES = BK * 128;   // one 64-column box of B
-    static constexpr int B_STAGE_BYTES = BK * BN * 2;
+    static constexpr int B_STAGE_BYTES = BK * BN_LOCAL * 2;
     static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+    static constexpr int TX_BYTES = STAGE_BYTES * CTAS;  // landing on the (even CTA's) full barrier
     static constexpr int EPI_WARPS = 4;
     static constexpr int C_BOX_BYTES = 32 * 128;   // 32 rows x 64 columns of 16-bit
     static constexpr int C_STAGING_BYTES = EPI_WARPS * 2 * C_BOX_BYTES;
@@ -81,7 +91,7 @@ struct TileConfig {
     static constexpr int SMEM_USED = OFF_BAR + NUM_BARS * 8 + 16;
     static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024
     static constexpr int THREADS = 192;
-    static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+    static_assert(BN_LOCAL % 64 == 0 && BN >= 64 && BN <= 256, "BN");
     static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM columns");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -100,20 +110,27 @@ __device__ __forceinline__ void tile_coords(int t, const GemmParams &p, int &tm,
 }
 
 // Bounded wait.  Returns false when the abort flag is raised by another role
-// or when this wait runs past timeout_ns (then it raises the flag itself).
+// (or by the peer CTA) or when this wait runs past timeout_ns; then it raises
+// the flag itself, and the peer's too when `peer_abort` (a shared::cluster
+// address) is non-zero.  CLUSTER_SCOPE acquires at cluster scope, for
+// barriers the peer CTA arrives on.
+template <bool CLUSTER_SCOPE = false>
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                             uint64_t timeout_ns, unsigned code)
+                                             uint64_t timeout_ns, unsigned code, uint32_t peer_abort = 0)
 {
-    if (mbar_try_wait(bar, parity))
+    auto test = [&]() { return CLUSTER_SCOPE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+    if (test())
         return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity))
+        if (test())
             return true;
         if (*abort_flag)
             return false;
         if (global_timer_ns() - t0 > timeout_ns) {
             *abort_flag = 1;
+            if (peer_abort)
+                st_shared_cluster_u32(peer_abort, 1u);
             atomicOr(&g_device_error, code);
             return false;
         }
@@ -168,11 +185,16 @@ __global__ void __launch_bounds__(192, 1)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_c, const GemmParams p)
 {
+    constexpr bool PAIR = CF::PAIR;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0: the CTA that issues the MMAs
+    const bool leader = rank == 0;
+    const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int num_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
     const uint32_t sA = smem_addr(smem + CF::OFF_A);
     const uint32_t sB = smem_addr(smem + CF::OFF_B);
@@ -186,6 +208,7 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t drain_bar = bar0 + 8u * (2 * CF::STAGES + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + CF::OFF_BAR + CF::NUM_BARS * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const uint32_t peer_abort = PAIR ? mapa_shared(smem_addr(tmem_slot + 1), rank ^ 1u) : 0u;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < CF::STAGES; ++s) {
@@ -194,7 +217,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar(a), 1);
-            mbar_init(tempty_bar(a), CF::EPI_WARPS);
+            mbar_init(tempty_bar(a), CF::EPI_WARPS * CF::CTAS);
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -208,11 +231,19 @@ __global__ void __launch_bounds__(192, 1)
             tma_prefetch_map(&tmap_c);
     }
     if (warp == 1) {
-        tmem_alloc(smem_addr(tmem_slot), CF::TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(smem_addr(tmem_slot), CF::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_addr(tmem_slot), CF::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before_sync();
-    __syncthreads();
+    if constexpr (PAIR)
+        cluster_sync();  // both CTAs' barriers and TMEM exist before any cross-CTA use
+    else
+        __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
     const uint64_t timeout = p.timeout_ns;
@@ -225,14 +256,16 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            bool skip = p.inject_fault != 0;
+            bool skip = p.inject_fault != 0 && leader;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+            for (int t = unit; ok && t < p.num_tiles; t += num_units) {
                 int tm, tn;
                 tile_coords(t, p, tm, tn);
-                const int m0 = tm * CF::BM, n0 = tn * CF::BN;
+                const int a_row = tm * CF::TILE_M + static_cast<int>(rank) * CF::BM;
+                const int b_col = tn * CF::BN + static_cast<int>(rank) * CF::BN_LOCAL;
                 for (int kb = 0; kb < p.num_kb; ++kb) {
-                    if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, timeout, ERR_PRODUCER)) {
+                    if (!wait_bounded<PAIR>(empty_bar(stage), phase ^ 1u, abort_flag, timeout, ERR_PRODUCER,
+                                            peer_abort)) {
                         ok = false;
                         break;
                     }
@@ -240,12 +273,25 @@ __global__ void __launch_bounds__(192, 1)
                         skip = false;
                     } else {
                         const uint32_t fb = full_bar(stage);
-                        mbar_arrive_expect_tx(fb, CF::STAGE_BYTES);
-                        tma_load_2d(sA + stage * CF::A_STAGE_BYTES, &tmap_a, fb, kb * CF::BK, m0);
+                        const uint32_t sa = sA + stage * CF::A_STAGE_BYTES;
+                        const uint32_t sb = sB + stage * CF::B_STAGE_BYTES;
+                        if constexpr (PAIR) {
+                            // both CTAs' bytes complete on the even CTA's barrier
+                            const uint32_t fb0 = mapa_shared(fb, 0);
+                            if (leader)
+                                mbar_arrive_expect_tx(fb, CF::TX_BYTES);
+                            tma_load_2d_pair(sa, &tmap_a, fb0, kb * CF::BK, a_row);
 #pragma unroll
-                        for (int j = 0; j < CF::BN / 64; ++j)
-                            tma_load_2d(sB + stage * CF::B_STAGE_BYTES + j * CF::B_BOX_BYTES, &tmap_b, fb,
-                                        n0 + 64 * j, kb * CF::BK);
+                            for (int j = 0; j < CF::BN_LOCAL / 64; ++j)
+                                tma_load_2d_pair(sb + j * CF::B_BOX_BYTES, &tmap_b, fb0, b_col + 64 * j,
+                                                 kb * CF::BK);
+                        } else {
+                            mbar_arrive_expect_tx(fb, CF::TX_BYTES);
+                            tma_load_2d(sa, &tmap_a, fb, kb * CF::BK, a_row);
+#pragma unroll
+                            for (int j = 0; j < CF::BN_LOCAL / 64; ++j)
+                                tma_load_2d(sb + j * CF::B_BOX_BYTES, &tmap_b, fb, b_col + 64 * j, kb * CF::BK);
+                        }
                         issued |= 1u << stage;
                         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                     }
@@ -258,9 +304,9 @@ __global__ void __launch_bounds__(192, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t IDESC = mma_idesc_f16(DT, CF::BM, CF::BN, 0, 1);
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (lane == 0 && leader) {
+            constexpr uint32_t IDESC = mma_idesc_f16(DT, CF::TILE_M, CF::BN, 0, 1);
             // A: K-major, rows of 128 B, 8-row atoms 1024 B apart (SBO); LBO unused.
             // B: N-major, 64-column boxes of BK rows (LBO = box bytes), 8-row atoms (SBO).
             const uint64_t a_desc0 = smem_desc_sw128(sA, 16, 1024);
@@ -270,15 +316,16 @@ __global__ void __launch_bounds__(192, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
-                if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, timeout, ERR_MMA_ACC)) {
+            for (int t = unit; ok && t < p.num_tiles; t += num_units) {
+                if (!wait_bounded<PAIR>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, timeout, ERR_MMA_ACC,
+                                        peer_abort)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * CF::ACC_COLS);
                 for (int kb = 0; kb < p.num_kb; ++kb) {
-                    if (!wait_bounded(full_bar(stage), phase, abort_flag, timeout, ERR_MMA_DATA)) {
+                    if (!wait_bounded(full_bar(stage), phase, abort_flag, timeout, ERR_MMA_DATA, peer_abort)) {
                         ok = false;
                         break;
                     }
@@ -288,10 +335,17 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                     for (int k = 0; k < CF::BK / 16; ++k) {
                         // K step of 16: +32 B inside A's swizzled row, +16 rows (2048 B) of B
-                        tc_mma_f16(d_tmem, a_desc + ((32 * k) >> 4), b_desc + ((2048 * k) >> 4), IDESC,
-                                   (kb | k) != 0 ? 1u : 0u);
+                        const uint64_t ad = a_desc + ((32 * k) >> 4), bd = b_desc + ((2048 * k) >> 4);
+                        const uint32_t accumulate = (kb | k) != 0 ? 1u : 0u;
+                        if constexpr (PAIR)
+                            tc_mma_f16_pair(d_tmem, ad, bd, IDESC, accumulate);
+                        else
+                            tc_mma_f16(d_tmem, ad, bd, IDESC, accumulate);
                     }
-                    tc_commit(empty_bar(stage));
+                    if constexpr (PAIR)
+                        tc_commit_pair_mc(empty_bar(stage), 0x3);
+                    else
+                        tc_commit(empty_bar(stage));
                     if (++stage == CF::STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -299,14 +353,20 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 if (!ok)
                     break;
-                tc_commit(tfull_bar(acc));
+                if constexpr (PAIR)
+                    tc_commit_pair_mc(tfull_bar(acc), 0x3);
+                else
+                    tc_commit(tfull_bar(acc));
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1u;
                 }
             }
             // every MMA issued above completes before TMEM is released
-            tc_commit(drain_bar);
+            if constexpr (PAIR)
+                tc_commit_pair_mc(drain_bar, 0x1);
+            else
+                tc_commit(drain_bar);
             wait_drain(drain_bar, 0, timeout);
         }
         __syncwarp();
@@ -317,12 +377,12 @@ __global__ void __launch_bounds__(192, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         int cbuf = 0;
-        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+        for (int t = unit; t < p.num_tiles; t += num_units) {
             int tm, tn;
             tile_coords(t, p, tm, tn);
-            const int m0 = tm * CF::BM, n0 = tn * CF::BN;
-            const int row0 = m0 + q * 32;  // first output row of this warp
-            if (!wait_bounded(tfull_bar(acc), acc_phase, abort_flag, timeout, ERR_EPILOGUE))
+            const int n0 = tn * CF::BN;
+            const int row0 = tm * CF::TILE_M + static_cast<int>(rank) * CF::BM + q * 32;  // this warp's rows
+            if (!wait_bounded<PAIR>(tfull_bar(acc), acc_phase, abort_flag, timeout, ERR_EPILOGUE, peer_abort))
                 break;
             tc_fence_after_sync();
 #pragma unroll 1
@@ -336,57 +396,84 @@ __global__ void __launch_bounds__(192, 1)
                     // accumulator fully read: hand it back to the MMA warp
                     tc_fence_before_sync();
                     __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(tempty_bar(acc));
+                    if (lane == 0) {
+                        if constexpr (PAIR)
+                            mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+                        else
+                            mbar_arrive(tempty_bar(acc));
+                    }
                 }
                 const int col0 = n0 + c * 64;
                 if (col0 >= p.N || row0 >= p.M)
                     continue;  // nothing of this chunk lies inside C
 
-                float v[64];
-#pragma unroll
-                for (int j = 0; j < 64; ++j)
-                    v[j] = __uint_as_float(r[j]);
-                if constexpr (EPI == 1) {
-                    if (p.bias_vec16 && col0 + 64 <= p.N) {
-                        const uint4 *bp = reinterpret_cast<const uint4 *>(p.bias + col0);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const uint4 w = __ldg(bp + i);
-                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int h = 0; h < 4; ++h) {
-                                v[8 * i + 2 * h] += to_float<DT>(static_cast<uint16_t>(ww[h] & 0xFFFFu));
-                                v[8 * i + 2 * h + 1] += to_float<DT>(static_cast<uint16_t>(ww[h] >> 16));
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 64; ++j)
-                            if (col0 + j < p.N)
-                                v[j] += to_float<DT>(__ldg(p.bias + col0 + j));
-                    }
-#pragma unroll
-                    for (int j = 0; j < 64; ++j)
-                        v[j] = gelu_erf(v[j]);
-                }
-                uint32_t packed[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    packed[j] = pack2<DT>(v[2 * j], v[2 * j + 1]);
-
+                uint8_t *buf = cstage + (q * 2 + cbuf) * CF::C_BOX_BYTES;
                 if constexpr (TMA_STORE) {
                     // staging buffer `cbuf` was last used two stores ago
                     if (lane == 0)
                         bulk_wait_group_read<1>();
                     __syncwarp();
-                    uint8_t *buf = cstage + (q * 2 + cbuf) * CF::C_BOX_BYTES;
-                    // row `lane` of the 32x64 box; 16-byte chunk i lands at i ^ (lane & 7)
+                }
+                // two halves of 32 columns: fewer values live at once
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        uint4 w = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-                        *reinterpret_cast<uint4 *>(buf + lane * 128 + ((i ^ (lane & 7)) << 4)) = w;
+                for (int h = 0; h < 2; ++h) {
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        v[j] = __uint_as_float(r[32 * h + j]);
+                    const int colh = col0 + 32 * h;
+                    if constexpr (EPI == 1) {
+                        if (p.bias_vec16 && colh + 32 <= p.N) {
+                            const uint4 *bp = reinterpret_cast<const uint4 *>(p.bias + colh);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const uint4 w = __ldg(bp + i);
+                                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    v[8 * i + 2 * e] += to_float<DT>(static_cast<uint16_t>(ww[e] & 0xFFFFu));
+                                    v[8 * i + 2 * e + 1] += to_float<DT>(static_cast<uint16_t>(ww[e] >> 16));
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (colh + j < p.N)
+                                    v[j] += to_float<DT>(__ldg(p.bias + colh + j));
+                        }
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            v[j] = gelu_erf(v[j]);
                     }
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        packed[j] = pack2<DT>(v[2 * j], v[2 * j + 1]);
+
+                    if constexpr (TMA_STORE) {
+                        // row `lane` of the 32 x 64 box; 16-byte chunk i lands at i ^ (lane & 7)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int chunk = 4 * h + i;
+                            *reinterpret_cast<uint4 *>(buf + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+                                make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                        }
+                    } else {
+                        const int m = row0 + lane;
+                        if (m < p.M) {
+                            uint16_t *crow = p.C + static_cast<int64_t>(m) * p.ldc;
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const int n = colh + 2 * j;
+                                if (n < p.N)
+                                    crow[n] = static_cast<uint16_t>(packed[j] & 0xFFFFu);
+                                if (n + 1 < p.N)
+                                    crow[n + 1] = static_cast<uint16_t>(packed[j] >> 16);
+                            }
+                        }
+                    }
+                }
+                if constexpr (TMA_STORE) {
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
@@ -394,19 +481,6 @@ __global__ void __launch_bounds__(192, 1)
                         bulk_commit_group();
                     }
                     cbuf ^= 1;
-                } else {
-                    const int m = row0 + lane;
-                    if (m < p.M) {
-                        uint16_t *crow = p.C + static_cast<int64_t>(m) * p.ldc;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int n = col0 + 2 * j;
-                            if (n < p.N)
-                                crow[n] = static_cast<uint16_t>(packed[j] & 0xFFFFu);
-                            if (n + 1 < p.N)
-                                crow[n + 1] = static_cast<uint16_t>(packed[j] >> 16);
-                        }
-                    }
                 }
             }
             if (++acc == 2) {
@@ -424,15 +498,31 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0 && lane == 0 && *abort_flag) {
-        // Some role gave up: copies it never consumed may still be landing.
-        for (int s = 0; s < CF::STAGES; ++s)
-            if (issued & (1u << s))
-                wait_drain(full_bar(s), (issued_parity >> s) & 1u, timeout);
+        if constexpr (PAIR) {
+            // The pair's copies complete on the even CTA's barriers, which an
+            // abort can leave short of their arrival: give whatever is still in
+            // flight a fixed grace period (loads finish in microseconds).
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < 200000ull) {
+            }
+        } else {
+            // Some role gave up: copies it never consumed may still be landing.
+            for (int s = 0; s < CF::STAGES; ++s)
+                if (issued & (1u << s))
+                    wait_drain(full_bar(s), (issued_parity >> s) & 1u, timeout);
+        }
     }
-    __syncthreads();
+    if constexpr (PAIR)
+        cluster_sync();  // the even CTA's MMAs write this CTA's TMEM and read its shared memory
+    else
+        __syncthreads();
     tc_fence_after_sync();
-    if (warp == 1)
-        tmem_dealloc(tmem_base, CF::TMEM_COLS);
+    if (warp == 1) {
+        if constexpr (PAIR)
+            tmem_dealloc_pair(tmem_base, CF::TMEM_COLS);
+        else
+            tmem_dealloc(tmem_base, CF::TMEM_COLS);
+    }
 }
 
 // Zero-padded copy of a rows x cols matrix of 16-bit values (any alignment of

@@ -25,6 +25,7 @@ using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
 struct ConfigEntry {
     const char *name;
     int bm, bn, bk, stages;
+    int ctas;                // 1, or 2 for a CTA pair (cluster of two, cta_group::2 MMA)
     int smem_bytes;
     KernelFn fn[2][2][2];  // [dtype][epilogue][tma_store]
 };
@@ -34,8 +35,9 @@ ConfigEntry make_entry(const char *name)
 {
     ConfigEntry e;
     e.name = name;
-    e.bm = CF::BM;
+    e.bm = CF::TILE_M;
     e.bn = CF::BN;
+    e.ctas = CF::CTAS;
     e.bk = CF::BK;
     e.stages = CF::STAGES;
     e.smem_bytes = CF::SMEM_BYTES;
@@ -57,6 +59,8 @@ const ConfigEntry kConfigs[] = {
     make_entry<TileConfig<256, 4>>("bm128_bn256_bk64_s4"),
     make_entry<TileConfig<128, 6>>("bm128_bn128_bk64_s6"),
     make_entry<TileConfig<64, 8>>("bm128_bn64_bk64_s8"),
+    make_entry<TileConfig<256, 6, true>>("bm256_bn256_bk64_s6_pair"),
+    make_entry<TileConfig<128, 8, true>>("bm256_bn128_bk64_s8_pair"),
 };
 
 int num_configs() { return static_cast<int>(sizeof(kConfigs) / sizeof(kConfigs[0])); }
@@ -87,14 +91,35 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // more shared memory per MMA flop).
 int model_config(int64_t M, int64_t N, int num_sms)
 {
-    static const double eff[] = {1.0, 0.88, 0.6};
+    // relative tensor-pipe efficiency of each configuration when it has enough
+    // tiles (operand bytes each SM must pull per MMA flop)
+    static const double eff[] = {0.62, 0.5, 0.33, 0.95, 0.7};
     int best = 0;
     double best_cost = 1e300;
     for (int i = 0; i < num_configs(); ++i) {
         const ConfigEntry &c = kConfigs[i];
         const int64_t tiles = ceil_div(M, c.bm) * ceil_div(N, c.bn);
-        const double waves = static_cast<double>(ceil_div(tiles, num_sms));
-        const double cost = waves * c.bn / eff[i < 3 ? i : 2];
+        const int64_t units = num_sms / c.ctas;
+        const double waves = static_cast<double>(ceil_div(tiles, units));
+        const double cost = waves * (static_cast<double>(c.bm) * c.bn / c.ctas) / eff[i];
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = i;
+        }
+    }
+    return best;
+}
+
+// Best single-CTA configuration by the same model (the fault hook needs one).
+int model_config_single(int64_t M, int64_t N, int num_sms)
+{
+    int best = 0;
+    double best_cost = 1e300;
+    static const double eff[] = {0.62, 0.5, 0.33};
+    for (int i = 0; i < 3; ++i) {
+        const ConfigEntry &c = kConfigs[i];
+        const int64_t tiles = ceil_div(M, c.bm) * ceil_div(N, c.bn);
+        const double cost = static_cast<double>(ceil_div(tiles, num_sms)) * c.bm * c.bn / eff[i];
         if (cost < best_cost - 1e-9) {
             best_cost = cost;
             best = i;
@@ -140,6 +165,8 @@ tl_status validate(const void *A, const void *B, const void *bias, void *C, int6
         return TL_ERR_INVALID_ARG;
     if (opt && (opt->inject_fault != 0 && opt->inject_fault != 1))
         return TL_ERR_INVALID_ARG;
+    if (opt && opt->inject_fault && opt->config > 0 && kConfigs[opt->config - 1].ctas != 1)
+        return TL_ERR_UNSUPPORTED;  // the fault hook exists for single-CTA configurations only
     const int64_t lim = 0x7FFFFFFFll;
     if (M > lim || N > lim || K > lim)
         return TL_ERR_UNSUPPORTED;
@@ -156,7 +183,9 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
         return st;
     if (num_sms <= 0)
         return TL_ERR_INVALID_ARG;
-    const int ci = (opt && opt->config > 0) ? opt->config - 1 : choose_config(M, N, K, dtype, epi, num_sms);
+    int ci = (opt && opt->config > 0) ? opt->config - 1 : choose_config(M, N, K, dtype, epi, num_sms);
+    if (opt && opt->inject_fault && kConfigs[ci].ctas != 1)
+        ci = model_config_single(M, N, num_sms);
     const ConfigEntry &c = kConfigs[ci];
     Plan p{};
     tl_plan &q = p.pub;
@@ -170,7 +199,9 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
     const int64_t tiles = static_cast<int64_t>(q.tiles_m) * q.tiles_n;
     if (tiles > 0x7FFFFFFFll)
         return TL_ERR_UNSUPPORTED;
-    q.grid = static_cast<int32_t>(tiles < num_sms ? tiles : num_sms);
+    const int64_t units = num_sms / c.ctas;
+    q.grid = static_cast<int32_t>((tiles < units ? tiles : units) * c.ctas);
+    q.cluster_ctas = c.ctas;
     q.smem_bytes = c.smem_bytes;
     // TMA needs a 16-byte-aligned base and row strides that are multiples of 16 bytes.
     q.pad_a = !(aligned(A, 16) && K % 8 == 0);
@@ -235,6 +266,7 @@ struct DeviceState {
     int cc_major = 0;
     cudaMemPool_t pool = nullptr;
     std::unordered_map<const void *, bool> smem_set;  // kernels whose smem limit is raised
+    std::unordered_map<const void *, int> max_clusters;  // resident clusters of two, per kernel
 };
 
 std::mutex g_mu;
@@ -291,6 +323,25 @@ tl_status raise_smem_limit(DeviceState *d, KernelFn fn, int bytes)
     return TL_OK;
 }
 
+tl_status max_active_clusters(DeviceState *d, KernelFn fn, const cudaLaunchConfig_t &cfg, int *out)
+{
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = d->max_clusters.find(reinterpret_cast<const void *>(fn));
+        if (it != d->max_clusters.end()) {
+            *out = it->second;
+            return TL_OK;
+        }
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess)
+        return TL_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    d->max_clusters[reinterpret_cast<const void *>(fn)] = n;
+    *out = n;
+    return TL_OK;
+}
+
 tl_status launch_pad(const void *src, int64_t rows, int64_t cols, void *dst, int64_t dst_cols, int num_sms,
                      cudaStream_t stream)
 {
@@ -343,7 +394,28 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
     gp.ldc = N;
     gp.timeout_ns = (opt && opt->timeout_ns) ? opt->timeout_ns : kDefaultTimeoutNs;
 
-    fn<<<p.pub.grid, 192, c.smem_bytes, stream>>>(ta, tb, tc, gp);
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(static_cast<unsigned>(p.pub.grid), 1, 1);
+    cfg.blockDim = dim3(192, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(c.smem_bytes);
+    cfg.stream = stream;
+    if (c.ctas == 2) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        // persistent pairs: no more clusters than can be resident at once
+        int max_clusters = 0;
+        if ((st = max_active_clusters(d, fn, cfg, &max_clusters)) != TL_OK)
+            return st;
+        if (max_clusters > 0 && p.pub.grid > 2 * max_clusters)
+            cfg.gridDim.x = static_cast<unsigned>(2 * max_clusters);
+    }
+    if (cudaLaunchKernelEx(&cfg, fn, ta, tb, tc, gp) != cudaSuccess)
+        return TL_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ERR_CUDA;
 }
 

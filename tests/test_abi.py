@@ -39,7 +39,7 @@ def test_version_and_strings():
     n = tg.tl_num_configs()
     assert n >= 3
     names = tg.configs()
-    assert all(re.fullmatch(r"bm\d+_bn\d+_bk\d+_s\d+", x) for x in names)
+    assert all(re.fullmatch(r"bm\d+_bn\d+_bk\d+_s\d+(_pair)?", x) for x in names)
     assert tg.tl_config_name(n) is None and tg.tl_config_name(-1) is None
 
 
@@ -92,13 +92,13 @@ def test_plan_aligned_headline_shape():
     assert p["pad_a"] == 0 and p["pad_b"] == 0 and p["direct_store"] == 0
     assert p["workspace_bytes"] == 0
     assert p["tiles_m"] == 4096 // p["block_m"] and p["tiles_n"] == 4096 // p["block_n"]
-    assert p["grid"] == min(148, p["tiles_m"] * p["tiles_n"])
+    assert p["grid"] == min(148 // p["cluster_ctas"], p["tiles_m"] * p["tiles_n"]) * p["cluster_ctas"]
     assert p["smem_bytes"] <= 232448
 
 
 def test_plan_grid_never_exceeds_tiles():
     p = tg.plan(100, 60, 30, tg.TL_BF16, None, num_sms=148)
-    assert p["tiles_m"] == 1 and p["tiles_n"] == 1 and p["grid"] == 1
+    assert p["tiles_m"] == 1 and p["tiles_n"] == 1 and p["grid"] == p["cluster_ctas"]
 
 
 def test_plan_unaligned_k_pads_A_only():
@@ -126,6 +126,21 @@ def test_plan_forced_config():
         p = tg.plan(4096, 4096, 4096, tg.TL_F16, None, num_sms=148, config=k)
         assert p["config"] == k - 1
         assert p["config_name"] == tg.tl_config_name(k - 1)
+        pair = p["config_name"].endswith("_pair")
+        assert p["cluster_ctas"] == (2 if pair else 1)
+        assert p["grid"] % p["cluster_ctas"] == 0 and p["grid"] <= 148
+
+
+def test_fault_hook_only_on_single_cta_configs():
+    for k in range(1, tg.tl_num_configs() + 1):
+        opt = tg.Options(config=k, inject_fault=1)
+        st, p = tg.tl_gemm_plan(P, P, 0, P, 512, 512, 512, 0, 0, 148, opt)
+        if tg.tl_config_name(k - 1).endswith("_pair"):
+            assert st == tg.Status.UNSUPPORTED
+        else:
+            assert st == 0 and p.cluster_ctas == 1
+    st, p = tg.tl_gemm_plan(P, P, 0, P, 4096, 4096, 4096, 0, 0, 148, tg.Options(inject_fault=1))
+    assert st == 0 and p.cluster_ctas == 1
 
 
 def test_plan_skinny_prefers_narrow_tiles():

@@ -28,13 +28,17 @@ def n_configs():
     return tg().tl_num_configs()
 
 
+# every compiled kernel configuration, as the 1-based option value tl_gemm_ex takes
+ALL_CONFIGS = list(range(1, n_configs() + 1))
+
+
 def inputs(M, N, K, dt, epi, seed=0):
     w = wl.custom("t", M, N, K, dt, epi)
     return wl.make_inputs(w, seed)
 
 
 # ------------------------------------------------------------------ layout probes
-@pytest.mark.parametrize("config", [1, 2, 3])
+@pytest.mark.parametrize("config", ALL_CONFIGS)
 @pytest.mark.parametrize("dt", [wl.F16, wl.BF16])
 def test_layout_probe_one_hot(config, dt):
     """A has one 1 per row (row i picks k(i)); B[k, j] encodes (k, j) as a small
@@ -55,7 +59,7 @@ def test_layout_probe_one_hot(config, dt):
     assert np.array_equal(got, code[kk, :].astype(np.float32))
 
 
-@pytest.mark.parametrize("config", [1, 2, 3])
+@pytest.mark.parametrize("config", ALL_CONFIGS)
 def test_identity_gives_B(config):
     n, N = 256, 384
     A = wl.round_to_bits(np.eye(n, dtype=np.float32), wl.BF16)
@@ -92,7 +96,7 @@ def test_small_shapes_vs_oracle(M, N, K, dt, epi):
     compare(C, ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
 
 
-@pytest.mark.parametrize("config", [1, 2, 3])
+@pytest.mark.parametrize("config", ALL_CONFIGS)
 @pytest.mark.parametrize("epi", [wl.EPI_NONE, wl.EPI_BIAS_GELU])
 def test_every_config_vs_oracle(config, epi):
     M, N, K = 700, 900, 333
