@@ -24,7 +24,8 @@ using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
 
 struct ConfigEntry {
     const char *name;
-    int bm, bn, bk, stages;
+    int bm, bn, bk, stages;  // bm: output rows per tile (256 for a CTA pair)
+    int cta_m;               // rows of A each CTA loads per tile (the A box height)
     int ctas;                // 1, or 2 for a CTA pair (cluster of two, cta_group::2 MMA)
     int smem_bytes;
     KernelFn fn[2][2][2];  // [dtype][epilogue][tma_store]
@@ -36,6 +37,7 @@ ConfigEntry make_entry(const char *name)
     ConfigEntry e;
     e.name = name;
     e.bm = CF::TILE_M;
+    e.cta_m = CF::BM;
     e.bn = CF::BN;
     e.ctas = CF::CTAS;
     e.bk = CF::BK;
@@ -371,7 +373,7 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
 
     CUtensorMap ta, tb, tc;
     std::memset(&tc, 0, sizeof(tc));
-    if (!encode_2d(&ta, A, dtype, M, K, p.lda, 64, c.bm))
+    if (!encode_2d(&ta, A, dtype, M, K, p.lda, 64, c.cta_m))
         return TL_ERR_CUDA;
     if (!encode_2d(&tb, B, dtype, K, N, p.ldb, 64, c.bk))
         return TL_ERR_CUDA;

@@ -71,6 +71,36 @@ def shapes(which):
     return named + extra
 
 
+def write_table(best_rows):
+    """Write csrc/config_table.inc from the fastest record per shape."""
+    lines = ["// Kernel configuration per measured shape: {M, N, K, dtype, epilogue, config}.",
+             "// Written by tensor_core_gemm_tl_b200/sweep.py from timings on a B200; shapes",
+             "// not listed fall back to the wave model in tl_gemm.cu."]
+    seen = set()
+    for r in best_rows:
+        key = (r["M"], r["N"], r["K"], r["dtype"], r["epi"])
+        if key in seen:
+            continue
+        seen.add(key)
+        dt = 0 if r["dtype"] == "f16" else 1
+        lines.append(f'{{{r["M"]}, {r["N"]}, {r["K"]}, {dt}, {r["epi"]}, "{r["config"]}"}},'
+                     f'  // {r["tflops"]} TFLOP/s')
+    lines.append('{0, 0, 0, -1, -1, ""},  // sentinel, never matches')
+    with open(TABLE, "w") as f:
+        f.write("\n".join(lines) + "\n")
+    print("wrote", TABLE, file=sys.stderr)
+
+
+def best_from_records(records):
+    """The fastest record (lowest median time) per workload, in input order."""
+    best = {}
+    for r in records:
+        k = r["workload"]
+        if k not in best or r["median_ms"] < best[k]["median_ms"]:
+            best[k] = r
+    return list(best.values())
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--write", action="store_true")
@@ -78,7 +108,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--shapes", default="named", choices=["named", "all"])
     ap.add_argument("--only", default=None, help="comma-separated workload names")
+    ap.add_argument("--from-jsonl", default=None, help="write the table from recorded sweep output")
     a = ap.parse_args(argv)
+    if a.from_jsonl:
+        with open(a.from_jsonl) as f:
+            write_table(best_from_records([json.loads(x) for x in f if x.strip()]))
+        return 0
     import torch
     import tensor_core_gemm_tl_b200 as tg
     torch.cuda.set_device(0)
@@ -100,22 +135,7 @@ def main(argv=None):
                 best = (med, rec)
         rows.append(best[1])
     if a.write:
-        lines = ["// Kernel configuration per measured shape: {M, N, K, dtype, epilogue, config}.",
-                 "// Written by tensor_core_gemm_tl_b200/sweep.py from timings on a B200; shapes",
-                 "// not listed fall back to the wave model in tl_gemm.cu."]
-        seen = set()
-        for r in rows:
-            key = (r["M"], r["N"], r["K"], r["dtype"], r["epi"])
-            if key in seen:
-                continue
-            seen.add(key)
-            dt = 0 if r["dtype"] == "f16" else 1
-            lines.append(f'{{{r["M"]}, {r["N"]}, {r["K"]}, {dt}, {r["epi"]}, "{r["config"]}"}},'
-                         f'  // {r["tflops"]} TFLOP/s')
-        lines.append('{0, 0, 0, -1, -1, ""},  // sentinel, never matches')
-        with open(TABLE, "w") as f:
-            f.write("\n".join(lines) + "\n")
-        print("wrote", TABLE, file=sys.stderr)
+        write_table(rows)
     return 0
 
 
