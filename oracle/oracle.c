@@ -76,10 +76,12 @@ static double decode(uint16_t h, int dtype)
 }
 
 /* Exact (erf) GELU: x * Phi(x) with Phi the standard normal CDF,
- * Phi(x) = (1 + erf(x / sqrt 2)) / 2.                                       */
+ * Phi(x) = (1 + erf(x / sqrt 2)) / 2 = erfc(-x / sqrt 2) / 2.
+ * The erfc form is the same function; for negative x the erf form subtracts
+ * two numbers close to 1 and keeps only a few correct digits of Phi.        */
 double oracle_gelu(double x)
 {
-    return 0.5 * x * (1.0 + erf(x / sqrt(2.0)));
+    return 0.5 * x * erfc(-x / sqrt(2.0));
 }
 
 void oracle_gelu_array(const double *x, double *y, int64_t n)

@@ -298,9 +298,23 @@ def pin_gelu_invariants(orc, seed=23):
     assert np.all(np.diff(orc.gelu(xs)) > 0)
 
 
+def pin_gelu_tail_relative(orc):
+    """Relative accuracy of GELU over the whole range, the far negative tail
+    included (where x * Phi(x) is tiny): mpmath at 40 digits."""
+    import mpmath
+    mpmath.mp.dps = 40
+    xs = np.concatenate([np.linspace(-35, -1, 300), np.linspace(1, 30, 100), [-0.3, 0.25]])
+    got = orc.gelu(xs)
+    for x, g in zip(xs, got):
+        ref = float(mpmath.mpf(x) * mpmath.ncdf(mpmath.mpf(x)))
+        # the rounding of x / sqrt 2 alone moves erfc by ~2 z^2 u relative (z = |x| / sqrt 2)
+        assert abs(g - ref) <= (1e-15 + 4e-16 * x * x) * abs(ref), (x, g, ref)
+
+
 ALL_PINS = [
     pin_decode_all_patterns, pin_hand_example, pin_exact_bruteforce,
     pin_exact_bruteforce_epilogue, pin_vs_numpy_matmul, pin_identity, pin_row_sums,
     pin_all_ones, pin_zero_B_gelu_table, pin_bias_then_gelu, pin_transpose,
     pin_power_of_two_scaling, pin_rows_and_points, pin_gelu_table, pin_gelu_invariants,
+    pin_gelu_tail_relative,
 ]

@@ -20,9 +20,12 @@ MUTANTS = [
     ("dropped_first_k", "for (int64_t k = 0; k < K; ++k) {", "for (int64_t k = 1; k < K; ++k) {"),
     ("wrong_sign", "c[j] += a * b[j];", "c[j] -= a * b[j];"),
     ("float_accumulator", "c[j] += a * b[j];", "c[j] = (float)(c[j] + a * b[j]);"),
-    ("tanh_gelu", "return 0.5 * x * (1.0 + erf(x / sqrt(2.0)));",
+    ("tanh_gelu", "return 0.5 * x * erfc(-x / sqrt(2.0));",
      "return 0.5 * x * (1.0 + tanh(0.7978845608028654 * (x + 0.044715 * x * x * x)));"),
-    ("gelu_wrong_scale", "erf(x / sqrt(2.0))", "erf(x / 2.0)"),
+    ("gelu_wrong_scale", "erfc(-x / sqrt(2.0))", "erfc(-x / 2.0)"),
+    ("gelu_cancelling_form", "return 0.5 * x * erfc(-x / sqrt(2.0));",
+     "return 0.5 * x * (1.0 + erf(x / sqrt(2.0)));"),
+    ("gelu_wrong_sign_in_erfc", "erfc(-x / sqrt(2.0))", "erfc(x / sqrt(2.0))"),
     ("bias_after_gelu", "c[j] = oracle_gelu(c[j] + decode(bias[j], dtype));",
      "c[j] = oracle_gelu(c[j]) + decode(bias[j], dtype);"),
     ("bias_by_row", "c[j] = oracle_gelu(c[j] + decode(bias[j], dtype));",
