@@ -15,10 +15,11 @@
 //          --tcgen05.ld--> registers: + bias, GELU, round once to fp16/bf16
 //          --st.shared (swizzled)--> TMA store --> global
 //
-// Warp roles (192 threads, one CTA per SM, persistent over output tiles):
+// Warp roles (320 threads, one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer (one lane)
 //   warp 1      TMEM allocator + MMA issuer (one lane)
-//   warps 2..5  epilogue; warp w reads TMEM lanes 32*(w%4) .. +31
+//   warps 2..9  epilogue; warp w reads TMEM lanes 32*(w%4) .. +31 and every
+//               other 64-column chunk of them (two warps per lane quarter)
 //
 // Two TMEM accumulators (2 x BN fp32 columns) let the epilogue of tile i run
 // while the MMAs of tile i+1 accumulate.  Every wait is bounded by a
@@ -78,9 +79,10 @@ struct TileConfig {
     static constexpr int B_STAGE_BYTES = BK * BN_LOCAL * 2;
     static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
     static constexpr int TX_BYTES = STAGE_BYTES * CTAS;  // landing on the (even CTA's) full barrier
-    static constexpr int EPI_WARPS = 4;
+    // two epilogue warps per TMEM lane quarter; they split the 64-column chunks
+    static constexpr int EPI_WARPS = 8;
     static constexpr int C_BOX_BYTES = 32 * 128;   // 32 rows x 64 columns of 16-bit
-    static constexpr int C_STAGING_BYTES = EPI_WARPS * 2 * C_BOX_BYTES;
+    static constexpr int C_STAGING_BYTES = EPI_WARPS * C_BOX_BYTES;  // one box per epilogue warp
     static constexpr int ACC_COLS = BN;             // fp32 TMEM columns per accumulator
     static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
     static constexpr int OFF_A = 0;
@@ -90,7 +92,7 @@ struct TileConfig {
     static constexpr int NUM_BARS = 2 * STAGES + 5;
     static constexpr int SMEM_USED = OFF_BAR + NUM_BARS * 8 + 16;
     static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = 64 + 32 * EPI_WARPS;  // producer, MMA, epilogue warps
     static_assert(BN_LOCAL % 64 == 0 && BN >= 64 && BN <= 256, "BN");
     static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM columns");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -177,21 +179,22 @@ __device__ __forceinline__ float to_float(uint16_t bits)
 // The substitution t is that of Abramowitz & Stegun, Handbook of Mathematical
 // Functions, 7.1.26; h is this library's own degree-8 least-squares fit to
 // exp(z^2) erfc(z) on z in [0, 9.25] (relative error of h ~3e-8; the
-// coefficients come from csrc/fit_gelu_erfcx.py).  exp(-z^2) = exp(-x^2/2) is
-// taken from x^2 split exactly into hi + lo (one fma), so the argument does
-// not lose bits as |x| grows.  Computing erfc of |x| avoids the cancellation
-// of 1 + erf(x / sqrt 2) for negative x.  Relative error about 4e-7 for
-// |x| <= 9 (a few float32 ulps; far below one fp16 / bf16 ulp); NaN stays NaN.
+// coefficients come from csrc/fit_gelu_erfcx.py).  exp(-z^2) = 2^(-x^2 log2(e) / 2)
+// is taken from x^2 split exactly into hi + lo (one fma), so the argument does
+// not lose the low bits of x^2 and loses only the rounding of one product as |x| grows.  Computing erfc of |x|
+// avoids the cancellation of 1 + erf(x / sqrt 2) for negative x.  Relative
+// error below 3e-6 for |x| <= 9 (below 1e-5 everywhere; one fp16 ulp is 5e-4,
+// one bf16 ulp 4e-3); NaN stays NaN.
 __device__ __forceinline__ float gelu_erf(float x)
 {
-    constexpr float P = 0.415f;
+    constexpr float P_SQRT1_2 = 0.415f * 0.70710678118654752f;  // p / sqrt 2: t = 1 / (1 + p' |x|)
     constexpr float C0 = 4.281122892280109e-05f, C1 = 0.23316948115825653f, C2 = 0.24358120560646057f,
                     C3 = 0.1621198058128357f, C4 = 0.34987202286720276f, C5 = -0.2624722123146057f,
                     C6 = 0.5700822472572327f, C7 = -0.3758394122123718f, C8 = 0.079444020986557f;
+    constexpr float NEG_HALF_LOG2E = -0.72134752044448170f;  // -log2(e) / 2
     // beyond |x| = 20, Phi is exactly 0 or 1 in float32; the clamp keeps x^2 finite
     const float a = fminf(fabsf(x), 20.0f);
-    const float z = a * 0.70710678118654752f;
-    const float t = __frcp_rn(fmaf(P, z, 1.0f));
+    const float t = rcp_approx(fmaf(P_SQRT1_2, a, 1.0f));
     float h = fmaf(C8, t, C7);
     h = fmaf(h, t, C6);
     h = fmaf(h, t, C5);
@@ -201,14 +204,14 @@ __device__ __forceinline__ float gelu_erf(float x)
     h = fmaf(h, t, C1);
     h = fmaf(h, t, C0);
     const float hi = a * a;
-    const float lo = fmaf(a, a, -hi);                          // a^2 = hi + lo exactly
-    const float e = __expf(-0.5f * hi) * fmaf(-0.5f, lo, 1.0f);  // exp(-x^2 / 2)
-    const float q = 0.5f * h * e;                               // erfc(z) / 2
+    const float lo = fmaf(a, a, -hi);                                   // a^2 = hi + lo exactly
+    const float e = exp2_approx(hi * NEG_HALF_LOG2E) * fmaf(-0.5f, lo, 1.0f);  // exp(-x^2 / 2)
+    const float q = 0.5f * h * e;                                       // erfc(z) / 2
     return x * (x >= 0.0f ? 1.0f - q : q);
 }
 
 template <class CF, int DT, int EPI, bool TMA_STORE>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(CF::THREADS, 1)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_c, const GemmParams p)
 {
@@ -399,11 +402,14 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int q = warp & 3;               // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;     // which of the quarter's two warps: chunks c = half, half + 2, ...
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        constexpr int CHUNKS = CF::BN / 64;
+        const int my_last = (CHUNKS - 1 - half) >= 0 ? half + 2 * ((CHUNKS - 1 - half) / 2) : -1;
+        uint8_t *buf = cstage + (warp - 2) * CF::C_BOX_BYTES;
         int acc = 0;
         uint32_t acc_phase = 0;
-        int cbuf = 0;
         for (int t = unit; t < p.num_tiles; t += num_units) {
             int tm, tn;
             tile_coords(t, p, tm, tn);
@@ -412,33 +418,36 @@ __global__ void __launch_bounds__(192, 1)
             if (!wait_bounded<PAIR>(tfull_bar(acc), acc_phase, abort_flag, timeout, ERR_EPILOGUE, peer_abort))
                 break;
             tc_fence_after_sync();
+            auto release_accumulator = [&]() {
+                // this warp's share of the accumulator is in registers: hand it back
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (PAIR)
+                        mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+                    else
+                        mbar_arrive(tempty_bar(acc));
+                }
+            };
+            if (my_last < 0)
+                release_accumulator();
 #pragma unroll 1
-            for (int c = 0; c < CF::BN / 64; ++c) {
+            for (int c = half; c < CHUNKS; c += 2) {
                 uint32_t r[64];
                 const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(acc * CF::ACC_COLS + c * 64);
                 tmem_load_32cols(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
                 tmem_load_32cols(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
                 tmem_load_wait();
-                if (c == CF::BN / 64 - 1) {
-                    // accumulator fully read: hand it back to the MMA warp
-                    tc_fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if constexpr (PAIR)
-                            mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
-                        else
-                            mbar_arrive(tempty_bar(acc));
-                    }
-                }
+                if (c == my_last)
+                    release_accumulator();
                 const int col0 = n0 + c * 64;
                 if (col0 >= p.N || row0 >= p.M)
                     continue;  // nothing of this chunk lies inside C
 
-                uint8_t *buf = cstage + (q * 2 + cbuf) * CF::C_BOX_BYTES;
                 if constexpr (TMA_STORE) {
-                    // staging buffer `cbuf` was last used two stores ago
+                    // this warp's staging box: its previous store must have read it
                     if (lane == 0)
-                        bulk_wait_group_read<1>();
+                        bulk_wait_group_read<0>();
                     __syncwarp();
                 }
                 // two halves of 32 columns: fewer values live at once
@@ -507,7 +516,6 @@ __global__ void __launch_bounds__(192, 1)
                         tma_store_2d(&tmap_c, smem_addr(buf), col0, row0);
                         bulk_commit_group();
                     }
-                    cbuf ^= 1;
                 }
             }
             if (++acc == 2) {

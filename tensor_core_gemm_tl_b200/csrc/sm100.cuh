@@ -179,6 +179,23 @@ __device__ __forceinline__ void tmem_load_wait()
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- fast arithmetic
+// Hardware approximate reciprocal and base-2 exponential (one MUFU op each;
+// relative error about 2^-23 and 2^-22).  No .ftz: subnormal results are kept.
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float exp2_approx(float x)
+{
+    float r;
+    asm("ex2.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor (tcgen05), 128-byte swizzle:
 //   bits  0-13 start address >> 4     bits 16-29 leading byte offset >> 4

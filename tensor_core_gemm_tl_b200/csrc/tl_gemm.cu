@@ -27,6 +27,7 @@ struct ConfigEntry {
     int bm, bn, bk, stages;  // bm: output rows per tile (256 for a CTA pair)
     int cta_m;               // rows of A each CTA loads per tile (the A box height)
     int ctas;                // 1, or 2 for a CTA pair (cluster of two, cta_group::2 MMA)
+    int threads;             // threads per CTA
     int smem_bytes;
     KernelFn fn[2][2][2];  // [dtype][epilogue][tma_store]
 };
@@ -40,6 +41,7 @@ ConfigEntry make_entry(const char *name)
     e.cta_m = CF::BM;
     e.bn = CF::BN;
     e.ctas = CF::CTAS;
+    e.threads = CF::THREADS;
     e.bk = CF::BK;
     e.stages = CF::STAGES;
     e.smem_bytes = CF::SMEM_BYTES;
@@ -399,7 +401,7 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];
     cfg.gridDim = dim3(static_cast<unsigned>(p.pub.grid), 1, 1);
-    cfg.blockDim = dim3(192, 1, 1);
+    cfg.blockDim = dim3(static_cast<unsigned>(c.threads), 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(c.smem_bytes);
     cfg.stream = stream;
     if (c.ctas == 2) {
