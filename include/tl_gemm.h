@@ -57,7 +57,8 @@ typedef enum {
     TL_ERR_UNSUPPORTED = 2,     /* size beyond the 32-bit coordinate range, no sm_100 device */
     TL_ERR_MISALIGNED = 3,      /* a pointer not aligned to its 2-byte element */
     TL_ERR_CUDA = 4,            /* a CUDA runtime or driver call failed */
-    TL_ERR_DEVICE_TIMEOUT = 5   /* a bounded wait inside a kernel ran out (see tl_check_device) */
+    TL_ERR_DEVICE_TIMEOUT = 5,  /* a bounded wait inside a kernel ran out (see tl_check_device) */
+    TL_ERR_SCRATCH_LIMIT = 6    /* tl_gemm_noalloc: the call needs more than TL_NOALLOC_SCRATCH_BYTES */
 } tl_status;
 
 /* A cudaStream_t, passed as an opaque pointer; NULL is the legacy default stream. */
@@ -93,6 +94,45 @@ typedef void *tl_stream;
 TL_API tl_status tl_gemm(const void *A, const void *B, const void *bias, void *C,
                   int64_t M, int64_t N, int64_t K,
                   tl_dtype dtype, tl_epilogue epi, tl_stream stream);
+
+/*
+ * tl_gemm_noalloc -- tl_gemm for callers that must not allocate device memory.
+ *
+ * The TileLang pages have no counterpart to this call; it exists for users of
+ * this library whose code cannot allocate at the moment it runs a GEMM: a
+ * plugin whose execute step an inference engine forbids from allocating, a
+ * service that reserves all of its device memory up front under a fixed
+ * budget, or code that must not call cudaMalloc because it would synchronize
+ * the device or fail inside a stream capture.  tl_gemm may take a temporary
+ * from a memory pool when an operand has to be copied into a zero-padded
+ * layout (K or N not a multiple of 8, or a base that is not 16-byte aligned);
+ * tl_gemm_noalloc instead uses a fixed scratch area of
+ * TL_NOALLOC_SCRATCH_BYTES that the library declares statically: each GPU the
+ * library is used on holds that much device memory until the process exits.
+ *
+ * Arguments, layout rules, results and errors are those of tl_gemm, plus
+ * TL_ERR_SCRATCH_LIMIT when the padded copies the call needs are larger than
+ * TL_NOALLOC_SCRATCH_BYTES (tl_gemm_plan reports the need as
+ * workspace_bytes).  Nothing is enqueued in that case.  A call whose operands
+ * need no padding uses no scratch at all.
+ *
+ * The scratch area is shared by all calls on a device and keeps what the last
+ * call wrote; each call rewrites every byte of it that it later reads.  Calls
+ * whose work can overlap on the GPU (different streams with no ordering
+ * between them) race on the scratch area and can give wrong results: order
+ * them on one stream, or with events.
+ *
+ * The first call on each device does a one-time set-up with that device
+ * current: it looks up the device address of the scratch area, raises the
+ * kernels' shared-memory limits and records a few bytes of host bookkeeping.
+ * Make that first call before any stream capture begins.  After it, a call
+ * allocates nothing, on the device or on the host.
+ */
+#define TL_NOALLOC_SCRATCH_BYTES (32ull << 20)
+
+TL_API tl_status tl_gemm_noalloc(const void *A, const void *B, const void *bias, void *C,
+                         int64_t M, int64_t N, int64_t K,
+                         tl_dtype dtype, tl_epilogue epi, tl_stream stream);
 
 /* Options for tl_gemm_ex.  Zero-initialise, then set what you need. */
 typedef struct {

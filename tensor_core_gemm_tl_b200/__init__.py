@@ -14,13 +14,13 @@ from __future__ import annotations
 
 from ._binding import (  # noqa: F401
     LIB_PATH, Options, Plan, Status, TLError, TL_BF16, TL_EPI_BIAS_GELU, TL_EPI_NONE, TL_F16,
-    SIGNATURES, tl_check_device, tl_config_name, tl_gemm, tl_gemm_ex, tl_gemm_plan, tl_num_configs,
+    SIGNATURES, tl_check_device, tl_config_name, tl_gemm, tl_gemm_ex, tl_gemm_noalloc, tl_gemm_plan, tl_num_configs,
     tl_status_string, tl_version,
 )
 
 __all__ = [
     "gemm", "check_device", "plan", "configs", "Options", "Plan", "Status", "TLError",
-    "tl_gemm", "tl_gemm_ex", "tl_check_device", "tl_gemm_plan", "tl_num_configs", "tl_config_name",
+    "tl_gemm", "tl_gemm_ex", "tl_gemm_noalloc", "tl_check_device", "tl_gemm_plan", "tl_num_configs", "tl_config_name",
     "tl_status_string", "tl_version", "TL_F16", "TL_BF16", "TL_EPI_NONE", "TL_EPI_BIAS_GELU",
 ]
 

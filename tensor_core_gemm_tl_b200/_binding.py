@@ -24,6 +24,7 @@ class Status(enum.IntEnum):
     MISALIGNED = 3
     CUDA = 4
     DEVICE_TIMEOUT = 5
+    SCRATCH_LIMIT = 6
 
 
 class TLError(RuntimeError):
@@ -56,6 +57,7 @@ class Plan(ctypes.Structure):
 _P, _I64, _I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
 SIGNATURES = {
     "tl_gemm": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, _P]),
+    "tl_gemm_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, _P]),
     "tl_gemm_ex": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, _P,
                                   ctypes.POINTER(Options)]),
     "tl_check_device": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
@@ -70,7 +72,7 @@ SIGNATURES = {
 
 def load(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
-        raise ImportError(f"{path} is missing: build it with `python -m tensor_core_gemm_tl_b200.build`")
+        raise ImportError(f"{path} is missing: build it with `python tensor_core_gemm_tl_b200/build.py`")
     lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)
@@ -91,6 +93,13 @@ def tl_gemm(A: int, B: int, bias: int | None, C: int, M: int, N: int, K: int, dt
             stream: int = 0) -> int:
     """C = epilogue(A.B) on device pointers; returns the tl_status code."""
     return _lib.tl_gemm(A, B, bias or None, C, M, N, K, dtype, epi, stream or None)
+
+
+def tl_gemm_noalloc(A: int, B: int, bias: int | None, C: int, M: int, N: int, K: int, dtype: int, epi: int,
+                    stream: int = 0) -> int:
+    """tl_gemm without any allocation: padded operand copies go to the library's
+    fixed scratch area; returns the tl_status code (SCRATCH_LIMIT if too big)."""
+    return _lib.tl_gemm_noalloc(A, B, bias or None, C, M, N, K, dtype, epi, stream or None)
 
 
 def tl_gemm_ex(A, B, bias, C, M, N, K, dtype, epi, stream=0, options: Options | None = None) -> int:

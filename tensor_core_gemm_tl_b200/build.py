@@ -1,6 +1,8 @@
 """Build libtlgemm.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
 
-    python -m tensor_core_gemm_tl_b200.build [--force] [--verbose-ptxas]
+    python tensor_core_gemm_tl_b200/build.py [--force] [--verbose-ptxas]
+
+(Run as a script: importing the package loads the library it builds.)
 """
 from __future__ import annotations
 

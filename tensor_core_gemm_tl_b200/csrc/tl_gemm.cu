@@ -464,10 +464,120 @@ tl_status gemm_impl(const void *A, const void *B, const void *bias, void *C, int
     return st;
 }
 
+// ------------------------------------------------------------------ allocation-free entry point
+// The scratch area of tl_gemm_noalloc: file scope, one per device, reserved
+// when the module is loaded.  Host code may only use the address that
+// cudaGetSymbolAddress returns for the current device, never the name.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[TL_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxNoallocDevices = 64;
+std::atomic<void *> g_noalloc_scratch_ptr[kMaxNoallocDevices];
+
+// One-time set-up per device (the device must be current): the scratch area's
+// device address, and every kernel's shared-memory limit and cluster
+// occupancy, so that later calls touch no allocator and insert into no map.
+tl_status noalloc_setup(DeviceState *d, void **scratch)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return TL_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxNoallocDevices)
+        return TL_ERR_UNSUPPORTED;
+    void *p = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (p) {
+        *scratch = p;
+        return TL_OK;
+    }
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lk(mu);
+    p = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        void *addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr)
+            return TL_ERR_CUDA;
+        for (int i = 0; i < num_configs(); ++i) {
+            const ConfigEntry &c = kConfigs[i];
+            for (int dt = 0; dt < 2; ++dt)
+                for (int epi = 0; epi < 2; ++epi)
+                    for (int st = 0; st < 2; ++st) {
+                        KernelFn fn = c.fn[dt][epi][st];
+                        tl_status r = raise_smem_limit(d, fn, c.smem_bytes);
+                        if (r != TL_OK)
+                            return r;
+                        if (c.ctas == 2) {
+                            cudaLaunchConfig_t cfg{};
+                            cudaLaunchAttribute attr[1];
+                            attr[0].id = cudaLaunchAttributeClusterDimension;
+                            attr[0].val.clusterDim.x = 2;
+                            attr[0].val.clusterDim.y = 1;
+                            attr[0].val.clusterDim.z = 1;
+                            cfg.gridDim = dim3(2, 1, 1);
+                            cfg.blockDim = dim3(static_cast<unsigned>(c.threads), 1, 1);
+                            cfg.dynamicSmemBytes = static_cast<size_t>(c.smem_bytes);
+                            cfg.attrs = attr;
+                            cfg.numAttrs = 1;
+                            int n = 0;
+                            if ((r = max_active_clusters(d, fn, cfg, &n)) != TL_OK)
+                                return r;
+                        }
+                    }
+        }
+        p = addr;
+        g_noalloc_scratch_ptr[dev].store(p, std::memory_order_release);
+    }
+    *scratch = p;
+    return TL_OK;
+}
+
+tl_status gemm_noalloc_impl(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N,
+                            int64_t K, int dtype, int epi, cudaStream_t stream)
+{
+    tl_status st = validate(A, B, bias, C, M, N, K, dtype, epi, nullptr);
+    if (st != TL_OK)
+        return st;
+    DeviceState *d = nullptr;
+    if ((st = device_state(&d)) != TL_OK)
+        return st;
+    if (d->cc_major != 10)
+        return TL_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if ((st = noalloc_setup(d, &scratch)) != TL_OK)
+        return st;
+    Plan p;
+    if ((st = make_plan(A, B, bias, C, M, N, K, dtype, epi, d->num_sms, nullptr, &p)) != TL_OK)
+        return st;
+    if (p.pub.workspace_bytes == 0)
+        return launch_gemm(p, A, B, bias, C, M, N, K, dtype, epi, stream, d, nullptr);
+    if (static_cast<uint64_t>(p.pub.workspace_bytes) > TL_NOALLOC_SCRATCH_BYTES)
+        return TL_ERR_SCRATCH_LIMIT;
+    // the padded copies overwrite every byte of scratch that the GEMM reads
+    const void *a_use = A, *b_use = B;
+    if (p.pub.pad_a) {
+        void *dst = static_cast<uint8_t *>(scratch) + p.a_ws_off;
+        if ((st = launch_pad(A, M, K, dst, p.lda, d->num_sms, stream)) != TL_OK)
+            return st;
+        a_use = dst;
+    }
+    if (p.pub.pad_b) {
+        void *dst = static_cast<uint8_t *>(scratch) + p.b_ws_off;
+        if ((st = launch_pad(B, K, N, dst, p.ldb, d->num_sms, stream)) != TL_OK)
+            return st;
+        b_use = dst;
+    }
+    return launch_gemm(p, a_use, b_use, bias, C, M, N, K, dtype, epi, stream, d, nullptr);
+}
+
 } // namespace
 } // namespace tl
 
 extern "C" {
+
+tl_status tl_gemm_noalloc(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N,
+                          int64_t K, tl_dtype dtype, tl_epilogue epi, tl_stream stream)
+{
+    return tl::gemm_noalloc_impl(A, B, bias, C, M, N, K, dtype, epi, static_cast<cudaStream_t>(stream));
+}
+
 
 tl_status tl_gemm(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
                   tl_dtype dtype, tl_epilogue epi, tl_stream stream)
@@ -535,6 +645,7 @@ const char *tl_status_string(tl_status s)
     case TL_ERR_MISALIGNED: return "TL_ERR_MISALIGNED";
     case TL_ERR_CUDA: return "TL_ERR_CUDA";
     case TL_ERR_DEVICE_TIMEOUT: return "TL_ERR_DEVICE_TIMEOUT";
+    case TL_ERR_SCRATCH_LIMIT: return "TL_ERR_SCRATCH_LIMIT";
     }
     return "TL_ERR_UNKNOWN";
 }
