@@ -143,6 +143,8 @@ typedef struct {
                              the consumer's bounded wait runs out and the kernel
                              returns with TL_ERR_DEVICE_TIMEOUT recorded          */
     uint64_t timeout_ns;  /* bound on every wait inside the kernel; 0 = 10 s     */
+    int32_t no_split;     /* 1: never split the tiles of a short last round      */
+    int32_t reserved;     /* must be 0                                           */
 } tl_gemm_options;
 
 /* tl_gemm with options (NULL options == tl_gemm).  Same arguments and errors;
@@ -172,9 +174,11 @@ typedef struct {
     int32_t config;          /* kernel configuration index                     */
     int32_t block_m, block_n, block_k, stages;
     int32_t tiles_m, tiles_n;
-    int32_t grid;            /* persistent CTAs launched (the launch may lower it
-                                to the number of CTA pairs that fit at once)   */
+    int32_t grid;            /* persistent CTAs launched                       */
     int32_t cluster_ctas;    /* 1, or 2 when pairs of CTAs share each tile     */
+    int32_t split;           /* K parts of each tile of the last, partial round
+                                of tiles (1: none are split)                   */
+    int32_t full_tiles;      /* tiles computed whole; the rest are split       */
     int32_t pad_a, pad_b;    /* 1 when the operand is first copied to a padded temporary */
     int32_t direct_store;    /* 1 when C is stored element by element          */
     int32_t smem_bytes;      /* dynamic shared memory per CTA                  */

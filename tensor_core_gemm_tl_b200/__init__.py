@@ -42,7 +42,8 @@ def _epi_code(epilogue):
     raise ValueError(f"unknown epilogue {epilogue!r}")
 
 
-def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0, timeout_ns: int = 0):
+def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0, timeout_ns: int = 0,
+         no_split: bool = False):
     """C = epilogue(A @ B) for row-major CUDA tensors A (M x K) and B (K x N).
 
     ``epilogue`` is None / "none" or "bias_gelu" (``bias`` of length N is then
@@ -71,8 +72,8 @@ def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0,
         raise ValueError("out must be a contiguous CUDA tensor of shape (M, N) and the input dtype")
     s = stream if stream is not None else torch.cuda.current_stream(A.device)
     with torch.cuda.device(A.device):
-        if config or timeout_ns:
-            opt = Options(config=config, inject_fault=0, timeout_ns=timeout_ns)
+        if config or timeout_ns or no_split:
+            opt = Options(config=config, inject_fault=0, timeout_ns=timeout_ns, no_split=int(no_split))
             st = tl_gemm_ex(A.data_ptr(), B.data_ptr(), bias.data_ptr() if bias is not None else 0,
                             out.data_ptr(), M, N, K, dt, epi, s.cuda_stream, opt)
         else:

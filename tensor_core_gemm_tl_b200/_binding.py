@@ -35,9 +35,10 @@ class TLError(RuntimeError):
 
 class Options(ctypes.Structure):
     """tl_gemm_options: config (0 = library's choice, k = configuration k-1),
-    inject_fault (test hook), timeout_ns (0 = 10 s)."""
+    inject_fault (test hook), timeout_ns (0 = 10 s), no_split (1 = never split
+    the tiles of a short last round)."""
     _fields_ = [("config", ctypes.c_int32), ("inject_fault", ctypes.c_int32),
-                ("timeout_ns", ctypes.c_uint64)]
+                ("timeout_ns", ctypes.c_uint64), ("no_split", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class Plan(ctypes.Structure):
@@ -45,7 +46,7 @@ class Plan(ctypes.Structure):
     _fields_ = [("config", ctypes.c_int32), ("block_m", ctypes.c_int32), ("block_n", ctypes.c_int32),
                 ("block_k", ctypes.c_int32), ("stages", ctypes.c_int32), ("tiles_m", ctypes.c_int32),
                 ("tiles_n", ctypes.c_int32), ("grid", ctypes.c_int32), ("cluster_ctas", ctypes.c_int32),
-                ("pad_a", ctypes.c_int32),
+                ("split", ctypes.c_int32), ("full_tiles", ctypes.c_int32), ("pad_a", ctypes.c_int32),
                 ("pad_b", ctypes.c_int32), ("direct_store", ctypes.c_int32),
                 ("smem_bytes", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64)]
 

@@ -1,0 +1,110 @@
+"""Time the library against PyTorch eager on the same workloads (needs a GPU).
+
+The TileLang pages compare their GEMM with PyTorch and cuBLAS, and their
+fused bias + GELU epilogue with PyTorch eager (TileLang GPU kernel design
+article, paragraphs 2 and 5).  This tool does the same on a B200: for each
+named workload it times
+
+  * tl_gemm (this library, through the C ABI),
+  * torch.matmul (cuBLAS), and for the epilogue workloads
+  * torch eager  A @ B + bias, then torch.nn.functional.gelu (exact form):
+    three kernels and two intermediates through HBM,
+
+with CUDA events over operands rotated beyond L2, median of the launches.
+It prints one JSON line per workload.  A diagnostic, not the benchmark.
+
+    python -m tensor_core_gemm_tl_b200.compare [--only name,...] [--launches 40]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _median_ms(fn, nsets, launches, warmup):
+    import torch
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        fn(i % nsets)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
+    for i, (s, e) in enumerate(ev):
+        s.record(stream)
+        fn(i % nsets)
+        e.record(stream)
+    torch.cuda.synchronize()
+    return float(np.median([s.elapsed_time(e) for s, e in ev]))
+
+
+def compare(w, launches=40, warmup=10):
+    import torch
+    import torch.nn.functional as F
+    import tensor_core_gemm_tl_b200 as tg
+    A_bits, B_bits, bias_bits = wl.make_inputs(w, 0)
+    tdt = torch.float16 if w.dtype == wl.F16 else torch.bfloat16
+
+    def dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).cuda().view(tdt)
+
+    A0, B0 = dev(A_bits), dev(B_bits)
+    bias = dev(bias_bits) if bias_bits is not None else None
+    set_bytes = 2 * (w.M * w.K + w.K * w.N + w.M * w.N)
+    nsets = max(2, int(np.ceil(3 * L2_BYTES / set_bytes)))
+    sets = [(A0.clone(), B0.clone(), torch.empty((w.M, w.N), dtype=tdt, device="cuda")) for _ in range(nsets)]
+    epi = "bias_gelu" if w.epi == wl.EPI_BIAS_GELU else None
+
+    def ours(i):
+        A, B, C = sets[i]
+        tg.gemm(A, B, bias, epilogue=epi, out=C)
+
+    def cublas(i):
+        A, B, C = sets[i]
+        torch.matmul(A, B, out=C)
+
+    def eager(i):
+        A, B, C = sets[i]
+        C.copy_(F.gelu(torch.matmul(A, B) + bias, approximate="none"))
+
+    res = {"workload": w.name, "M": w.M, "N": w.N, "K": w.K}
+    t = _median_ms(ours, nsets, launches, warmup)
+    res["tl_gemm_tflops"] = round(w.flops / t / 1e9, 1)
+    t = _median_ms(cublas, nsets, launches, warmup)
+    res["torch_matmul_tflops"] = round(w.flops / t / 1e9, 1)
+    if epi:
+        t = _median_ms(eager, nsets, launches, warmup)
+        res["torch_eager_bias_gelu_tflops"] = round(w.flops / t / 1e9, 1)
+    if tg.check_device() != 0:
+        raise RuntimeError("device error")
+    return res
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--only", default=None)
+    ap.add_argument("--launches", type=int, default=40)
+    a = ap.parse_args(argv)
+    import torch
+    torch.cuda.set_device(0)
+    todo = list(wl.WORKLOADS.values())
+    if a.only:
+        keep = set(a.only.split(","))
+        todo = [w for w in todo if w.name in keep]
+    for w in todo:
+        print(json.dumps(compare(w, a.launches)), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -46,6 +46,7 @@ enum : unsigned {
     ERR_MMA_ACC = 4u,
     ERR_EPILOGUE = 8u,
     ERR_DRAIN = 16u,
+    ERR_SPLIT = 32u,   // the last part of a split tile gave up waiting for an earlier part
 };
 
 struct GemmParams {
@@ -58,7 +59,50 @@ struct GemmParams {
     uint16_t *C;             // direct-store path only
     int64_t ldc;             // direct-store path only (elements)
     uint64_t timeout_ns;
+    // Work items: tiles [0, full_tiles) whole, then each remaining tile split
+    // along K into `split` parts, item = full_tiles + r * split + part.  Parts
+    // 0 .. split-2 leave fp32 partial sums in `partials` and stamp their flag
+    // with `epoch`; the last part adds them, in part order, to its own sum and
+    // runs the epilogue.
+    int32_t full_tiles, split, num_items;
+    float *partials;
+    unsigned long long *flags;
+    unsigned long long epoch;  // unique per launch
 };
+
+struct WorkItem {
+    int tile, part, kb0, kb1;  // output tile, part index, k-block range [kb0, kb1)
+};
+
+__device__ __forceinline__ WorkItem work_item(int item, const GemmParams &p)
+{
+    WorkItem w;
+    if (item < p.full_tiles) {
+        w.tile = item;
+        w.part = 0;
+        w.kb0 = 0;
+        w.kb1 = p.num_kb;
+    } else {
+        const int r = (item - p.full_tiles) / p.split;
+        w.part = item - p.full_tiles - r * p.split;
+        w.tile = p.full_tiles + r;
+        w.kb0 = (w.part * p.num_kb) / p.split;
+        w.kb1 = ((w.part + 1) * p.num_kb) / p.split;
+    }
+    return w;
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *addr)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_u64(unsigned long long *addr, unsigned long long v)
+{
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(addr), "l"(v) : "memory");
+}
 
 // Compile-time tile configuration.  Each CTA owns BM = 128 output rows (one
 // TMEM lane per row) and BK = 64 (one 128-byte swizzle row of 16-bit values).
@@ -150,6 +194,30 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
         }
     }
     return true;
+}
+
+// Bounded wait, by every lane, until an earlier part of a split tile has
+// stamped its flag with this launch's epoch.
+__device__ __forceinline__ bool wait_part(const unsigned long long *flag, unsigned long long epoch,
+                                          volatile int *abort_flag, uint64_t timeout_ns, uint32_t peer_abort)
+{
+    if (ld_acquire_u64(flag) == epoch)
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        __nanosleep(100);
+        if (ld_acquire_u64(flag) == epoch)
+            return true;
+        if (*abort_flag)
+            return false;
+        if (global_timer_ns() - t0 > timeout_ns) {
+            *abort_flag = 1;
+            if (peer_abort)
+                st_shared_cluster_u32(peer_abort, 1u);
+            atomicOr(&g_device_error, ERR_SPLIT);
+            return false;
+        }
+    }
 }
 
 template <int DT>
@@ -288,12 +356,13 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
             uint32_t phase = 0;
             bool skip = p.inject_fault != 0 && leader;
             bool ok = true;
-            for (int t = unit; ok && t < p.num_tiles; t += num_units) {
+            for (int item = unit; ok && item < p.num_items; item += num_units) {
+                const WorkItem w = work_item(item, p);
                 int tm, tn;
-                tile_coords(t, p, tm, tn);
+                tile_coords(w.tile, p, tm, tn);
                 const int a_row = tm * CF::TILE_M + static_cast<int>(rank) * CF::BM;
                 const int b_col = tn * CF::BN + static_cast<int>(rank) * CF::BN_LOCAL;
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!wait_bounded<PAIR>(empty_bar(stage), phase ^ 1u, abort_flag, timeout, ERR_PRODUCER,
                                             peer_abort)) {
                         ok = false;
@@ -346,7 +415,8 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int t = unit; ok && t < p.num_tiles; t += num_units) {
+            for (int item = unit; ok && item < p.num_items; item += num_units) {
+                const WorkItem w = work_item(item, p);
                 if (!wait_bounded<PAIR>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, timeout, ERR_MMA_ACC,
                                         peer_abort)) {
                     ok = false;
@@ -354,7 +424,7 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * CF::ACC_COLS);
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!wait_bounded(full_bar(stage), phase, abort_flag, timeout, ERR_MMA_DATA, peer_abort)) {
                         ok = false;
                         break;
@@ -366,7 +436,7 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                     for (int k = 0; k < CF::BK / 16; ++k) {
                         // K step of 16: +32 B inside A's swizzled row, +16 rows (2048 B) of B
                         const uint64_t ad = a_desc + ((32 * k) >> 4), bd = b_desc + ((2048 * k) >> 4);
-                        const uint32_t accumulate = (kb | k) != 0 ? 1u : 0u;
+                        const uint32_t accumulate = (kb != w.kb0 || k != 0) ? 1u : 0u;
                         if constexpr (PAIR)
                             tc_mma_f16_pair(d_tmem, ad, bd, IDESC, accumulate);
                         else
@@ -410,10 +480,13 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
         uint8_t *buf = cstage + (warp - 2) * CF::C_BOX_BYTES;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = unit; t < p.num_tiles; t += num_units) {
+        for (int item = unit; item < p.num_items; item += num_units) {
+            const WorkItem w = work_item(item, p);
             int tm, tn;
-            tile_coords(t, p, tm, tn);
+            tile_coords(w.tile, p, tm, tn);
             const int n0 = tn * CF::BN;
+            const bool split_tile = w.tile >= p.full_tiles;
+            const int r_tail = w.tile - p.full_tiles;
             const int row0 = tm * CF::TILE_M + static_cast<int>(rank) * CF::BM + q * 32;  // this warp's rows
             if (!wait_bounded<PAIR>(tfull_bar(acc), acc_phase, abort_flag, timeout, ERR_EPILOGUE, peer_abort))
                 break;
@@ -443,6 +516,51 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                 const int col0 = n0 + c * 64;
                 if (col0 >= p.N || row0 >= p.M)
                     continue;  // nothing of this chunk lies inside C
+
+                if (split_tile) {
+                    // partial sums of one split tile: [part < split-1][cta][128 rows][BN cols] fp32,
+                    // one flag per (part, cta, lane quarter, chunk)
+                    const size_t slab0 = static_cast<size_t>(r_tail) * (p.split - 1) * CF::CTAS + rank;
+                    const size_t slab_step = CF::CTAS;  // from part to part + 1
+                    const size_t row_off = (static_cast<size_t>(q) * 32 + lane) * CF::BN + c * 64;
+                    const size_t flag_off = static_cast<size_t>(q) * CHUNKS + c;
+                    if (w.part < p.split - 1) {
+                        const size_t slab = slab0 + w.part * slab_step;
+                        float4 *dst = reinterpret_cast<float4 *>(p.partials + slab * CF::BM * CF::BN + row_off);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            __stcg(dst + i, make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                        __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
+                        __threadfence();
+                        __syncwarp();
+                        if (lane == 0)
+                            st_release_u64(p.flags + slab * 4 * CHUNKS + flag_off, p.epoch);
+                        continue;  // the last part stores this chunk of C
+                    }
+                    // last part: sum = part 0 + part 1 + ... + this part, in that order
+                    bool have = true;
+                    for (int part = 0; have && part < p.split - 1; ++part)
+                        have = wait_part(p.flags + (slab0 + part * slab_step) * 4 * CHUNKS + flag_off, p.epoch,
+                                         abort_flag, timeout, peer_abort);
+                    if (!__all_sync(0xffffffffu, have))
+                        continue;  // recorded in the error word; C stays incomplete
+                    const float4 *src0 = reinterpret_cast<const float4 *>(p.partials + slab0 * CF::BM * CF::BN + row_off);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float4 a = __ldcg(src0 + i);
+                        for (int part = 1; part < p.split - 1; ++part) {
+                            const float4 b = __ldcg(src0 + part * slab_step * CF::BM * CF::BN / 4 + i);
+                            a.x += b.x;
+                            a.y += b.y;
+                            a.z += b.z;
+                            a.w += b.w;
+                        }
+                        r[4 * i] = __float_as_uint(a.x + __uint_as_float(r[4 * i]));
+                        r[4 * i + 1] = __float_as_uint(a.y + __uint_as_float(r[4 * i + 1]));
+                        r[4 * i + 2] = __float_as_uint(a.z + __uint_as_float(r[4 * i + 2]));
+                        r[4 * i + 3] = __float_as_uint(a.w + __uint_as_float(r[4 * i + 3]));
+                    }
+                }
 
                 if constexpr (TMA_STORE) {
                     // this warp's staging box: its previous store must have read it

@@ -10,6 +10,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <random>
 #include <unordered_map>
 
 #include "tl_gemm.h"
@@ -75,6 +76,7 @@ struct TableRow {
     int64_t m, n, k;
     int dtype, epi;
     const char *config;
+    int split;  // 1: split the tiles of a short last round; 0: never
 };
 const TableRow kTable[] = {
 #include "config_table.inc"
@@ -132,15 +134,21 @@ int model_config_single(int64_t M, int64_t N, int num_sms)
     return best;
 }
 
-int choose_config(int64_t M, int64_t N, int64_t K, int dtype, int epi, int num_sms)
+// The measured choice for this shape, else the wave model without splitting
+// (on a power-capped B200 the sweep found splitting the last round a loss for
+// most shapes).
+int choose_config(int64_t M, int64_t N, int64_t K, int dtype, int epi, int num_sms, bool *split)
 {
     for (const TableRow &r : kTable) {
         if (r.m == M && r.n == N && r.k == K && r.dtype == dtype && r.epi == epi) {
             const int i = config_index(r.config);
-            if (i >= 0)
+            if (i >= 0) {
+                *split = r.split != 0;
                 return i;
+            }
         }
     }
+    *split = false;
     return model_config(M, N, num_sms);
 }
 
@@ -150,6 +158,8 @@ struct Plan {
     tl_plan pub;
     int64_t lda, ldb;        // row lengths (elements) of the operands the kernel reads
     int64_t a_ws_off, b_ws_off;
+    int64_t partial_off, flag_off;  // split-tile partial sums and their flags
+    int32_t num_kb;
 };
 
 tl_status validate(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N,
@@ -169,6 +179,8 @@ tl_status validate(const void *A, const void *B, const void *bias, void *C, int6
         return TL_ERR_INVALID_ARG;
     if (opt && (opt->inject_fault != 0 && opt->inject_fault != 1))
         return TL_ERR_INVALID_ARG;
+    if (opt && ((opt->no_split != 0 && opt->no_split != 1) || opt->reserved != 0))
+        return TL_ERR_INVALID_ARG;
     if (opt && opt->inject_fault && opt->config > 0 && kConfigs[opt->config - 1].ctas != 1)
         return TL_ERR_UNSUPPORTED;  // the fault hook exists for single-CTA configurations only
     const int64_t lim = 0x7FFFFFFFll;
@@ -179,15 +191,43 @@ tl_status validate(const void *A, const void *B, const void *bias, void *C, int6
     return TL_OK;
 }
 
+// How the tiles of one launch are cut into work items.  Tiles fill whole
+// rounds of `units` (CTAs, or CTA pairs) first; when the last round would be
+// at most half full, each of its tiles is split along K into `split` parts so
+// that the round takes 1/split of a tile's time.  (With fewer tiles than
+// units, the same rule is plain split-K.)  Every unit then holds at most one
+// part of the last round, and all units are resident together, so the last
+// part of a tile can wait for the earlier parts without any risk of waiting
+// on work that is queued behind it.
+void split_tail(int64_t tiles, int64_t units, int64_t num_kb, int32_t *split, int64_t *full_tiles)
+{
+    *split = 1;
+    *full_tiles = tiles;
+    const int64_t rem = tiles % units;
+    if (rem == 0 || num_kb < 8)
+        return;
+    int64_t s = units / rem;
+    if (s > 4)
+        s = 4;
+    if (s > num_kb / 4)
+        s = num_kb / 4;
+    if (s >= 2) {
+        *split = static_cast<int32_t>(s);
+        *full_tiles = tiles - rem;
+    }
+}
+
 tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N,
-                    int64_t K, int dtype, int epi, int num_sms, const tl_gemm_options *opt, Plan *out)
+                    int64_t K, int dtype, int epi, int num_sms, int max_units, const tl_gemm_options *opt,
+                    Plan *out)
 {
     tl_status st = validate(A, B, bias, C, M, N, K, dtype, epi, opt);
     if (st != TL_OK)
         return st;
     if (num_sms <= 0)
         return TL_ERR_INVALID_ARG;
-    int ci = (opt && opt->config > 0) ? opt->config - 1 : choose_config(M, N, K, dtype, epi, num_sms);
+    bool table_split = true;  // a forced configuration splits unless told not to
+    int ci = (opt && opt->config > 0) ? opt->config - 1 : choose_config(M, N, K, dtype, epi, num_sms, &table_split);
     if (opt && opt->inject_fault && kConfigs[ci].ctas != 1)
         ci = model_config_single(M, N, num_sms);
     const ConfigEntry &c = kConfigs[ci];
@@ -203,8 +243,18 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
     const int64_t tiles = static_cast<int64_t>(q.tiles_m) * q.tiles_n;
     if (tiles > 0x7FFFFFFFll)
         return TL_ERR_UNSUPPORTED;
-    const int64_t units = num_sms / c.ctas;
-    q.grid = static_cast<int32_t>((tiles < units ? tiles : units) * c.ctas);
+    int64_t units = num_sms / c.ctas;
+    if (max_units > 0 && max_units < units)
+        units = max_units;
+    p.num_kb = static_cast<int32_t>(ceil_div(K, c.bk));
+    int64_t full_tiles = tiles;
+    int32_t split = 1;
+    if (table_split && !(opt && (opt->inject_fault || opt->no_split)))
+        split_tail(tiles, units, p.num_kb, &split, &full_tiles);
+    const int64_t items = full_tiles + (tiles - full_tiles) * split;
+    q.split = split;
+    q.full_tiles = static_cast<int32_t>(full_tiles);
+    q.grid = static_cast<int32_t>((items < units ? items : units) * c.ctas);
     q.cluster_ctas = c.ctas;
     q.smem_bytes = c.smem_bytes;
     // TMA needs a 16-byte-aligned base and row strides that are multiples of 16 bytes.
@@ -222,6 +272,14 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
     if (q.pad_b) {
         p.b_ws_off = ws;
         ws += ceil_div(K * p.ldb * 2, 256) * 256;
+    }
+    p.partial_off = p.flag_off = -1;
+    if (split > 1) {
+        const int64_t slabs = (tiles - full_tiles) * (split - 1) * c.ctas;  // 128-row partial slabs
+        p.partial_off = ws;
+        ws += ceil_div(slabs * 128 * c.bn * 4, 256) * 256;
+        p.flag_off = ws;
+        ws += ceil_div(slabs * 4 * (c.bn / 64) * 8, 256) * 256;
     }
     q.workspace_bytes = ws;
     *out = p;
@@ -362,9 +420,26 @@ tl_status launch_pad(const void *src, int64_t rows, int64_t cols, void *dst, int
 }
 
 // Launch the GEMM itself with operands the kernel can read through TMA.
+std::atomic<unsigned long long> g_epoch{0};
+
+// A launch stamp no earlier launch of this process has used, starting from a
+// random point so that memory left by another process never matches it.
+unsigned long long next_epoch()
+{
+    unsigned long long e = g_epoch.fetch_add(1) + 1;
+    if (e == 1) {
+        std::random_device rd;
+        const unsigned long long base = ((static_cast<unsigned long long>(rd()) << 32) ^ rd()) | 1ull;
+        unsigned long long expected = 1;
+        g_epoch.compare_exchange_strong(expected, base);
+        e = g_epoch.fetch_add(1) + 1;
+    }
+    return e;
+}
+
 tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *bias, void *C, int64_t M,
                       int64_t N, int64_t K, int dtype, int epi, cudaStream_t stream, DeviceState *d,
-                      const tl_gemm_options *opt)
+                      const tl_gemm_options *opt, void *workspace)
 {
     const ConfigEntry &c = kConfigs[p.pub.config];
     const bool tma_store = !p.pub.direct_store;
@@ -397,6 +472,19 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
     gp.C = static_cast<uint16_t *>(C);
     gp.ldc = N;
     gp.timeout_ns = (opt && opt->timeout_ns) ? opt->timeout_ns : kDefaultTimeoutNs;
+    gp.split = p.pub.split;
+    gp.full_tiles = p.pub.full_tiles;
+    gp.num_items = p.pub.full_tiles + (gp.num_tiles - p.pub.full_tiles) * p.pub.split;
+    gp.partials = nullptr;
+    gp.flags = nullptr;
+    gp.epoch = 0;
+    if (p.pub.split > 1) {
+        if (!workspace)
+            return TL_ERR_INVALID_ARG;
+        gp.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + p.partial_off);
+        gp.flags = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + p.flag_off);
+        gp.epoch = next_epoch();
+    }
 
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];
@@ -411,16 +499,45 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        // persistent pairs: no more clusters than can be resident at once
-        int max_clusters = 0;
-        if ((st = max_active_clusters(d, fn, cfg, &max_clusters)) != TL_OK)
-            return st;
-        if (max_clusters > 0 && p.pub.grid > 2 * max_clusters)
-            cfg.gridDim.x = static_cast<unsigned>(2 * max_clusters);
     }
     if (cudaLaunchKernelEx(&cfg, fn, ta, tb, tc, gp) != cudaSuccess)
         return TL_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ERR_CUDA;
+}
+
+// The plan for this device: for CTA-pair configurations, no more pairs than
+// can be resident at once (the split-tile rule relies on it).
+tl_status device_plan(DeviceState *d, const void *A, const void *B, const void *bias, void *C, int64_t M,
+                      int64_t N, int64_t K, int dtype, int epi, const tl_gemm_options *opt, Plan *p)
+{
+    tl_status st = make_plan(A, B, bias, C, M, N, K, dtype, epi, d->num_sms, 0, opt, p);
+    if (st != TL_OK)
+        return st;
+    const ConfigEntry &c = kConfigs[p->pub.config];
+    if (c.ctas != 2)
+        return TL_OK;
+    KernelFn fn = c.fn[dtype][epi][p->pub.direct_store ? 0 : 1];
+    if ((st = raise_smem_limit(d, fn, c.smem_bytes)) != TL_OK)
+        return st;
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(static_cast<unsigned>(c.threads), 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(c.smem_bytes);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int max_clusters = 0;
+    if ((st = max_active_clusters(d, fn, cfg, &max_clusters)) != TL_OK)
+        return st;
+    if (max_clusters <= 0)
+        return TL_ERR_CUDA;
+    if (max_clusters < d->num_sms / 2)
+        st = make_plan(A, B, bias, C, M, N, K, dtype, epi, d->num_sms, max_clusters, opt, p);
+    return st;
 }
 
 tl_status gemm_impl(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N, int64_t K,
@@ -435,11 +552,11 @@ tl_status gemm_impl(const void *A, const void *B, const void *bias, void *C, int
     if (d->cc_major != 10)
         return TL_ERR_UNSUPPORTED;
     Plan p;
-    if ((st = make_plan(A, B, bias, C, M, N, K, dtype, epi, d->num_sms, opt, &p)) != TL_OK)
+    if ((st = device_plan(d, A, B, bias, C, M, N, K, dtype, epi, opt, &p)) != TL_OK)
         return st;
 
     if (p.pub.workspace_bytes == 0)
-        return launch_gemm(p, A, B, bias, C, M, N, K, dtype, epi, stream, d, opt);
+        return launch_gemm(p, A, B, bias, C, M, N, K, dtype, epi, stream, d, opt, nullptr);
 
     if ((st = ensure_pool(d)) != TL_OK)
         return st;
@@ -458,7 +575,7 @@ tl_status gemm_impl(const void *A, const void *B, const void *bias, void *C, int
         b_use = dst;
     }
     if (st == TL_OK)
-        st = launch_gemm(p, a_use, b_use, bias, C, M, N, K, dtype, epi, stream, d, opt);
+        st = launch_gemm(p, a_use, b_use, bias, C, M, N, K, dtype, epi, stream, d, opt, ws);
     if (cudaFreeAsync(ws, stream) != cudaSuccess && st == TL_OK)
         st = TL_ERR_CUDA;
     return st;
@@ -544,13 +661,15 @@ tl_status gemm_noalloc_impl(const void *A, const void *B, const void *bias, void
     if ((st = noalloc_setup(d, &scratch)) != TL_OK)
         return st;
     Plan p;
-    if ((st = make_plan(A, B, bias, C, M, N, K, dtype, epi, d->num_sms, nullptr, &p)) != TL_OK)
+    if ((st = device_plan(d, A, B, bias, C, M, N, K, dtype, epi, nullptr, &p)) != TL_OK)
         return st;
     if (p.pub.workspace_bytes == 0)
-        return launch_gemm(p, A, B, bias, C, M, N, K, dtype, epi, stream, d, nullptr);
+        return launch_gemm(p, A, B, bias, C, M, N, K, dtype, epi, stream, d, nullptr, nullptr);
     if (static_cast<uint64_t>(p.pub.workspace_bytes) > TL_NOALLOC_SCRATCH_BYTES)
         return TL_ERR_SCRATCH_LIMIT;
-    // the padded copies overwrite every byte of scratch that the GEMM reads
+    // the padded copies overwrite every byte of scratch that the GEMM reads; the
+    // split-tile partials are written before they are read, under flags stamped
+    // with this launch's own epoch
     const void *a_use = A, *b_use = B;
     if (p.pub.pad_a) {
         void *dst = static_cast<uint8_t *>(scratch) + p.a_ws_off;
@@ -564,7 +683,7 @@ tl_status gemm_noalloc_impl(const void *A, const void *B, const void *bias, void
             return st;
         b_use = dst;
     }
-    return launch_gemm(p, a_use, b_use, bias, C, M, N, K, dtype, epi, stream, d, nullptr);
+    return launch_gemm(p, a_use, b_use, bias, C, M, N, K, dtype, epi, stream, d, nullptr, scratch);
 }
 
 } // namespace
@@ -621,7 +740,7 @@ tl_status tl_gemm_plan(const void *A, const void *B, const void *bias, void *C, 
         num_sms = d->num_sms;
     }
     tl::Plan p;
-    st = tl::make_plan(A, B, bias, C, M, N, K, dtype, epi, num_sms, options, &p);
+    st = tl::make_plan(A, B, bias, C, M, N, K, dtype, epi, num_sms, 0, options, &p);
     if (st == TL_OK)
         *plan = p.pub;
     return st;

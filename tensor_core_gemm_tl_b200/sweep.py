@@ -28,7 +28,7 @@ TABLE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc", "config
 L2_BYTES = 126 * 1024 * 1024
 
 
-def time_config(w, config, launches, warmup, seed=0):
+def time_config(w, config, launches, warmup, seed=0, no_split=False):
     import torch
     import tensor_core_gemm_tl_b200 as tg
     A_bits, B_bits, bias_bits = wl.make_inputs(w, seed)
@@ -47,13 +47,13 @@ def time_config(w, config, launches, warmup, seed=0):
     stream = torch.cuda.current_stream()
     for i in range(warmup):
         A, B, C = sets[i % nsets]
-        tg.gemm(A, B, bias, epilogue=epi, out=C, config=config, stream=stream)
+        tg.gemm(A, B, bias, epilogue=epi, out=C, config=config, stream=stream, no_split=no_split)
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
     for i, (s, e) in enumerate(ev):
         A, B, C = sets[i % nsets]
         s.record(stream)
-        tg.gemm(A, B, bias, epilogue=epi, out=C, config=config, stream=stream)
+        tg.gemm(A, B, bias, epilogue=epi, out=C, config=config, stream=stream, no_split=no_split)
         e.record(stream)
     torch.cuda.synchronize()
     if tg.check_device() != 0:
@@ -73,7 +73,7 @@ def shapes(which):
 
 def write_table(best_rows):
     """Write csrc/config_table.inc from the fastest record per shape."""
-    lines = ["// Kernel configuration per measured shape: {M, N, K, dtype, epilogue, config}.",
+    lines = ["// Kernel configuration per measured shape: {M, N, K, dtype, epilogue, config, split}.",
              "// Written by tensor_core_gemm_tl_b200/sweep.py from timings on a B200; shapes",
              "// not listed fall back to the wave model in tl_gemm.cu."]
     seen = set()
@@ -83,9 +83,10 @@ def write_table(best_rows):
             continue
         seen.add(key)
         dt = 0 if r["dtype"] == "f16" else 1
-        lines.append(f'{{{r["M"]}, {r["N"]}, {r["K"]}, {dt}, {r["epi"]}, "{r["config"]}"}},'
+        split = int(r.get("split", 0))
+        lines.append(f'{{{r["M"]}, {r["N"]}, {r["K"]}, {dt}, {r["epi"]}, "{r["config"]}", {split}}},'
                      f'  // {r["tflops"]} TFLOP/s')
-    lines.append('{0, 0, 0, -1, -1, ""},  // sentinel, never matches')
+    lines.append('{0, 0, 0, -1, -1, "", 0},  // sentinel, never matches')
     with open(TABLE, "w") as f:
         f.write("\n".join(lines) + "\n")
     print("wrote", TABLE, file=sys.stderr)
@@ -125,14 +126,17 @@ def main(argv=None):
     for w in todo:
         best = None
         for k in range(1, tg.tl_num_configs() + 1):
-            med, mean = time_config(w, k, a.launches, a.warmup)
-            tflops = w.flops / (med / 1e3) / 1e12
-            rec = {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "dtype": wl.DTYPE_NAMES[w.dtype],
-                   "epi": w.epi, "config": tg.tl_config_name(k - 1), "median_ms": round(med, 5),
-                   "mean_ms": round(mean, 5), "tflops": round(tflops, 1)}
-            print(json.dumps(rec), flush=True)
-            if best is None or med < best[0]:
-                best = (med, rec)
+            p = tg.plan(w.M, w.N, w.K, w.dtype, "bias_gelu" if w.epi else None,
+                        num_sms=torch.cuda.get_device_properties(0).multi_processor_count, config=k)
+            for split in ((1, 0) if p["split"] > 1 else (0,)):
+                med, mean = time_config(w, k, a.launches, a.warmup, no_split=not split)
+                tflops = w.flops / (med / 1e3) / 1e12
+                rec = {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "dtype": wl.DTYPE_NAMES[w.dtype],
+                       "epi": w.epi, "config": tg.tl_config_name(k - 1), "split": split,
+                       "median_ms": round(med, 5), "mean_ms": round(mean, 5), "tflops": round(tflops, 1)}
+                print(json.dumps(rec), flush=True)
+                if best is None or med < best[0]:
+                    best = (med, rec)
         rows.append(best[1])
     if a.write:
         write_table(rows)

@@ -90,7 +90,7 @@ def test_no_device_is_a_cuda_error_not_a_crash():
 def test_plan_aligned_headline_shape():
     p = tg.plan(4096, 4096, 4096, tg.TL_F16, None, num_sms=148)
     assert p["pad_a"] == 0 and p["pad_b"] == 0 and p["direct_store"] == 0
-    assert p["workspace_bytes"] == 0
+    assert (p["workspace_bytes"] == 0) == (p["split"] == 1)  # only split tiles need a workspace
     assert p["tiles_m"] == 4096 // p["block_m"] and p["tiles_n"] == 4096 // p["block_n"]
     assert p["grid"] == min(148 // p["cluster_ctas"], p["tiles_m"] * p["tiles_n"]) * p["cluster_ctas"]
     assert p["smem_bytes"] <= 232448
@@ -160,3 +160,34 @@ def test_torch_wrapper_rejects_bad_tensors():
         tg.gemm(A, torch.zeros(5, 4, dtype=torch.float16))
     with pytest.raises(ValueError):
         tg._epi_code("relu")
+
+
+@pytest.mark.parametrize("M,N,K,config,split,full", [
+    (4096, 4096, 4096, 4, 2, 222),   # 256 pair tiles on 74 pairs: 3 rounds + 34 tiles split in two
+    (4096, 4096, 4096, 1, 2, 444),   # 512 single-CTA tiles on 148: 68 left over, split in two
+    (1024, 1024, 2048, 1, 4, 0),     # 32 tiles on 148 SMs: plain split-K, 4 parts
+    (1024, 1024, 1024, 4, 4, 0),     # 16 pair tiles on 74 pairs: 4 parts
+    (1280, 1536, 1024, 4, 2, 0),     # 30 tiles: 2 parts
+    (1024, 1280, 1536, 4, 3, 0),     # 20 tiles: 3 parts
+    (2560, 640, 1024, 3, 2, 148),    # 200 tiles of 128 x 64: one full round, 52 tiles split
+    (8192, 16384, 4096, 4, 1, 2048), # last round 50 of 74: not worth splitting
+    (700, 900, 333, 4, 1, 12),       # too few k blocks to split
+])
+def test_plan_splits_only_a_short_last_round(M, N, K, config, split, full):
+    p = tg.plan(M, N, K, tg.TL_BF16, None, num_sms=148, config=config)
+    tiles = p["tiles_m"] * p["tiles_n"]
+    assert p["split"] == split and p["full_tiles"] == full
+    units = 148 // p["cluster_ctas"]
+    items = p["full_tiles"] + (tiles - p["full_tiles"]) * p["split"]
+    assert p["grid"] == min(items, units) * p["cluster_ctas"]
+    if split > 1:
+        # every unit holds at most one part of the last round
+        assert (tiles - full) * split <= units and full % units == 0
+        assert p["workspace_bytes"] >= (tiles - full) * (split - 1) * p["cluster_ctas"] * 128 * p["block_n"] * 4
+    else:
+        assert p["workspace_bytes"] == 0 or p["pad_a"] or p["pad_b"]
+
+
+def test_fault_hook_disables_the_split():
+    st, p = tg.tl_gemm_plan(P, P, 0, P, 1024, 1024, 2048, 0, 0, 148, tg.Options(config=1, inject_fault=1))
+    assert st == 0 and p.split == 1

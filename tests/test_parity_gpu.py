@@ -107,6 +107,33 @@ def test_every_config_vs_oracle(config, epi):
         compare(C, ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
 
 
+SPLIT_CASES = [
+    # (M, N, K, config, dtype, epilogue): the tiles of a short last round are
+    # split along K and their partial sums added by the last part
+    (1024, 1024, 2048, 1, wl.BF16, wl.EPI_BIAS_GELU),   # 4 parts, single CTA
+    (1024, 1024, 1024, 4, wl.F16, wl.EPI_NONE),         # 4 parts, CTA pairs
+    (1280, 1536, 1024, 4, wl.BF16, wl.EPI_BIAS_GELU),   # 2 parts, CTA pairs
+    (1024, 1280, 1536, 4, wl.F16, wl.EPI_BIAS_GELU),    # 3 parts, CTA pairs
+    (2560, 640, 1024, 3, wl.BF16, wl.EPI_NONE),         # a full round, then 2 parts
+    (1000, 1000, 2000, 1, wl.F16, wl.EPI_BIAS_GELU),    # ragged M, N tails, 4 parts
+    (1001, 999, 2051, 4, wl.BF16, wl.EPI_BIAS_GELU),    # padded A and B, element stores, 4 parts
+]
+
+
+@pytest.mark.parametrize("M,N,K,config,dt,epi", SPLIT_CASES)
+def test_split_tiles_vs_oracle(M, N, K, config, dt, epi):
+    import tensor_core_gemm_tl_b200 as m
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    p = m.plan(M, N, K, dt, "bias_gelu" if epi else None, num_sms=sms, config=config)
+    A, B, bias = inputs(M, N, K, dt, epi, seed=M + N + K)
+    ref = oracle.gemm(A, B, bias, dt, epi)
+    C1 = run_library(A, B, bias, dt, epi, config=config)
+    compare(C1, ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
+    C2 = run_library(A, B, bias, dt, epi, config=config)
+    assert np.array_equal(C1, C2), "split tiles must be bit-reproducible"
+    assert p["split"] > 1 or sms != 148
+
+
 @pytest.mark.parametrize("offsets", [(1, 0, 0, 0), (0, 3, 0, 0), (0, 0, 1, 0), (0, 0, 0, 5), (2, 1, 3, 7)])
 def test_unaligned_bases(offsets):
     """Bases 2-byte but not 16-byte aligned: padded operand copies, the scalar
