@@ -161,7 +161,8 @@ TL_API tl_status tl_gemm_ex(const void *A, const void *B, const void *bias, void
  * early, C is incomplete), TL_ERR_CUDA if the synchronization failed, TL_OK
  * otherwise.  `detail`, if not NULL, receives the raw error word (which waits
  * gave up: bit 0 copy warp, bit 1 MMA warp on data, bit 2 MMA warp on the
- * accumulator, bit 3 epilogue warps, bit 4 final drain).
+ * accumulator, bit 3 epilogue warps, bit 4 final drain, bit 5 the last K part
+ * of a split tile waiting for an earlier part).
  */
 TL_API tl_status tl_check_device(tl_stream stream, uint32_t *detail);
 

@@ -345,6 +345,11 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
     const uint64_t timeout = p.timeout_ns;
+    // Everything above touches only this CTA's own state, so it may overlap the
+    // previous kernel on the stream; global memory is read and written only
+    // after that kernel has completed.
+    grid_dependency_wait();
+    grid_launch_dependents();
 
     // Last fill issued per stage (bit s set) and its phase parity: on an abort,
     // every copy issued is waited for before the CTA exits.

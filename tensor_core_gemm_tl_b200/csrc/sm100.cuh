@@ -227,6 +227,22 @@ __host__ __device__ constexpr uint32_t mma_idesc_f16(int bf16, int m, int n, int
 
 } // namespace tl
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Wait until the grids this one depends on (the previous kernels on the
+// stream) have completed and their memory is visible; a no-op when the launch
+// did not allow overlap.
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next kernel on the stream to begin launching (its own
+// grid_dependency_wait still waits for this grid to complete).
+__device__ __forceinline__ void grid_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- CTA pairs (clusters of 2)
 namespace tl {
 

@@ -487,18 +487,23 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
     }
 
     cudaLaunchConfig_t cfg{};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cfg.gridDim = dim3(static_cast<unsigned>(p.pub.grid), 1, 1);
     cfg.blockDim = dim3(static_cast<unsigned>(c.threads), 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(c.smem_bytes);
     cfg.stream = stream;
+    // The kernel's set-up may overlap the previous kernel on the stream: it
+    // waits for that kernel (griddepcontrol.wait) before touching global memory.
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (c.ctas == 2) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = 2;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
     }
     if (cudaLaunchKernelEx(&cfg, fn, ta, tb, tc, gp) != cudaSuccess)
         return TL_ERR_CUDA;
