@@ -31,6 +31,8 @@ F16 = 0
 BF16 = 1
 EPI_NONE = 0
 EPI_BIAS_GELU = 1
+EPI_BIAS = 2
+EPI_GELU = 3
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
@@ -91,10 +93,10 @@ def _ptr(a):
 def _check_shapes(A, B, bias, epi):
     if A.ndim != 2 or B.ndim != 2 or A.shape[1] != B.shape[0]:
         raise ValueError(f"shapes A{A.shape} B{B.shape} do not chain")
-    if epi == EPI_BIAS_GELU:
+    if epi in (EPI_BIAS_GELU, EPI_BIAS):
         if bias is None or bias.shape != (B.shape[1],):
-            raise ValueError("the bias+GELU epilogue needs a bias of length N")
-    elif epi != EPI_NONE:
+            raise ValueError("this epilogue needs a bias of length N")
+    elif epi not in (EPI_NONE, EPI_GELU):
         raise ValueError(f"unknown epilogue {epi}")
 
 

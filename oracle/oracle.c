@@ -17,7 +17,8 @@
  *   - TileLang GPU kernel design article, paragraph 5 (fused GEMM epilogue):
  *     bias add, then GELU, applied to the accumulator before the one write
  *     of the output.  Read as: per-column bias (length N), added
- *     first; GELU in its exact form 0.5 x (1 + erf(x / sqrt 2)).
+ *     first; GELU in its exact form 0.5 x (1 + erf(x / sqrt 2)).  The bias-only
+ *     and GELU-only epilogues are the same steps with one of them left out.
  *
  * Plain definition, no blocking, no reordering: for each output element the
  * sum over k runs k = 0 .. K-1 in order, in double.  The result is kept in
@@ -35,6 +36,8 @@
 #define ORACLE_BF16 1
 #define ORACLE_EPI_NONE 0
 #define ORACLE_EPI_BIAS_GELU 1
+#define ORACLE_EPI_BIAS 2
+#define ORACLE_EPI_GELU 3
 
 /* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits.
  * Normal: (1024 + f) * 2^(e - 25).  Subnormal (e = 0): f * 2^-24.          */
@@ -106,7 +109,7 @@ int oracle_gemm_rows(int64_t M, int64_t N, int64_t K,
     for (int64_t r = 0; r < nrows; ++r)
         if (rows[r] < 0 || rows[r] >= M)
             return -1;
-    if (epi == ORACLE_EPI_BIAS_GELU && bias == NULL)
+    if ((epi == ORACLE_EPI_BIAS_GELU || epi == ORACLE_EPI_BIAS) && bias == NULL)
         return -1;
 
     /* B decoded once; every row reads all of it. */
@@ -132,6 +135,12 @@ int oracle_gemm_rows(int64_t M, int64_t N, int64_t K,
         if (epi == ORACLE_EPI_BIAS_GELU)
             for (int64_t j = 0; j < N; ++j)
                 c[j] = oracle_gelu(c[j] + decode(bias[j], dtype));
+        else if (epi == ORACLE_EPI_BIAS)
+            for (int64_t j = 0; j < N; ++j)
+                c[j] = c[j] + decode(bias[j], dtype);
+        else if (epi == ORACLE_EPI_GELU)
+            for (int64_t j = 0; j < N; ++j)
+                c[j] = oracle_gelu(c[j]);
     }
     free(Bd);
     return 0;
@@ -161,7 +170,7 @@ int oracle_gemm_points(int64_t M, int64_t N, int64_t K,
     for (int64_t p = 0; p < npts; ++p)
         if (ii[p] < 0 || ii[p] >= M || jj[p] < 0 || jj[p] >= N)
             return -1;
-    if (epi == ORACLE_EPI_BIAS_GELU && bias == NULL)
+    if ((epi == ORACLE_EPI_BIAS_GELU || epi == ORACLE_EPI_BIAS) && bias == NULL)
         return -1;
     int64_t p;
 #pragma omp parallel for schedule(static)
@@ -172,6 +181,10 @@ int oracle_gemm_points(int64_t M, int64_t N, int64_t K,
             s += decode(A[i * K + k], dtype) * decode(B[k * N + j], dtype);
         if (epi == ORACLE_EPI_BIAS_GELU)
             s = oracle_gelu(s + decode(bias[j], dtype));
+        else if (epi == ORACLE_EPI_BIAS)
+            s = s + decode(bias[j], dtype);
+        else if (epi == ORACLE_EPI_GELU)
+            s = oracle_gelu(s);
         out[p] = s;
     }
     return 0;

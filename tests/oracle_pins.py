@@ -256,20 +256,45 @@ def pin_power_of_two_scaling(orc, seed=17):
 
 def pin_rows_and_points(orc, seed=19):
     """The row-subset and single-point entry points agree bit for bit with the
-    whole product, in both epilogue modes."""
+    whole product, in every epilogue mode."""
     rng = np.random.default_rng(seed)
     M, N, K = 23, 31, 45
     for dt in (F16, BF16):
         A = rand_bits(rng, (M, K), dt, 1.0)
         B = rand_bits(rng, (K, N), dt, 1.0)
         bias = rand_bits(rng, (N,), dt, 0.5, "normal")
-        for epi, b in ((EPI_NONE, None), (EPI_BIAS_GELU, bias)):
+        for epi, b in ((EPI_NONE, None), (EPI_BIAS_GELU, bias), (wl.EPI_BIAS, bias), (wl.EPI_GELU, None)):
             full = orc.gemm(A, B, b, dt, epi)
             rows = np.array([22, 0, 5, 5, 17])
             assert np.array_equal(orc.gemm(A, B, b, dt, epi, rows=rows), full[rows])
             ii = rng.integers(0, M, 50)
             jj = rng.integers(0, N, 50)
             assert np.array_equal(orc.gemm_points(A, B, b, dt, epi, ii, jj), full[ii, jj])
+
+
+def pin_bias_only_and_gelu_only(orc, seed=29):
+    """Bias-only: numpy's fp64 matmul plus the bias row.  GELU-only with A = I:
+    C = GELU(B) elementwise, checked on the standard normal table."""
+    rng = np.random.default_rng(seed)
+    for dt, (M, N, K) in ((F16, (9, 17, 33)), (BF16, (12, 8, 40))):
+        A = rand_bits(rng, (M, K), dt, 1.0)
+        B = rand_bits(rng, (K, N), dt, 1.0)
+        bias = rand_bits(rng, (N,), dt, 1.0, "normal")
+        Af = wl.bits_to_float32(A, dt).astype(np.float64)
+        Bf = wl.bits_to_float32(B, dt).astype(np.float64)
+        ref = Af @ Bf + wl.bits_to_float32(bias, dt).astype(np.float64)[None, :]
+        got = orc.gemm(A, B, bias, dt, wl.EPI_BIAS)
+        assert np.all(np.abs(got - ref) <= 2 * K * U53 * (np.abs(Af) @ np.abs(Bf) + 1) + 1e-300)
+    xs, ps = load_phi_table()
+    xs_all = np.concatenate([xs, -xs[1:]])
+    phi_all = np.concatenate([ps, 1.0 - ps[1:]])
+    for dt in (F16, BF16):
+        n = xs_all.size
+        A = wl.round_to_bits(np.eye(n, dtype=np.float32), dt)
+        B = wl.round_to_bits(np.tile(xs_all.astype(np.float32), (n, 1)), dt)  # every row = the table
+        got = orc.gemm(A, B, None, dt, wl.EPI_GELU)
+        expect = (xs_all * phi_all)[None, :]
+        assert np.all(np.abs(got - expect) <= 6e-11 * np.maximum(np.abs(xs_all), 1.0)[None, :])
 
 
 # ---------------------------------------------------------------- GELU alone
@@ -316,5 +341,5 @@ ALL_PINS = [
     pin_exact_bruteforce_epilogue, pin_vs_numpy_matmul, pin_identity, pin_row_sums,
     pin_all_ones, pin_zero_B_gelu_table, pin_bias_then_gelu, pin_transpose,
     pin_power_of_two_scaling, pin_rows_and_points, pin_gelu_table, pin_gelu_invariants,
-    pin_gelu_tail_relative,
+    pin_gelu_tail_relative, pin_bias_only_and_gelu_only,
 ]

@@ -30,6 +30,9 @@ MUTANTS = [
      "c[j] = oracle_gelu(c[j]) + decode(bias[j], dtype);"),
     ("bias_by_row", "c[j] = oracle_gelu(c[j] + decode(bias[j], dtype));",
      "c[j] = oracle_gelu(c[j] + decode(bias[i % N], dtype));"),
+    ("bias_only_drops_bias", "c[j] = c[j] + decode(bias[j], dtype);", "c[j] = c[j];"),
+    ("gelu_only_adds_bias", "            s = oracle_gelu(s);", "            s = oracle_gelu(s + 1.0);"),
+    ("gelu_only_rows_skip_gelu", "                c[j] = oracle_gelu(c[j]);", "                c[j] = c[j];"),
     ("f16_exponent_bias", "v = ldexp((double)(f + 1024), e - 25);", "v = ldexp((double)(f + 1024), e - 24);"),
     ("f16_subnormal_as_normal", "v = ldexp((double)f, -24);", "v = ldexp((double)(f + 1024), -25);"),
     ("bf16_exponent_bias", "v = ldexp((double)(f + 128), e - 134);", "v = ldexp((double)(f + 128), e - 133);"),
