@@ -47,8 +47,10 @@ extern "C" {
 typedef enum { TL_F16 = 0, TL_BF16 = 1 } tl_dtype;
 
 typedef enum {
-    TL_EPI_NONE = 0,      /* C = A.B                                   */
-    TL_EPI_BIAS_GELU = 1  /* C = GELU(A.B + bias[col]), exact erf GELU */
+    TL_EPI_NONE = 0,       /* C = A.B                                   */
+    TL_EPI_BIAS_GELU = 1,  /* C = GELU(A.B + bias[col]), exact erf GELU */
+    TL_EPI_BIAS = 2,       /* C = A.B + bias[col]                       */
+    TL_EPI_GELU = 3        /* C = GELU(A.B)                             */
 } tl_epilogue;
 
 typedef enum {
@@ -70,8 +72,8 @@ typedef void *tl_stream;
  *
  *   A     device pointer, M x K, row-major (leading dimension K), `dtype`
  *   B     device pointer, K x N, row-major (leading dimension N), `dtype`
- *   bias  device pointer to N values of `dtype`; required when
- *         epi == TL_EPI_BIAS_GELU, ignored (may be NULL) otherwise
+ *   bias  device pointer to N values of `dtype`; required when epi is
+ *         TL_EPI_BIAS_GELU or TL_EPI_BIAS, ignored (may be NULL) otherwise
  *   C     device pointer, M x N, row-major (leading dimension N), `dtype`;
  *         written, never read.  C must not overlap A, B or bias (not checked).
  *   M, N, K   sizes, each in [1, 2^31 - 1]
@@ -144,7 +146,9 @@ typedef struct {
                              returns with TL_ERR_DEVICE_TIMEOUT recorded          */
     uint64_t timeout_ns;  /* bound on every wait inside the kernel; 0 = 10 s     */
     int32_t no_split;     /* 1: never split the tiles of a short last round      */
-    int32_t reserved;     /* must be 0                                           */
+    int32_t b_layout;     /* 0: B is K x N row-major (leading dimension N);
+                             1: B is given transposed, N x K row-major (leading
+                             dimension K) -- the layout of a weight W in A.W^T */
 } tl_gemm_options;
 
 /* tl_gemm with options (NULL options == tl_gemm).  Same arguments and errors;

@@ -13,7 +13,8 @@ or library fallback.
 from __future__ import annotations
 
 from ._binding import (  # noqa: F401
-    LIB_PATH, Options, Plan, Status, TLError, TL_BF16, TL_EPI_BIAS_GELU, TL_EPI_NONE, TL_F16,
+    LIB_PATH, Options, Plan, Status, TLError, TL_BF16, TL_EPI_BIAS, TL_EPI_BIAS_GELU, TL_EPI_GELU,
+    TL_EPI_NONE, TL_F16,
     SIGNATURES, tl_check_device, tl_config_name, tl_gemm, tl_gemm_ex, tl_gemm_noalloc, tl_gemm_plan, tl_num_configs,
     tl_status_string, tl_version,
 )
@@ -22,6 +23,7 @@ __all__ = [
     "gemm", "check_device", "plan", "configs", "Options", "Plan", "Status", "TLError",
     "tl_gemm", "tl_gemm_ex", "tl_gemm_noalloc", "tl_check_device", "tl_gemm_plan", "tl_num_configs", "tl_config_name",
     "tl_status_string", "tl_version", "TL_F16", "TL_BF16", "TL_EPI_NONE", "TL_EPI_BIAS_GELU",
+    "TL_EPI_BIAS", "TL_EPI_GELU",
 ]
 
 
@@ -34,26 +36,34 @@ def _dtype_code(t):
     raise TypeError(f"expected float16 or bfloat16, got {t.dtype}")
 
 
+_EPILOGUES = {None: TL_EPI_NONE, "none": TL_EPI_NONE, "bias_gelu": TL_EPI_BIAS_GELU,
+              "bias+gelu": TL_EPI_BIAS_GELU, "bias": TL_EPI_BIAS, "gelu": TL_EPI_GELU}
+
+
 def _epi_code(epilogue):
-    if epilogue in (None, "none", TL_EPI_NONE):
-        return TL_EPI_NONE
-    if epilogue in ("bias_gelu", "bias+gelu", TL_EPI_BIAS_GELU):
-        return TL_EPI_BIAS_GELU
+    if isinstance(epilogue, int) and epilogue in (TL_EPI_NONE, TL_EPI_BIAS_GELU, TL_EPI_BIAS, TL_EPI_GELU):
+        return epilogue
+    if epilogue in _EPILOGUES:
+        return _EPILOGUES[epilogue]
     raise ValueError(f"unknown epilogue {epilogue!r}")
 
 
 def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0, timeout_ns: int = 0,
-         no_split: bool = False):
-    """C = epilogue(A @ B) for row-major CUDA tensors A (M x K) and B (K x N).
+         no_split: bool = False, b_transposed: bool = False):
+    """C = epilogue(A @ B) for row-major CUDA tensors A (M x K) and B (K x N),
+    or B given as N x K (``b_transposed=True``: C = epilogue(A @ B.T), the
+    layout of a linear layer's weight).
 
-    ``epilogue`` is None / "none" or "bias_gelu" (``bias`` of length N is then
-    required).  ``out`` (M x N, same dtype) is written if given, else
-    allocated.  Runs asynchronously on ``stream`` (default: torch's current
-    stream).  ``config`` = k > 0 forces kernel configuration k - 1.
+    ``epilogue`` is None / "none", "bias_gelu", "bias" or "gelu" (``bias`` of
+    length N for the first two; default "bias_gelu" when a bias is given).
+    ``out`` (M x N, same dtype) is written if given, else allocated.  Runs
+    asynchronously on ``stream`` (default: torch's current stream).
+    ``config`` = k > 0 forces kernel configuration k - 1.
     """
     import torch
     epi = _epi_code(epilogue if epilogue is not None else ("bias_gelu" if bias is not None else None))
-    if A.dim() != 2 or B.dim() != 2 or A.shape[1] != B.shape[0]:
+    k_of_b = B.shape[1] if (b_transposed and B.dim() == 2) else (B.shape[0] if B.dim() == 2 else None)
+    if A.dim() != 2 or B.dim() != 2 or A.shape[1] != k_of_b:
         raise ValueError(f"shapes {tuple(A.shape)} and {tuple(B.shape)} do not chain")
     for name, t in (("A", A), ("B", B)):
         if not t.is_cuda or not t.is_contiguous():
@@ -62,22 +72,23 @@ def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0,
     if B.dtype != A.dtype:
         raise TypeError("A and B must have the same dtype")
     M, K = A.shape
-    N = B.shape[1]
-    if epi == TL_EPI_BIAS_GELU:
+    N = B.shape[0] if b_transposed else B.shape[1]
+    if epi in (TL_EPI_BIAS_GELU, TL_EPI_BIAS):
         if bias is None or bias.shape != (N,) or bias.dtype != A.dtype or not bias.is_cuda or not bias.is_contiguous():
-            raise ValueError("bias_gelu needs a contiguous CUDA bias of length N in the input dtype")
+            raise ValueError("this epilogue needs a contiguous CUDA bias of length N in the input dtype")
     if out is None:
         out = torch.empty((M, N), dtype=A.dtype, device=A.device)
     elif out.shape != (M, N) or out.dtype != A.dtype or not out.is_contiguous() or not out.is_cuda:
         raise ValueError("out must be a contiguous CUDA tensor of shape (M, N) and the input dtype")
     s = stream if stream is not None else torch.cuda.current_stream(A.device)
     with torch.cuda.device(A.device):
-        if config or timeout_ns or no_split:
-            opt = Options(config=config, inject_fault=0, timeout_ns=timeout_ns, no_split=int(no_split))
-            st = tl_gemm_ex(A.data_ptr(), B.data_ptr(), bias.data_ptr() if bias is not None else 0,
+        if config or timeout_ns or no_split or b_transposed:
+            opt = Options(config=config, inject_fault=0, timeout_ns=timeout_ns, no_split=int(no_split),
+                          b_layout=int(bool(b_transposed)))
+            st = tl_gemm_ex(A.data_ptr(), B.data_ptr(), bias.data_ptr() if bias is not None and epi in (1, 2) else 0,
                             out.data_ptr(), M, N, K, dt, epi, s.cuda_stream, opt)
         else:
-            st = tl_gemm(A.data_ptr(), B.data_ptr(), bias.data_ptr() if bias is not None else 0,
+            st = tl_gemm(A.data_ptr(), B.data_ptr(), bias.data_ptr() if bias is not None and epi in (1, 2) else 0,
                          out.data_ptr(), M, N, K, dt, epi, s.cuda_stream)
     if st != 0:
         raise TLError(st, "tl_gemm")
@@ -94,12 +105,14 @@ def check_device(stream=None) -> int:
     return word
 
 
-def plan(M, N, K, dtype=TL_F16, epilogue=None, num_sms=148, config=0, ptrs=(256, 256, 256, 256)) -> dict:
+def plan(M, N, K, dtype=TL_F16, epilogue=None, num_sms=148, config=0, ptrs=(256, 256, 256, 256),
+         b_transposed=False, no_split=False) -> dict:
     """The host plan for a call (no GPU needed): config, grid, padding, store path."""
     a, b, bias, c = ptrs
     epi = _epi_code(epilogue)
-    opt = Options(config=config) if config else None
-    st, p = tl_gemm_plan(a, b, bias if epi else 0, c, M, N, K, dtype, epi, num_sms, opt)
+    opt = Options(config=config, b_layout=int(b_transposed), no_split=int(no_split)) \
+        if (config or b_transposed or no_split) else None
+    st, p = tl_gemm_plan(a, b, bias if epi in (1, 2) else 0, c, M, N, K, dtype, epi, num_sms, opt)
     if st != 0:
         raise TLError(st, "tl_gemm_plan")
     d = p.as_dict()

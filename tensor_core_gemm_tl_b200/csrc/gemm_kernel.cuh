@@ -54,6 +54,8 @@ struct GemmParams {
     int32_t tiles_m, tiles_n, num_tiles, num_kb;
     int32_t group_m;         // output-tile rows per rasterisation group
     const uint16_t *bias;    // N values of the input dtype (epilogue only)
+    int32_t epi_bias;        // fused epilogue: add bias[col]
+    int32_t epi_gelu;        // fused epilogue: apply exact GELU
     int32_t bias_vec16;      // bias is 16-byte aligned: load 8 values per access
     int32_t inject_fault;    // test hook: skip the first stage's copy
     uint16_t *C;             // direct-store path only
@@ -278,7 +280,10 @@ __device__ __forceinline__ float gelu_erf(float x)
     return x * (x >= 0.0f ? 1.0f - q : q);
 }
 
-template <class CF, int DT, int EPI, bool TMA_STORE>
+// EPI = 0: C = A.B.  EPI = 1: the fused epilogue, its steps chosen at run
+// time (bias add and/or GELU).  BT: B is given as N x K row-major (K-major
+// operand) instead of K x N.
+template <class CF, int DT, int EPI, bool TMA_STORE, bool BT>
 __global__ void __launch_bounds__(CF::THREADS, 1)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_c, const GemmParams p)
@@ -385,16 +390,25 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                             if (leader)
                                 mbar_arrive_expect_tx(fb, CF::TX_BYTES);
                             tma_load_2d_pair(sa, &tmap_a, fb0, kb * CF::BK, a_row);
+                            if constexpr (BT) {
+                                tma_load_2d_pair(sb, &tmap_b, fb0, kb * CF::BK, b_col);  // BN_LOCAL rows of B^T
+                            } else {
 #pragma unroll
-                            for (int j = 0; j < CF::BN_LOCAL / 64; ++j)
-                                tma_load_2d_pair(sb + j * CF::B_BOX_BYTES, &tmap_b, fb0, b_col + 64 * j,
-                                                 kb * CF::BK);
+                                for (int j = 0; j < CF::BN_LOCAL / 64; ++j)
+                                    tma_load_2d_pair(sb + j * CF::B_BOX_BYTES, &tmap_b, fb0, b_col + 64 * j,
+                                                     kb * CF::BK);
+                            }
                         } else {
                             mbar_arrive_expect_tx(fb, CF::TX_BYTES);
                             tma_load_2d(sa, &tmap_a, fb, kb * CF::BK, a_row);
+                            if constexpr (BT) {
+                                tma_load_2d(sb, &tmap_b, fb, kb * CF::BK, b_col);  // BN_LOCAL rows of B^T
+                            } else {
 #pragma unroll
-                            for (int j = 0; j < CF::BN_LOCAL / 64; ++j)
-                                tma_load_2d(sb + j * CF::B_BOX_BYTES, &tmap_b, fb, b_col + 64 * j, kb * CF::BK);
+                                for (int j = 0; j < CF::BN_LOCAL / 64; ++j)
+                                    tma_load_2d(sb + j * CF::B_BOX_BYTES, &tmap_b, fb, b_col + 64 * j,
+                                                kb * CF::BK);
+                            }
                         }
                         issued |= 1u << stage;
                         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -410,11 +424,12 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (even CTA)
         if (lane == 0 && leader) {
-            constexpr uint32_t IDESC = mma_idesc_f16(DT, CF::TILE_M, CF::BN, 0, 1);
+            constexpr uint32_t IDESC = mma_idesc_f16(DT, CF::TILE_M, CF::BN, 0, BT ? 0 : 1);
             // A: K-major, rows of 128 B, 8-row atoms 1024 B apart (SBO); LBO unused.
-            // B: N-major, 64-column boxes of BK rows (LBO = box bytes), 8-row atoms (SBO).
+            // B: N-major, 64-column boxes of BK rows (LBO = box bytes), 8-row atoms (SBO);
+            //    or, given as B^T, K-major like A.
             const uint64_t a_desc0 = smem_desc_sw128(sA, 16, 1024);
-            const uint64_t b_desc0 = smem_desc_sw128(sB, CF::B_BOX_BYTES, 1024);
+            const uint64_t b_desc0 = BT ? smem_desc_sw128(sB, 16, 1024) : smem_desc_sw128(sB, CF::B_BOX_BYTES, 1024);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -439,8 +454,10 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                     const uint64_t b_desc = b_desc0 + ((stage * CF::B_STAGE_BYTES) >> 4);
 #pragma unroll
                     for (int k = 0; k < CF::BK / 16; ++k) {
-                        // K step of 16: +32 B inside A's swizzled row, +16 rows (2048 B) of B
-                        const uint64_t ad = a_desc + ((32 * k) >> 4), bd = b_desc + ((2048 * k) >> 4);
+                        // K step of 16: +32 B inside A's swizzled row; B: +16 rows (2048 B),
+                        // or +32 B when B is K-major
+                        const uint64_t ad = a_desc + ((32 * k) >> 4);
+                        const uint64_t bd = b_desc + (((BT ? 32 : 2048) * k) >> 4);
                         const uint32_t accumulate = (kb != w.kb0 || k != 0) ? 1u : 0u;
                         if constexpr (PAIR)
                             tc_mma_f16_pair(d_tmem, ad, bd, IDESC, accumulate);
@@ -582,6 +599,7 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                         v[j] = __uint_as_float(r[32 * h + j]);
                     const int colh = col0 + 32 * h;
                     if constexpr (EPI == 1) {
+                      if (p.epi_bias) {
                         if (p.bias_vec16 && colh + 32 <= p.N) {
                             const uint4 *bp = reinterpret_cast<const uint4 *>(p.bias + colh);
 #pragma unroll
@@ -600,9 +618,12 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                                 if (colh + j < p.N)
                                     v[j] += to_float<DT>(__ldg(p.bias + colh + j));
                         }
+                      }
+                      if (p.epi_gelu) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
                             v[j] = gelu_erf(v[j]);
+                      }
                     }
                     uint32_t packed[16];
 #pragma unroll

@@ -30,7 +30,7 @@ struct ConfigEntry {
     int ctas;                // 1, or 2 for a CTA pair (cluster of two, cta_group::2 MMA)
     int threads;             // threads per CTA
     int smem_bytes;
-    KernelFn fn[2][2][2];  // [dtype][epilogue][tma_store]
+    KernelFn fn[2][2][2][2];  // [dtype][fused epilogue][tma_store][B given transposed]
 };
 
 template <class CF>
@@ -46,14 +46,22 @@ ConfigEntry make_entry(const char *name)
     e.bk = CF::BK;
     e.stages = CF::STAGES;
     e.smem_bytes = CF::SMEM_BYTES;
-    e.fn[0][0][0] = gemm_sm100_kernel<CF, 0, 0, false>;
-    e.fn[0][0][1] = gemm_sm100_kernel<CF, 0, 0, true>;
-    e.fn[0][1][0] = gemm_sm100_kernel<CF, 0, 1, false>;
-    e.fn[0][1][1] = gemm_sm100_kernel<CF, 0, 1, true>;
-    e.fn[1][0][0] = gemm_sm100_kernel<CF, 1, 0, false>;
-    e.fn[1][0][1] = gemm_sm100_kernel<CF, 1, 0, true>;
-    e.fn[1][1][0] = gemm_sm100_kernel<CF, 1, 1, false>;
-    e.fn[1][1][1] = gemm_sm100_kernel<CF, 1, 1, true>;
+    e.fn[0][0][0][0] = gemm_sm100_kernel<CF, 0, 0, false, false>;
+    e.fn[0][0][1][0] = gemm_sm100_kernel<CF, 0, 0, true, false>;
+    e.fn[0][1][0][0] = gemm_sm100_kernel<CF, 0, 1, false, false>;
+    e.fn[0][1][1][0] = gemm_sm100_kernel<CF, 0, 1, true, false>;
+    e.fn[1][0][0][0] = gemm_sm100_kernel<CF, 1, 0, false, false>;
+    e.fn[1][0][1][0] = gemm_sm100_kernel<CF, 1, 0, true, false>;
+    e.fn[1][1][0][0] = gemm_sm100_kernel<CF, 1, 1, false, false>;
+    e.fn[1][1][1][0] = gemm_sm100_kernel<CF, 1, 1, true, false>;
+    e.fn[0][0][0][1] = gemm_sm100_kernel<CF, 0, 0, false, true>;
+    e.fn[0][0][1][1] = gemm_sm100_kernel<CF, 0, 0, true, true>;
+    e.fn[0][1][0][1] = gemm_sm100_kernel<CF, 0, 1, false, true>;
+    e.fn[0][1][1][1] = gemm_sm100_kernel<CF, 0, 1, true, true>;
+    e.fn[1][0][0][1] = gemm_sm100_kernel<CF, 1, 0, false, true>;
+    e.fn[1][0][1][1] = gemm_sm100_kernel<CF, 1, 0, true, true>;
+    e.fn[1][1][0][1] = gemm_sm100_kernel<CF, 1, 1, false, true>;
+    e.fn[1][1][1][1] = gemm_sm100_kernel<CF, 1, 1, true, true>;
     return e;
 }
 
@@ -140,7 +148,7 @@ int model_config_single(int64_t M, int64_t N, int num_sms)
 int choose_config(int64_t M, int64_t N, int64_t K, int dtype, int epi, int num_sms, bool *split)
 {
     for (const TableRow &r : kTable) {
-        if (r.m == M && r.n == N && r.k == K && r.dtype == dtype && r.epi == epi) {
+        if (r.m == M && r.n == N && r.k == K && r.dtype == dtype && r.epi == (epi != 0 ? 1 : 0)) {
             const int i = config_index(r.config);
             if (i >= 0) {
                 *split = r.split != 0;
@@ -171,22 +179,23 @@ tl_status validate(const void *A, const void *B, const void *bias, void *C, int6
         return TL_ERR_INVALID_ARG;
     if (dtype != TL_F16 && dtype != TL_BF16)
         return TL_ERR_INVALID_ARG;
-    if (epi != TL_EPI_NONE && epi != TL_EPI_BIAS_GELU)
+    if (epi < TL_EPI_NONE || epi > TL_EPI_GELU)
         return TL_ERR_INVALID_ARG;
-    if (epi == TL_EPI_BIAS_GELU && !bias)
+    const bool needs_bias = epi == TL_EPI_BIAS_GELU || epi == TL_EPI_BIAS;
+    if (needs_bias && !bias)
         return TL_ERR_INVALID_ARG;
     if (opt && (opt->config < 0 || opt->config > num_configs()))
         return TL_ERR_INVALID_ARG;
     if (opt && (opt->inject_fault != 0 && opt->inject_fault != 1))
         return TL_ERR_INVALID_ARG;
-    if (opt && ((opt->no_split != 0 && opt->no_split != 1) || opt->reserved != 0))
+    if (opt && ((opt->no_split != 0 && opt->no_split != 1) || (opt->b_layout != 0 && opt->b_layout != 1)))
         return TL_ERR_INVALID_ARG;
     if (opt && opt->inject_fault && opt->config > 0 && kConfigs[opt->config - 1].ctas != 1)
         return TL_ERR_UNSUPPORTED;  // the fault hook exists for single-CTA configurations only
     const int64_t lim = 0x7FFFFFFFll;
     if (M > lim || N > lim || K > lim)
         return TL_ERR_UNSUPPORTED;
-    if (!aligned(A, 2) || !aligned(B, 2) || !aligned(C, 2) || (epi == TL_EPI_BIAS_GELU && !aligned(bias, 2)))
+    if (!aligned(A, 2) || !aligned(B, 2) || !aligned(C, 2) || (needs_bias && !aligned(bias, 2)))
         return TL_ERR_MISALIGNED;
     return TL_OK;
 }
@@ -258,11 +267,14 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
     q.cluster_ctas = c.ctas;
     q.smem_bytes = c.smem_bytes;
     // TMA needs a 16-byte-aligned base and row strides that are multiples of 16 bytes.
+    const bool bt = opt && opt->b_layout == 1;  // B given as N x K
+    const int64_t b_cols = bt ? K : N;         // row length of B as stored
+    const int64_t b_rows = bt ? N : K;
     q.pad_a = !(aligned(A, 16) && K % 8 == 0);
-    q.pad_b = !(aligned(B, 16) && N % 8 == 0);
+    q.pad_b = !(aligned(B, 16) && b_cols % 8 == 0);
     q.direct_store = !(aligned(C, 16) && N % 8 == 0);
     p.lda = q.pad_a ? ceil_div(K, 8) * 8 : K;
-    p.ldb = q.pad_b ? ceil_div(N, 8) * 8 : N;
+    p.ldb = q.pad_b ? ceil_div(b_cols, 8) * 8 : b_cols;
     int64_t ws = 0;
     p.a_ws_off = p.b_ws_off = -1;
     if (q.pad_a) {
@@ -271,7 +283,7 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
     }
     if (q.pad_b) {
         p.b_ws_off = ws;
-        ws += ceil_div(K * p.ldb * 2, 256) * 256;
+        ws += ceil_div(b_rows * p.ldb * 2, 256) * 256;
     }
     p.partial_off = p.flag_off = -1;
     if (split > 1) {
@@ -443,7 +455,8 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
 {
     const ConfigEntry &c = kConfigs[p.pub.config];
     const bool tma_store = !p.pub.direct_store;
-    KernelFn fn = c.fn[dtype][epi][tma_store ? 1 : 0];
+    const int bt = (opt && opt->b_layout == 1) ? 1 : 0;
+    KernelFn fn = c.fn[dtype][epi != 0][tma_store ? 1 : 0][bt];
     tl_status st = raise_smem_limit(d, fn, c.smem_bytes);
     if (st != TL_OK)
         return st;
@@ -452,7 +465,8 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
     std::memset(&tc, 0, sizeof(tc));
     if (!encode_2d(&ta, A, dtype, M, K, p.lda, 64, c.cta_m))
         return TL_ERR_CUDA;
-    if (!encode_2d(&tb, B, dtype, K, N, p.ldb, 64, c.bk))
+    if (bt ? !encode_2d(&tb, B, dtype, N, K, p.ldb, 64, c.bn / c.ctas)   // B^T: BN/CTAS rows of 64 k
+           : !encode_2d(&tb, B, dtype, K, N, p.ldb, 64, c.bk))
         return TL_ERR_CUDA;
     if (tma_store && !encode_2d(&tc, C, dtype, M, N, N, 64, 32))
         return TL_ERR_CUDA;
@@ -468,6 +482,10 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
     gp.group_m = 8;
     gp.bias = static_cast<const uint16_t *>(bias);
     gp.bias_vec16 = bias && aligned(bias, 16);
+    gp.epi_bias = epi == TL_EPI_BIAS_GELU || epi == TL_EPI_BIAS;
+    gp.epi_gelu = epi == TL_EPI_BIAS_GELU || epi == TL_EPI_GELU;
+    if (!gp.epi_bias)
+        gp.bias = nullptr;
     gp.inject_fault = opt ? opt->inject_fault : 0;
     gp.C = static_cast<uint16_t *>(C);
     gp.ldc = N;
@@ -521,7 +539,7 @@ tl_status device_plan(DeviceState *d, const void *A, const void *B, const void *
     const ConfigEntry &c = kConfigs[p->pub.config];
     if (c.ctas != 2)
         return TL_OK;
-    KernelFn fn = c.fn[dtype][epi][p->pub.direct_store ? 0 : 1];
+    KernelFn fn = c.fn[dtype][epi != 0][p->pub.direct_store ? 0 : 1][(opt && opt->b_layout == 1) ? 1 : 0];
     if ((st = raise_smem_limit(d, fn, c.smem_bytes)) != TL_OK)
         return st;
     cudaLaunchConfig_t cfg{};
@@ -576,7 +594,8 @@ tl_status gemm_impl(const void *A, const void *B, const void *bias, void *C, int
     }
     if (st == TL_OK && p.pub.pad_b) {
         void *dst = static_cast<uint8_t *>(ws) + p.b_ws_off;
-        st = launch_pad(B, K, N, dst, p.ldb, d->num_sms, stream);
+        const bool bt = opt && opt->b_layout == 1;
+        st = launch_pad(B, bt ? N : K, bt ? K : N, dst, p.ldb, d->num_sms, stream);
         b_use = dst;
     }
     if (st == TL_OK)
@@ -621,28 +640,29 @@ tl_status noalloc_setup(DeviceState *d, void **scratch)
             const ConfigEntry &c = kConfigs[i];
             for (int dt = 0; dt < 2; ++dt)
                 for (int epi = 0; epi < 2; ++epi)
-                    for (int st = 0; st < 2; ++st) {
-                        KernelFn fn = c.fn[dt][epi][st];
-                        tl_status r = raise_smem_limit(d, fn, c.smem_bytes);
-                        if (r != TL_OK)
-                            return r;
-                        if (c.ctas == 2) {
-                            cudaLaunchConfig_t cfg{};
-                            cudaLaunchAttribute attr[1];
-                            attr[0].id = cudaLaunchAttributeClusterDimension;
-                            attr[0].val.clusterDim.x = 2;
-                            attr[0].val.clusterDim.y = 1;
-                            attr[0].val.clusterDim.z = 1;
-                            cfg.gridDim = dim3(2, 1, 1);
-                            cfg.blockDim = dim3(static_cast<unsigned>(c.threads), 1, 1);
-                            cfg.dynamicSmemBytes = static_cast<size_t>(c.smem_bytes);
-                            cfg.attrs = attr;
-                            cfg.numAttrs = 1;
-                            int n = 0;
-                            if ((r = max_active_clusters(d, fn, cfg, &n)) != TL_OK)
+                    for (int st = 0; st < 2; ++st)
+                        for (int bt = 0; bt < 2; ++bt) {
+                            KernelFn fn = c.fn[dt][epi][st][bt];
+                            tl_status r = raise_smem_limit(d, fn, c.smem_bytes);
+                            if (r != TL_OK)
                                 return r;
+                            if (c.ctas == 2) {
+                                cudaLaunchConfig_t cfg{};
+                                cudaLaunchAttribute attr[1];
+                                attr[0].id = cudaLaunchAttributeClusterDimension;
+                                attr[0].val.clusterDim.x = 2;
+                                attr[0].val.clusterDim.y = 1;
+                                attr[0].val.clusterDim.z = 1;
+                                cfg.gridDim = dim3(2, 1, 1);
+                                cfg.blockDim = dim3(static_cast<unsigned>(c.threads), 1, 1);
+                                cfg.dynamicSmemBytes = static_cast<size_t>(c.smem_bytes);
+                                cfg.attrs = attr;
+                                cfg.numAttrs = 1;
+                                int n = 0;
+                                if ((r = max_active_clusters(d, fn, cfg, &n)) != TL_OK)
+                                    return r;
+                            }
                         }
-                    }
         }
         p = addr;
         g_noalloc_scratch_ptr[dev].store(p, std::memory_order_release);

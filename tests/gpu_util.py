@@ -37,12 +37,14 @@ def from_device(t) -> np.ndarray:
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def run_library(A_bits, B_bits, bias_bits, dt, epi, config=0, offsets=(0, 0, 0, 0), sync=True):
-    """C bits from tl_gemm (through the C ABI) for host bit arrays."""
+def run_library(A_bits, B_bits, bias_bits, dt, epi, config=0, offsets=(0, 0, 0, 0), sync=True,
+                b_transposed=False):
+    """C bits from tl_gemm (through the C ABI) for host bit arrays.  B_bits is
+    K x N; with b_transposed the library is given its transpose (N x K)."""
     import torch
     import tensor_core_gemm_tl_b200 as tg
     A = to_device(A_bits, dt, offsets[0])
-    B = to_device(B_bits, dt, offsets[1])
+    B = to_device(np.ascontiguousarray(B_bits.T) if b_transposed else B_bits, dt, offsets[1])
     bias = to_device(bias_bits, dt, offsets[2]) if bias_bits is not None else None
     M, N = A_bits.shape[0], B_bits.shape[1]
     if offsets[3]:
@@ -50,7 +52,7 @@ def run_library(A_bits, B_bits, bias_bits, dt, epi, config=0, offsets=(0, 0, 0, 
         out = buf[offsets[3]:].view(M, N)
     else:
         out = torch.empty((M, N), dtype=torch_dtype(dt), device="cuda")
-    tg.gemm(A, B, bias, epilogue="bias_gelu" if epi == wl.EPI_BIAS_GELU else None, out=out, config=config)
+    tg.gemm(A, B, bias, epilogue=int(epi), out=out, config=config, b_transposed=b_transposed)
     if sync:
         torch.cuda.synchronize()
         assert tg.check_device() == 0
@@ -90,9 +92,12 @@ def accumulation_bound(A_bits, B_bits, bias_bits, dt, epi, ref, rows=None, point
         Ar = Af if rows is None else Af[rows]
         absdot = np.abs(Ar) @ np.abs(Bf)
     e = K * 2.0 ** -23 * absdot
-    if epi == wl.EPI_BIAS_GELU:
-        b = np.abs(wl.bits_to_float32(bias_bits, dt).astype(np.float64))
-        b = b[points[1]] if points is not None else b[None, :]
+    if epi != wl.EPI_NONE:
+        if bias_bits is not None and epi in (wl.EPI_BIAS_GELU, wl.EPI_BIAS):
+            b = np.abs(wl.bits_to_float32(bias_bits, dt).astype(np.float64))
+            b = b[points[1]] if points is not None else b[None, :]
+        else:
+            b = 0.0
         e = 1.2 * (e + 2.0 ** -22 * (absdot + b)) + 1e-5 * np.abs(ref)
     return 0.5 * ulp(np.abs(ref) + e, dt) + e + 1e-45
 

@@ -52,7 +52,10 @@ def test_version_and_strings():
     (dict(K=0), tg.Status.INVALID_ARG),
     (dict(dtype=2), tg.Status.INVALID_ARG),
     (dict(epi=7), tg.Status.INVALID_ARG),
+    (dict(epi=-1), tg.Status.INVALID_ARG),
     (dict(epi=1, bias=0), tg.Status.INVALID_ARG),
+    (dict(epi=2, bias=0), tg.Status.INVALID_ARG),
+    (dict(epi=2, bias=P + 1), tg.Status.MISALIGNED),
     (dict(M=1 << 31), tg.Status.UNSUPPORTED),
     (dict(K=1 << 40), tg.Status.UNSUPPORTED),
     (dict(A=P + 1), tg.Status.MISALIGNED),
@@ -191,3 +194,19 @@ def test_plan_splits_only_a_short_last_round(M, N, K, config, split, full):
 def test_fault_hook_disables_the_split():
     st, p = tg.tl_gemm_plan(P, P, 0, P, 1024, 1024, 2048, 0, 0, 148, tg.Options(config=1, inject_fault=1))
     assert st == 0 and p.split == 1
+
+
+def test_gelu_only_needs_no_bias_and_b_layout_is_validated():
+    st, _ = tg.tl_gemm_plan(P, P, 0, P, 256, 256, 256, 0, tg.TL_EPI_GELU, 148)
+    assert st == 0
+    assert tg.tl_gemm_ex(P, P, 0, P, 8, 8, 8, 0, 0, 0, tg.Options(b_layout=2)) == tg.Status.INVALID_ARG
+
+
+def test_plan_transposed_b_pads_on_k():
+    # B given as N x K: its rows are K long, so an odd K pads B (and A), not N
+    p = tg.plan(512, 1000, 2050, tg.TL_BF16, None, num_sms=148, b_transposed=True)
+    assert p["pad_a"] == 1 and p["pad_b"] == 1 and p["direct_store"] == 0
+    p = tg.plan(512, 1001, 2048, tg.TL_BF16, None, num_sms=148, b_transposed=True)
+    assert p["pad_a"] == 0 and p["pad_b"] == 0 and p["direct_store"] == 1
+    p = tg.plan(512, 1001, 2048, tg.TL_BF16, None, num_sms=148)
+    assert p["pad_b"] == 1

@@ -168,6 +168,42 @@ def test_epilogue_matches_plain_plus_gelu_structure():
     compare(fused, rf, dt, accumulation_bound(A, B, bias, dt, wl.EPI_BIAS_GELU, rf))
 
 
+# ------------------------------------------------------------------ B given transposed, epilogue variants
+@pytest.mark.parametrize("config", ALL_CONFIGS)
+@pytest.mark.parametrize("dt", [wl.F16, wl.BF16])
+def test_transposed_b_layout_probe(config, dt):
+    """B handed over as N x K (K-major): the one-hot layout probe again."""
+    M, N, K = 384, 320, 192
+    kk = (np.arange(M) * 37 + 5) % K
+    A = np.zeros((M, K), np.float32)
+    A[np.arange(M), kk] = 1.0
+    code = (np.arange(K)[:, None] % 16) * 16 + (np.arange(N)[None, :] % 16)
+    Ab = wl.round_to_bits(A, dt)
+    Bb = wl.round_to_bits(code.astype(np.float32), dt)
+    C = run_library(Ab, Bb, None, dt, wl.EPI_NONE, config=config, b_transposed=True)
+    assert np.array_equal(wl.bits_to_float32(C, dt), code[kk, :].astype(np.float32))
+
+
+@pytest.mark.parametrize("config", ALL_CONFIGS)
+@pytest.mark.parametrize("M,N,K", [(700, 900, 336), (300, 1001, 2050), (129, 255, 64)])
+def test_transposed_b_vs_oracle(config, M, N, K):
+    dt, epi = wl.BF16, wl.EPI_BIAS_GELU
+    A, B, bias = inputs(M, N, K, dt, epi, seed=M + config)
+    ref = oracle.gemm(A, B, bias, dt, epi)
+    C = run_library(A, B, bias, dt, epi, config=config, b_transposed=True)
+    compare(C, ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
+
+
+@pytest.mark.parametrize("epi", [wl.EPI_BIAS, wl.EPI_GELU])
+@pytest.mark.parametrize("dt", [wl.F16, wl.BF16])
+@pytest.mark.parametrize("M,N,K", [(256, 512, 256), (300, 520, 200), (4096, 1024, 512)])
+def test_bias_only_and_gelu_only_vs_oracle(epi, dt, M, N, K):
+    A, B, bias = inputs(M, N, K, dt, epi, seed=K + epi)
+    ref = oracle.gemm(A, B, bias, dt, epi)
+    C = run_library(A, B, bias, dt, epi)
+    compare(C, ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
+
+
 # ------------------------------------------------------------------ the named workloads
 def _sample_rows(M, n, rng):
     rows = {0, M - 1, M // 2}
