@@ -17,6 +17,9 @@ What it computes, and where that is stated:
   * TileLang GPU kernel design article, paragraph 5 (fused GEMM epilogue):
     bias add then GELU on the accumulator before the single store; bias is
     per column, GELU is the exact erf form.
+  * The same article, paragraph 6 (attention forward with online softmax,
+    checked against PyTorch's scaled dot-product attention): the plain
+    definition softmax(scale Q K^T) V, causal mask keeping key j <= query i.
 """
 from __future__ import annotations
 
@@ -66,6 +69,9 @@ def _bind(path):
     lib.oracle_decode_array.restype = None
     lib.oracle_gelu_array.argtypes = [p, p, i64]
     lib.oracle_gelu_array.restype = None
+    lib.oracle_attention_rows.argtypes = [i64, i64, i64, i64, p, p, p, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_double, p, p, i64, p, p]
+    lib.oracle_attention_rows.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = ctypes.c_int
     return lib
@@ -157,6 +163,35 @@ class Oracle:
         self._lib.oracle_gelu_array(_ptr(a), _ptr(out), a.size)
         return out
 
+    def attention(self, Q, K, V, dtype, causal, scale, rows=None):
+        """softmax(scale Q K^T [causal]) V in fp64 for Q (B, H, Sq, D), K and V
+        (B, H, Sk, D) uint16 bit arrays.  Returns (O, lse): all of O (B, H, Sq, D)
+        and lse (B, H, Sq), or, with rows = (bh_idx, q_idx) arrays, O (n, D) and
+        lse (n,) for those (flattened batch*head, query) rows."""
+        Q, K, V = _bits(Q, "Q"), _bits(K, "K"), _bits(V, "V")
+        if Q.ndim != 4 or K.shape != V.shape or K.ndim != 4 or Q.shape[:2] != K.shape[:2] \
+                or Q.shape[3] != K.shape[3]:
+            raise ValueError(f"shapes Q{Q.shape} K{K.shape} V{V.shape} do not match")
+        B, H, Sq, D = Q.shape
+        Sk = K.shape[2]
+        BH = B * H
+        if rows is None:
+            bh = np.repeat(np.arange(BH, dtype=np.int64), Sq)
+            qi = np.tile(np.arange(Sq, dtype=np.int64), BH)
+        else:
+            bh = np.ascontiguousarray(rows[0], dtype=np.int64)
+            qi = np.ascontiguousarray(rows[1], dtype=np.int64)
+        O = np.empty((bh.size, D), np.float64)
+        lse = np.empty(bh.size, np.float64)
+        rc = self._lib.oracle_attention_rows(BH, Sq, Sk, D, _ptr(Q), _ptr(K), _ptr(V), dtype,
+                                             int(bool(causal)), float(scale), _ptr(bh), _ptr(qi),
+                                             bh.size, _ptr(O), _ptr(lse))
+        if rc != 0:
+            raise ValueError("oracle_attention_rows: bad index or size")
+        if rows is None:
+            return O.reshape(B, H, Sq, D), lse.reshape(B, H, Sq)
+        return O, lse
+
     def max_threads(self) -> int:
         """OpenMP threads the oracle uses (OMP_NUM_THREADS, else all cores)."""
         return int(self._lib.oracle_max_threads())
@@ -195,6 +230,11 @@ def decode(bits, dtype) -> np.ndarray:
 def gelu(x) -> np.ndarray:
     """Exact GELU x * Phi(x) in fp64, elementwise."""
     return _oracle().gelu(x)
+
+
+def attention(Q, K, V, dtype, causal, scale, rows=None):
+    """softmax(scale Q K^T [causal]) V and its log-sum-exp, in fp64."""
+    return _oracle().attention(Q, K, V, dtype, causal, scale, rows)
 
 
 def max_threads() -> int:

@@ -199,3 +199,74 @@ int oracle_max_threads(void)
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------
+ * Attention forward, the plain definition (fp64):
+ *
+ *     O = softmax(scale * Q K^T  [causal: keys j > query i removed]) V
+ *     lse_i = log sum_j exp(scale * q_i . k_j)      (over the kept keys)
+ *
+ * It follows the TileLang GPU kernel design article, paragraph 6 (attention
+ * over query, key and value tiles with online softmax: running maximum,
+ * normaliser and rescaling -- an evaluation order of this same definition),
+ * checked there against PyTorch's scaled dot-product attention, whose
+ * causal mask keeps key j <= query i.  Here the scores are summed in d
+ * order, the maximum is subtracted before exponentiating (the same value),
+ * and the normaliser is applied once at the end.
+ *
+ * Layout: Q is [BH][Sq][D], K and V are [BH][Sk][D], row-major 16-bit
+ * patterns.  Row p of the output is (bh_idx[p], q_idx[p]): O[p][0..D),
+ * lse[p] (natural log).  Returns 0, or -1 for an index out of range.
+ * ------------------------------------------------------------------------ */
+int oracle_attention_rows(int64_t BH, int64_t Sq, int64_t Sk, int64_t D,
+                          const uint16_t *Q, const uint16_t *K, const uint16_t *V, int dtype,
+                          int causal, double scale,
+                          const int64_t *bh_idx, const int64_t *q_idx, int64_t nrows,
+                          double *O, double *lse)
+{
+    for (int64_t p = 0; p < nrows; ++p)
+        if (bh_idx[p] < 0 || bh_idx[p] >= BH || q_idx[p] < 0 || q_idx[p] >= Sq)
+            return -1;
+    if (Sk < 1 || D < 1)
+        return -1;
+    int64_t p;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (p = 0; p < nrows; ++p) {
+        const int64_t bh = bh_idx[p], i = q_idx[p];
+        const uint16_t *q = Q + (bh * Sq + i) * D;
+        const int64_t nkeys = causal ? (i + 1 < Sk ? i + 1 : Sk) : Sk;
+        double *s = (double *)malloc((size_t)nkeys * sizeof(double));
+        double *o = O + p * D;
+        if (!s) {
+            for (int64_t d = 0; d < D; ++d)
+                o[d] = NAN;
+            lse[p] = NAN;
+            continue;
+        }
+        double m = -INFINITY;
+        for (int64_t j = 0; j < nkeys; ++j) {
+            const uint16_t *k = K + (bh * Sk + j) * D;
+            double acc = 0.0;
+            for (int64_t d = 0; d < D; ++d)
+                acc += decode(q[d], dtype) * decode(k[d], dtype);
+            s[j] = scale * acc;
+            if (s[j] > m)
+                m = s[j];
+        }
+        double l = 0.0;
+        for (int64_t d = 0; d < D; ++d)
+            o[d] = 0.0;
+        for (int64_t j = 0; j < nkeys; ++j) {
+            const double w = exp(s[j] - m);
+            const uint16_t *v = V + (bh * Sk + j) * D;
+            l += w;
+            for (int64_t d = 0; d < D; ++d)
+                o[d] += w * decode(v[d], dtype);
+        }
+        for (int64_t d = 0; d < D; ++d)
+            o[d] /= l;
+        lse[p] = m + log(l);
+        free(s);
+    }
+    return 0;
+}

@@ -10,6 +10,7 @@ sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 
 import oracle  # noqa: E402
 from oracle_pins import ALL_PINS  # noqa: E402
+from oracle_pins_attention import ATTENTION_PINS  # noqa: E402
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 
@@ -33,6 +34,14 @@ MUTANTS = [
     ("bias_only_drops_bias", "c[j] = c[j] + decode(bias[j], dtype);", "c[j] = c[j];"),
     ("gelu_only_adds_bias", "            s = oracle_gelu(s);", "            s = oracle_gelu(s + 1.0);"),
     ("gelu_only_rows_skip_gelu", "                c[j] = oracle_gelu(c[j]);", "                c[j] = c[j];"),
+    ("attn_mask_wrong_direction", "const int64_t nkeys = causal ? (i + 1 < Sk ? i + 1 : Sk) : Sk;",
+     "const int64_t nkeys = causal ? (i < Sk ? i : Sk) + (i == 0) : Sk;"),
+    ("attn_scale_ignored", "s[j] = scale * acc;", "s[j] = acc;"),
+    ("attn_no_max_subtraction", "const double w = exp(s[j] - m);", "const double w = exp(s[j]);"),
+    ("attn_unnormalised", "o[d] /= l;", "o[d] /= 1.0;"),
+    ("attn_v_from_query_row", "const uint16_t *v = V + (bh * Sk + j) * D;",
+     "const uint16_t *v = V + (bh * Sk + (j + i) % Sk) * D;"),
+    ("attn_lse_without_max", "lse[p] = m + log(l);", "lse[p] = log(l);"),
     ("f16_exponent_bias", "v = ldexp((double)(f + 1024), e - 25);", "v = ldexp((double)(f + 1024), e - 24);"),
     ("f16_subnormal_as_normal", "v = ldexp((double)f, -24);", "v = ldexp((double)(f + 1024), -25);"),
     ("bf16_exponent_bias", "v = ldexp((double)(f + 128), e - 134);", "v = ldexp((double)(f + 128), e - 133);"),
@@ -52,7 +61,7 @@ def test_mutant_fails_a_pin(tmp_path, name, old, new):
     so = oracle.build(force=True, src=str(csrc), out=str(tmp_path / f"liboracle_{name}.so"))
     orc = oracle.from_library(so)
     failed = []
-    for pin in ALL_PINS:
+    for pin in ALL_PINS + ATTENTION_PINS:
         try:
             pin(orc)
         except AssertionError:

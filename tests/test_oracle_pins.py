@@ -5,6 +5,7 @@ import pytest
 
 import oracle
 from oracle_pins import ALL_PINS
+from oracle_pins_attention import ATTENTION_PINS
 
 
 @pytest.fixture(scope="module")
@@ -12,7 +13,7 @@ def orc():
     return oracle._oracle()
 
 
-@pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
+@pytest.mark.parametrize("pin", ALL_PINS + ATTENTION_PINS, ids=lambda f: f.__name__)
 def test_pin(orc, pin):
     pin(orc)
 
