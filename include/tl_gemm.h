@@ -136,6 +136,36 @@ TL_API tl_status tl_gemm_noalloc(const void *A, const void *B, const void *bias,
                          int64_t M, int64_t N, int64_t K,
                          tl_dtype dtype, tl_epilogue epi, tl_stream stream);
 
+/*
+ * tl_attention_fwd -- attention forward with an online softmax on the tensor
+ * cores (the TileLang GPU kernel design article, paragraph 6: query, key and
+ * value tiles, running maximum, normaliser and rescaling, the score matrix
+ * never written to global memory, checked against PyTorch's scaled
+ * dot-product attention):
+ *
+ *   O[b,h,i,:] = sum_j softmax_j(scale * Q[b,h,i,:] . K[b,h,j,:]) V[b,h,j,:]
+ *   lse[b,h,i] = log sum_j exp(scale * Q[b,h,i,:] . K[b,h,j,:])
+ *
+ * with j over all keys, or over j <= i when `causal` (PyTorch's is_causal).
+ *
+ *   Q    device pointer, [batch][heads][seq_q][head_dim], `dtype`, contiguous
+ *   K, V device pointers, [batch][heads][seq_k][head_dim], `dtype`, contiguous
+ *   O    device pointer, [batch][heads][seq_q][head_dim], `dtype`; written
+ *   lse  device pointer to batch*heads*seq_q floats, or NULL; written
+ *   head_dim        64 or 128
+ *   batch * heads   at most 65535
+ *   softmax_scale   > 0, or 0 for 1 / sqrt(head_dim)
+ *
+ * The products run on 16-bit inputs with fp32 accumulation; the softmax
+ * weights are rounded to `dtype` before the product with V (as in
+ * FlashAttention); O is rounded once.  Q, K, V, O must be 16-byte aligned
+ * (TL_ERR_MISALIGNED otherwise), lse 4-byte aligned.  Asynchronous on
+ * `stream`; allocates nothing; bounded waits report through tl_check_device.
+ */
+TL_API tl_status tl_attention_fwd(const void *Q, const void *K, const void *V, void *O, float *lse,
+                          int64_t batch, int64_t heads, int64_t seq_q, int64_t seq_k, int64_t head_dim,
+                          tl_dtype dtype, int32_t causal, float softmax_scale, tl_stream stream);
+
 /* Options for tl_gemm_ex.  Zero-initialise, then set what you need. */
 typedef struct {
     int32_t config;       /* 0: the library's choice for the shape; k > 0: kernel

@@ -15,12 +15,13 @@ from __future__ import annotations
 from ._binding import (  # noqa: F401
     LIB_PATH, Options, Plan, Status, TLError, TL_BF16, TL_EPI_BIAS, TL_EPI_BIAS_GELU, TL_EPI_GELU,
     TL_EPI_NONE, TL_F16,
-    SIGNATURES, tl_check_device, tl_config_name, tl_gemm, tl_gemm_ex, tl_gemm_noalloc, tl_gemm_plan, tl_num_configs,
+    SIGNATURES, tl_attention_fwd, tl_check_device, tl_config_name, tl_gemm, tl_gemm_ex, tl_gemm_noalloc,
+    tl_gemm_plan, tl_num_configs,
     tl_status_string, tl_version,
 )
 
 __all__ = [
-    "gemm", "check_device", "plan", "configs", "Options", "Plan", "Status", "TLError",
+    "gemm", "attention", "check_device", "plan", "configs", "tl_attention_fwd", "Options", "Plan", "Status", "TLError",
     "tl_gemm", "tl_gemm_ex", "tl_gemm_noalloc", "tl_check_device", "tl_gemm_plan", "tl_num_configs", "tl_config_name",
     "tl_status_string", "tl_version", "TL_F16", "TL_BF16", "TL_EPI_NONE", "TL_EPI_BIAS_GELU",
     "TL_EPI_BIAS", "TL_EPI_GELU",
@@ -92,6 +93,35 @@ def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0,
                          out.data_ptr(), M, N, K, dt, epi, s.cuda_stream)
     if st != 0:
         raise TLError(st, "tl_gemm")
+    return out
+
+
+def attention(q, k, v, causal: bool = False, scale: float = 0.0, out=None, lse=None, stream=None):
+    """softmax(scale q k^T [causal]) v for CUDA tensors q (B, H, Sq, D) and
+    k, v (B, H, Sk, D), fp16 or bf16, D in {64, 128}; scale 0 = 1/sqrt(D).
+    Returns out (B, H, Sq, D); fills `lse` (B, H, Sq) float32 if given."""
+    import torch
+    if q.dim() != 4 or k.shape != v.shape or k.dim() != 4 or q.shape[:2] != k.shape[:2] or q.shape[3] != k.shape[3]:
+        raise ValueError(f"shapes q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)} do not match")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype:
+            raise ValueError(f"{name} must be a contiguous CUDA tensor of q's dtype")
+    dt = _dtype_code(q)
+    B, H, Sq, D = q.shape
+    Sk = k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
+        raise ValueError("out must be contiguous, of q's shape and dtype")
+    if lse is not None and (lse.shape != (B, H, Sq) or lse.dtype != torch.float32 or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 tensor of shape (B, H, Sq)")
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = tl_attention_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                              lse.data_ptr() if lse is not None else 0, B, H, Sq, Sk, D, dt, causal, scale,
+                              s.cuda_stream)
+    if st != 0:
+        raise TLError(st, "tl_attention_fwd")
     return out
 
 

@@ -62,6 +62,8 @@ SIGNATURES = {
     "tl_gemm_ex": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, _P,
                                   ctypes.POINTER(Options)]),
     "tl_check_device": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "tl_attention_fwd": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int, _I32,
+                                        ctypes.c_float, _P]),
     "tl_gemm_plan": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, _I32,
                                     ctypes.POINTER(Options), ctypes.POINTER(Plan)]),
     "tl_num_configs": (_I32, []),
@@ -106,6 +108,13 @@ def tl_gemm_noalloc(A: int, B: int, bias: int | None, C: int, M: int, N: int, K:
 def tl_gemm_ex(A, B, bias, C, M, N, K, dtype, epi, stream=0, options: Options | None = None) -> int:
     return _lib.tl_gemm_ex(A, B, bias or None, C, M, N, K, dtype, epi, stream or None,
                            ctypes.byref(options) if options is not None else None)
+
+
+def tl_attention_fwd(Q, K, V, O, lse, batch, heads, seq_q, seq_k, head_dim, dtype, causal, softmax_scale,
+                     stream=0) -> int:
+    """Attention forward on device pointers; returns the tl_status code."""
+    return _lib.tl_attention_fwd(Q, K, V, O, lse or None, batch, heads, seq_q, seq_k, head_dim, dtype,
+                                 int(bool(causal)), float(softmax_scale), stream or None)
 
 
 def tl_check_device(stream: int = 0) -> tuple[int, int]:

@@ -345,3 +345,18 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint32_t bar, uint16_t mask)
 }
 
 } // namespace tl
+
+namespace tl {
+
+// 3-D tiled load global -> shared (x innermost), completion counted in bytes.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int32_t x,
+                                            int32_t y, int32_t z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(map), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+} // namespace tl

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
@@ -15,6 +16,7 @@
 
 #include "tl_gemm.h"
 #include "gemm_kernel.cuh"
+#include "attention_kernel.cuh"
 
 namespace tl {
 namespace {
@@ -605,6 +607,114 @@ tl_status gemm_impl(const void *A, const void *B, const void *bias, void *C, int
     return st;
 }
 
+// ------------------------------------------------------------------ attention forward
+using AttnFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, AttnParams);
+
+struct AttnEntry {
+    int smem_bytes;
+    AttnFn fn[2];  // [dtype]
+};
+
+template <int D>
+AttnEntry make_attn_entry()
+{
+    using CF = AttnConfig<D>;
+    AttnEntry e;
+    e.smem_bytes = CF::SMEM_BYTES;
+    e.fn[0] = attention_fwd_kernel<CF, 0>;
+    e.fn[1] = attention_fwd_kernel<CF, 1>;
+    return e;
+}
+
+const AttnEntry kAttn64 = make_attn_entry<64>();
+const AttnEntry kAttn128 = make_attn_entry<128>();
+
+// [BH][S][D] 16-bit tensor as a 3-D map (D innermost), box 64 x 128 x 1,
+// 128-byte swizzle: rows past S read as zero within each (batch, head).
+bool encode_3d_rows(CUtensorMap *map, const void *base, int dtype, int64_t BH, int64_t S, int64_t D)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(S * D) * 2};
+    const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapDataType dt = dtype == TL_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    return fn(map, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+tl_status attention_validate(const void *Q, const void *K, const void *V, void *O, const float *lse, int64_t batch,
+                             int64_t heads, int64_t seq_q, int64_t seq_k, int64_t head_dim, int dtype,
+                             float softmax_scale)
+{
+    if (!Q || !K || !V || !O)
+        return TL_ERR_INVALID_ARG;
+    if (batch < 1 || heads < 1 || seq_q < 1 || seq_k < 1)
+        return TL_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128)
+        return TL_ERR_UNSUPPORTED;
+    if (dtype != TL_F16 && dtype != TL_BF16)
+        return TL_ERR_INVALID_ARG;
+    if (!(softmax_scale >= 0.0f) || softmax_scale == INFINITY)
+        return TL_ERR_INVALID_ARG;
+    if (batch * heads > 65535 || seq_q > 0x7FFFFFFFll || seq_k > 0x7FFFFFFFll)
+        return TL_ERR_UNSUPPORTED;
+    if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || (lse && !aligned(lse, 4)))
+        return TL_ERR_MISALIGNED;
+    return TL_OK;
+}
+
+tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, float *lse, int64_t batch,
+                         int64_t heads, int64_t seq_q, int64_t seq_k, int64_t head_dim, int dtype, int causal,
+                         float softmax_scale, cudaStream_t stream)
+{
+    tl_status st = attention_validate(Q, K, V, O, lse, batch, heads, seq_q, seq_k, head_dim, dtype, softmax_scale);
+    if (st != TL_OK)
+        return st;
+    DeviceState *d = nullptr;
+    if ((st = device_state(&d)) != TL_OK)
+        return st;
+    if (d->cc_major != 10)
+        return TL_ERR_UNSUPPORTED;
+    const AttnEntry &e = head_dim == 64 ? kAttn64 : kAttn128;
+    AttnFn fn = e.fn[dtype];
+    if ((st = raise_smem_limit(d, reinterpret_cast<KernelFn>(fn), e.smem_bytes)) != TL_OK)
+        return st;
+    const int64_t BH = batch * heads;
+    CUtensorMap tq, tk, tv;
+    if (!encode_3d_rows(&tq, Q, dtype, BH, seq_q, head_dim) || !encode_3d_rows(&tk, K, dtype, BH, seq_k, head_dim) ||
+        !encode_3d_rows(&tv, V, dtype, BH, seq_k, head_dim))
+        return TL_ERR_CUDA;
+    AttnParams ap{};
+    ap.Sq = static_cast<int32_t>(seq_q);
+    ap.Sk = static_cast<int32_t>(seq_k);
+    ap.BH = static_cast<int32_t>(BH);
+    ap.num_qtiles = static_cast<int32_t>(ceil_div(seq_q, 128));
+    ap.causal = causal ? 1 : 0;
+    const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(head_dim));
+    ap.scale_log2 = scale * 1.4426950408889634f;
+    ap.O = static_cast<uint16_t *>(O);
+    ap.lse = lse;
+    ap.timeout_ns = kDefaultTimeoutNs;
+
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(static_cast<unsigned>(ap.num_qtiles), static_cast<unsigned>(BH), 1);
+    cfg.blockDim = dim3(192, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(e.smem_bytes);
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, fn, tq, tk, tv, ap) != cudaSuccess)
+        return TL_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ allocation-free entry point
 // The scratch area of tl_gemm_noalloc: file scope, one per device, reserved
 // when the module is loaded.  Host code may only use the address that
@@ -733,6 +843,14 @@ tl_status tl_gemm_ex(const void *A, const void *B, const void *bias, void *C, in
                      tl_dtype dtype, tl_epilogue epi, tl_stream stream, const tl_gemm_options *options)
 {
     return tl::gemm_impl(A, B, bias, C, M, N, K, dtype, epi, static_cast<cudaStream_t>(stream), options);
+}
+
+tl_status tl_attention_fwd(const void *Q, const void *K, const void *V, void *O, float *lse, int64_t batch,
+                           int64_t heads, int64_t seq_q, int64_t seq_k, int64_t head_dim, tl_dtype dtype,
+                           int32_t causal, float softmax_scale, tl_stream stream)
+{
+    return tl::attention_impl(Q, K, V, O, lse, batch, heads, seq_q, seq_k, head_dim, dtype, causal, softmax_scale,
+                              static_cast<cudaStream_t>(stream));
 }
 
 tl_status tl_check_device(tl_stream stream, uint32_t *detail)

@@ -210,3 +210,25 @@ def test_plan_transposed_b_pads_on_k():
     assert p["pad_a"] == 0 and p["pad_b"] == 0 and p["direct_store"] == 1
     p = tg.plan(512, 1001, 2048, tg.TL_BF16, None, num_sms=148)
     assert p["pad_b"] == 1
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(Q=0), tg.Status.INVALID_ARG),
+    (dict(O=0), tg.Status.INVALID_ARG),
+    (dict(batch=0), tg.Status.INVALID_ARG),
+    (dict(seq_k=0), tg.Status.INVALID_ARG),
+    (dict(head_dim=96), tg.Status.UNSUPPORTED),
+    (dict(head_dim=256), tg.Status.UNSUPPORTED),
+    (dict(dtype=5), tg.Status.INVALID_ARG),
+    (dict(scale=-1.0), tg.Status.INVALID_ARG),
+    (dict(scale=float("nan")), tg.Status.INVALID_ARG),
+    (dict(batch=256, heads=256), tg.Status.UNSUPPORTED),
+    (dict(K=P + 2), tg.Status.MISALIGNED),
+    (dict(lse=P + 2), tg.Status.MISALIGNED),
+])
+def test_attention_validation_before_any_cuda_call(args, status):
+    a = dict(Q=P, K=P, V=P, O=P, lse=0, batch=1, heads=2, seq_q=64, seq_k=64, head_dim=64, dtype=0, scale=0.0)
+    a.update(args)
+    st = tg.tl_attention_fwd(a["Q"], a["K"], a["V"], a["O"], a["lse"], a["batch"], a["heads"], a["seq_q"],
+                             a["seq_k"], a["head_dim"], a["dtype"], False, a["scale"], 0)
+    assert st == status
