@@ -20,6 +20,8 @@ What it computes, and where that is stated:
   * The same article, paragraph 6 (attention forward with online softmax,
     checked against PyTorch's scaled dot-product attention): the plain
     definition softmax(scale Q K^T) V, causal mask keeping key j <= query i.
+  * The same article, paragraphs 5 and 3: a row softmax, and a float32 vector
+    add (also the blog retelling, Step 3).
 """
 from __future__ import annotations
 
@@ -72,6 +74,10 @@ def _bind(path):
     lib.oracle_attention_rows.argtypes = [i64, i64, i64, i64, p, p, p, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_double, p, p, i64, p, p]
     lib.oracle_attention_rows.restype = ctypes.c_int
+    lib.oracle_softmax_rows.argtypes = [i64, i64, p, ctypes.c_int, p]
+    lib.oracle_softmax_rows.restype = ctypes.c_int
+    lib.oracle_vector_add.argtypes = [i64, p, p, p]
+    lib.oracle_vector_add.restype = None
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = ctypes.c_int
     return lib
@@ -192,6 +198,26 @@ class Oracle:
             return O.reshape(B, H, Sq, D), lse.reshape(B, H, Sq)
         return O, lse
 
+    def softmax_rows(self, X, dtype) -> np.ndarray:
+        """Row softmax of a (rows, cols) uint16 bit array, in fp64."""
+        X = _bits(X, "X")
+        if X.ndim != 2:
+            raise ValueError("X must be 2-D")
+        Y = np.empty(X.shape, np.float64)
+        if self._lib.oracle_softmax_rows(X.shape[0], X.shape[1], _ptr(X), dtype, _ptr(Y)) != 0:
+            raise ValueError("oracle_softmax_rows: bad size")
+        return Y
+
+    def vector_add(self, A, B) -> np.ndarray:
+        """A + B for float32 vectors, each sum rounded once to float32."""
+        A = np.ascontiguousarray(A, dtype=np.float32)
+        B = np.ascontiguousarray(B, dtype=np.float32)
+        if A.shape != B.shape:
+            raise ValueError("shapes differ")
+        C = np.empty_like(A)
+        self._lib.oracle_vector_add(A.size, _ptr(A), _ptr(B), _ptr(C))
+        return C
+
     def max_threads(self) -> int:
         """OpenMP threads the oracle uses (OMP_NUM_THREADS, else all cores)."""
         return int(self._lib.oracle_max_threads())
@@ -235,6 +261,16 @@ def gelu(x) -> np.ndarray:
 def attention(Q, K, V, dtype, causal, scale, rows=None):
     """softmax(scale Q K^T [causal]) V and its log-sum-exp, in fp64."""
     return _oracle().attention(Q, K, V, dtype, causal, scale, rows)
+
+
+def softmax_rows(X, dtype) -> np.ndarray:
+    """Row softmax in fp64."""
+    return _oracle().softmax_rows(X, dtype)
+
+
+def vector_add(A, B) -> np.ndarray:
+    """float32 A + B."""
+    return _oracle().vector_add(A, B)
 
 
 def max_threads() -> int:

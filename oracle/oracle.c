@@ -270,3 +270,46 @@ int oracle_attention_rows(int64_t BH, int64_t Sq, int64_t Sk, int64_t D,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Row softmax (TileLang GPU kernel design article, paragraph 5: a row-wise
+ * softmax with max and sum reductions): for each row x of a rows x cols
+ * matrix, y_j = exp(x_j - max x) / sum_k exp(x_k - max x), in fp64 from the
+ * 16-bit inputs.  Returns 0, or -1 for bad sizes.
+ * ------------------------------------------------------------------------ */
+int oracle_softmax_rows(int64_t rows, int64_t cols, const uint16_t *X, int dtype, double *Y)
+{
+    if (rows < 0 || cols < 1)
+        return -1;
+    int64_t r;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < rows; ++r) {
+        const uint16_t *x = X + r * cols;
+        double *y = Y + r * cols;
+        double m = -INFINITY;
+        for (int64_t j = 0; j < cols; ++j) {
+            y[j] = decode(x[j], dtype);
+            if (y[j] > m)
+                m = y[j];
+        }
+        double s = 0.0;
+        for (int64_t j = 0; j < cols; ++j) {
+            y[j] = exp(y[j] - m);
+            s += y[j];
+        }
+        for (int64_t j = 0; j < cols; ++j)
+            y[j] /= s;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Vector add (TileLang GPU kernel design article, paragraph 3; blog retelling,
+ * Step 3): C[i] = A[i] + B[i] in float32.  The sum of two floats is exact in
+ * double, so rounding it once to float gives the IEEE float32 sum.
+ * ------------------------------------------------------------------------ */
+void oracle_vector_add(int64_t n, const float *A, const float *B, float *C)
+{
+    for (int64_t i = 0; i < n; ++i)
+        C[i] = (float)((double)A[i] + (double)B[i]);
+}

@@ -11,6 +11,7 @@ sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 import oracle  # noqa: E402
 from oracle_pins import ALL_PINS  # noqa: E402
 from oracle_pins_attention import ATTENTION_PINS  # noqa: E402
+from oracle_pins_elementwise import ELEMENTWISE_PINS  # noqa: E402
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 
@@ -42,6 +43,12 @@ MUTANTS = [
     ("attn_v_from_query_row", "const uint16_t *v = V + (bh * Sk + j) * D;",
      "const uint16_t *v = V + (bh * Sk + (j + i) % Sk) * D;"),
     ("attn_lse_without_max", "lse[p] = m + log(l);", "lse[p] = log(l);"),
+    ("softmax_no_max_subtraction", "            y[j] = exp(y[j] - m);", "            y[j] = exp(y[j]);"),
+    ("softmax_unnormalised", "            y[j] /= s;", "            y[j] /= 1.0;"),
+    ("softmax_max_of_first_only", "            if (y[j] > m)\n                m = y[j];",
+     "            if (j == 0)\n                m = y[j];"),
+    ("vector_add_in_float_twice", "C[i] = (float)((double)A[i] + (double)B[i]);",
+     "C[i] = (float)((double)A[i] + (double)(float)(B[i] * 1.0000001f));"),
     ("f16_exponent_bias", "v = ldexp((double)(f + 1024), e - 25);", "v = ldexp((double)(f + 1024), e - 24);"),
     ("f16_subnormal_as_normal", "v = ldexp((double)f, -24);", "v = ldexp((double)(f + 1024), -25);"),
     ("bf16_exponent_bias", "v = ldexp((double)(f + 128), e - 134);", "v = ldexp((double)(f + 128), e - 133);"),
@@ -61,7 +68,7 @@ def test_mutant_fails_a_pin(tmp_path, name, old, new):
     so = oracle.build(force=True, src=str(csrc), out=str(tmp_path / f"liboracle_{name}.so"))
     orc = oracle.from_library(so)
     failed = []
-    for pin in ALL_PINS + ATTENTION_PINS:
+    for pin in ALL_PINS + ATTENTION_PINS + ELEMENTWISE_PINS:
         try:
             pin(orc)
         except AssertionError:

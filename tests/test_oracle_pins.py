@@ -6,6 +6,7 @@ import pytest
 import oracle
 from oracle_pins import ALL_PINS
 from oracle_pins_attention import ATTENTION_PINS
+from oracle_pins_elementwise import ELEMENTWISE_PINS
 
 
 @pytest.fixture(scope="module")
@@ -13,7 +14,7 @@ def orc():
     return oracle._oracle()
 
 
-@pytest.mark.parametrize("pin", ALL_PINS + ATTENTION_PINS, ids=lambda f: f.__name__)
+@pytest.mark.parametrize("pin", ALL_PINS + ATTENTION_PINS + ELEMENTWISE_PINS, ids=lambda f: f.__name__)
 def test_pin(orc, pin):
     pin(orc)
 
