@@ -166,6 +166,26 @@ TL_API tl_status tl_attention_fwd(const void *Q, const void *K, const void *V, v
                           int64_t batch, int64_t heads, int64_t seq_q, int64_t seq_k, int64_t head_dim,
                           tl_dtype dtype, int32_t causal, float softmax_scale, tl_stream stream);
 
+/*
+ * tl_softmax_rows -- Y[r, :] = softmax(X[r, :]) for each of `rows` rows of
+ * `cols` values (the TileLang GPU kernel design article, paragraph 5: a
+ * row-wise softmax with max and sum reductions).  X and Y are device pointers
+ * to rows x cols row-major `dtype` values (2-byte aligned; 16-byte aligned with
+ * cols a multiple of 8 for the vectorised path); Y may equal X.  Computed in
+ * fp32 with the row maximum subtracted, rounded once to `dtype`.  rows, cols
+ * >= 1.  Asynchronous on `stream`; allocates nothing.
+ */
+TL_API tl_status tl_softmax_rows(const void *X, void *Y, int64_t rows, int64_t cols, tl_dtype dtype,
+                         tl_stream stream);
+
+/*
+ * tl_vector_add -- C[i] = A[i] + B[i] for i < n, float32 (the same article,
+ * paragraph 3, and the blog retelling's Step 3: a bandwidth-bound kernel).
+ * Device pointers, 4-byte aligned (16-byte aligned for the vectorised path);
+ * n >= 1.  Asynchronous on `stream`; allocates nothing.
+ */
+TL_API tl_status tl_vector_add(const float *A, const float *B, float *C, int64_t n, tl_stream stream);
+
 /* Options for tl_gemm_ex.  Zero-initialise, then set what you need. */
 typedef struct {
     int32_t config;       /* 0: the library's choice for the shape; k > 0: kernel

@@ -16,12 +16,13 @@ from ._binding import (  # noqa: F401
     LIB_PATH, Options, Plan, Status, TLError, TL_BF16, TL_EPI_BIAS, TL_EPI_BIAS_GELU, TL_EPI_GELU,
     TL_EPI_NONE, TL_F16,
     SIGNATURES, tl_attention_fwd, tl_check_device, tl_config_name, tl_gemm, tl_gemm_ex, tl_gemm_noalloc,
-    tl_gemm_plan, tl_num_configs,
+    tl_gemm_plan, tl_num_configs, tl_softmax_rows, tl_vector_add,
     tl_status_string, tl_version,
 )
 
 __all__ = [
-    "gemm", "attention", "check_device", "plan", "configs", "tl_attention_fwd", "Options", "Plan", "Status", "TLError",
+    "gemm", "attention", "softmax", "vector_add", "check_device", "plan", "configs", "tl_attention_fwd",
+    "tl_softmax_rows", "tl_vector_add", "Options", "Plan", "Status", "TLError",
     "tl_gemm", "tl_gemm_ex", "tl_gemm_noalloc", "tl_check_device", "tl_gemm_plan", "tl_num_configs", "tl_config_name",
     "tl_status_string", "tl_version", "TL_F16", "TL_BF16", "TL_EPI_NONE", "TL_EPI_BIAS_GELU",
     "TL_EPI_BIAS", "TL_EPI_GELU",
@@ -122,6 +123,37 @@ def attention(q, k, v, causal: bool = False, scale: float = 0.0, out=None, lse=N
                               s.cuda_stream)
     if st != 0:
         raise TLError(st, "tl_attention_fwd")
+    return out
+
+
+def softmax(x, out=None, stream=None):
+    """Row softmax of a contiguous 2-D fp16/bf16 CUDA tensor (over the last dim)."""
+    import torch
+    if x.dim() != 2 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D CUDA tensor")
+    dt = _dtype_code(x)
+    out = torch.empty_like(x) if out is None else out
+    if out.shape != x.shape or out.dtype != x.dtype or not out.is_contiguous():
+        raise ValueError("out must match x")
+    s = stream if stream is not None else torch.cuda.current_stream(x.device)
+    with torch.cuda.device(x.device):
+        st = tl_softmax_rows(x.data_ptr(), out.data_ptr(), x.shape[0], x.shape[1], dt, s.cuda_stream)
+    if st != 0:
+        raise TLError(st, "tl_softmax_rows")
+    return out
+
+
+def vector_add(a, b, out=None, stream=None):
+    """a + b for contiguous float32 CUDA tensors of one shape."""
+    import torch
+    if a.shape != b.shape or a.dtype != torch.float32 or b.dtype != torch.float32 or not a.is_cuda:
+        raise ValueError("a and b must be float32 CUDA tensors of one shape")
+    out = torch.empty_like(a) if out is None else out
+    s = stream if stream is not None else torch.cuda.current_stream(a.device)
+    with torch.cuda.device(a.device):
+        st = tl_vector_add(a.data_ptr(), b.data_ptr(), out.data_ptr(), a.numel(), s.cuda_stream)
+    if st != 0:
+        raise TLError(st, "tl_vector_add")
     return out
 
 

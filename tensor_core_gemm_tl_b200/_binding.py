@@ -62,6 +62,8 @@ SIGNATURES = {
     "tl_gemm_ex": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, _P,
                                   ctypes.POINTER(Options)]),
     "tl_check_device": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "tl_softmax_rows": (ctypes.c_int, [_P, _P, _I64, _I64, ctypes.c_int, _P]),
+    "tl_vector_add": (ctypes.c_int, [_P, _P, _P, _I64, _P]),
     "tl_attention_fwd": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int, _I32,
                                         ctypes.c_float, _P]),
     "tl_gemm_plan": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, _I32,
@@ -115,6 +117,14 @@ def tl_attention_fwd(Q, K, V, O, lse, batch, heads, seq_q, seq_k, head_dim, dtyp
     """Attention forward on device pointers; returns the tl_status code."""
     return _lib.tl_attention_fwd(Q, K, V, O, lse or None, batch, heads, seq_q, seq_k, head_dim, dtype,
                                  int(bool(causal)), float(softmax_scale), stream or None)
+
+
+def tl_softmax_rows(X, Y, rows, cols, dtype, stream=0) -> int:
+    return _lib.tl_softmax_rows(X, Y, rows, cols, dtype, stream or None)
+
+
+def tl_vector_add(A, B, C, n, stream=0) -> int:
+    return _lib.tl_vector_add(A, B, C, n, stream or None)
 
 
 def tl_check_device(stream: int = 0) -> tuple[int, int]:

@@ -13,7 +13,12 @@ named workload it times
 with CUDA events over operands rotated beyond L2, median of the launches.
 It prints one JSON line per workload.  A diagnostic, not the benchmark.
 
-    python -m tensor_core_gemm_tl_b200.compare [--only name,...] [--launches 40]
+    python -m tensor_core_gemm_tl_b200.compare [--only name,...] [--launches 40] [--attention]
+
+With --attention it times tl_attention_fwd against PyTorch's
+scaled_dot_product_attention (bf16, random inputs) on a few
+transformer-sized shapes; with --rowwise, the row softmax and the vector add
+as achieved HBM GB/s against torch.softmax and torch.add.
 """
 from __future__ import annotations
 
@@ -90,13 +95,110 @@ def compare(w, launches=40, warmup=10):
     return res
 
 
+def attention_flops(B, H, Sq, Sk, D, causal):
+    """4 D flops per kept (query, key) pair: Q K^T and P V."""
+    if causal:
+        kept = sum(min(i + 1, Sk) for i in range(Sq))
+    else:
+        kept = Sq * Sk
+    return 4.0 * B * H * D * kept
+
+
+ATTENTION_SHAPES = [
+    # B, H, Sq, Sk, D, causal
+    (4, 16, 4096, 4096, 128, False),
+    (4, 16, 4096, 4096, 128, True),
+    (8, 16, 2048, 2048, 64, False),
+    (8, 16, 2048, 2048, 64, True),
+    (1, 32, 8192, 8192, 128, True),
+]
+
+
+def compare_attention(B, H, Sq, Sk, D, causal, launches=20, warmup=5):
+    import torch
+    import torch.nn.functional as F
+    import tensor_core_gemm_tl_b200 as tg
+    g = torch.Generator(device="cuda").manual_seed(0)
+    q = torch.randn(B, H, Sq, D, device="cuda", dtype=torch.bfloat16, generator=g)
+    k = torch.randn(B, H, Sk, D, device="cuda", dtype=torch.bfloat16, generator=g)
+    v = torch.randn(B, H, Sk, D, device="cuda", dtype=torch.bfloat16, generator=g)
+    out = torch.empty_like(q)
+
+    def ours(_):
+        tg.attention(q, k, v, causal=causal, out=out)
+
+    def sdpa(_):
+        F.scaled_dot_product_attention(q, k, v, is_causal=causal)
+
+    fl = attention_flops(B, H, Sq, Sk, D, causal)
+    res = {"attention": f"B{B} H{H} Sq{Sq} Sk{Sk} D{D}", "causal": causal, "dtype": "bf16"}
+    res["tl_attention_tflops"] = round(fl / _median_ms(ours, 1, launches, warmup) / 1e9, 1)
+    res["torch_sdpa_tflops"] = round(fl / _median_ms(sdpa, 1, launches, warmup) / 1e9, 1)
+    if tg.check_device() != 0:
+        raise RuntimeError("device error")
+    return res
+
+
+ROWWISE_SHAPES = [(16384, 8192), (65536, 1024), (4096, 50257), (262144, 128)]
+
+
+def compare_rowwise(launches=20, warmup=5):
+    """Achieved HBM bandwidth (compulsory bytes / time) of the row softmax and
+    the vector add against torch.softmax and torch.add."""
+    import torch
+    import tensor_core_gemm_tl_b200 as tg
+    out = []
+    for rows, cols in ROWWISE_SHAPES:
+        x = torch.randn(rows, cols, device="cuda", dtype=torch.bfloat16)
+        y = torch.empty_like(x)
+        nbytes = 2 * 2 * rows * cols
+
+        def ours(_):
+            tg.softmax(x, out=y)
+
+        def ref(_):
+            torch.softmax(x, dim=-1, out=y)
+
+        out.append({"softmax": f"{rows}x{cols} bf16",
+                    "tl_gbs": round(nbytes / _median_ms(ours, 1, launches, warmup) / 1e6, 1),
+                    "torch_gbs": round(nbytes / _median_ms(ref, 1, launches, warmup) / 1e6, 1)})
+    n = 1 << 28
+    a = torch.randn(n, device="cuda")
+    b = torch.randn(n, device="cuda")
+    c = torch.empty_like(a)
+
+    def ours_add(_):
+        tg.vector_add(a, b, out=c)
+
+    def ref_add(_):
+        torch.add(a, b, out=c)
+
+    nbytes = 3 * 4 * n
+    out.append({"vector_add": f"{n} float32",
+                "tl_gbs": round(nbytes / _median_ms(ours_add, 1, launches, warmup) / 1e6, 1),
+                "torch_gbs": round(nbytes / _median_ms(ref_add, 1, launches, warmup) / 1e6, 1)})
+    if tg.check_device() != 0:
+        raise RuntimeError("device error")
+    return out
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--only", default=None)
     ap.add_argument("--launches", type=int, default=40)
+    ap.add_argument("--attention", action="store_true", help="time attention forward instead of the GEMMs")
+    ap.add_argument("--rowwise", action="store_true", help="time the row softmax and the vector add")
     a = ap.parse_args(argv)
     import torch
     torch.cuda.set_device(0)
+    if a.attention:
+        for shape in ATTENTION_SHAPES:
+            print(json.dumps(compare_attention(*shape)), flush=True)
+        return 0
+    if a.rowwise:
+        for rec in compare_rowwise():
+            print(json.dumps(rec), flush=True)
+        return 0
     todo = list(wl.WORKLOADS.values())
     if a.only:
         keep = set(a.only.split(","))

@@ -17,6 +17,7 @@
 #include "tl_gemm.h"
 #include "gemm_kernel.cuh"
 #include "attention_kernel.cuh"
+#include "rowwise_kernels.cuh"
 
 namespace tl {
 namespace {
@@ -715,6 +716,80 @@ tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, f
     return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ row softmax and vector add
+tl_status softmax_impl(const void *X, void *Y, int64_t rows, int64_t cols, int dtype, cudaStream_t stream)
+{
+    if (!X || !Y || rows < 1 || cols < 1)
+        return TL_ERR_INVALID_ARG;
+    if (dtype != TL_F16 && dtype != TL_BF16)
+        return TL_ERR_INVALID_ARG;
+    if (cols > 0x7FFFFFFFll)
+        return TL_ERR_UNSUPPORTED;
+    if (!aligned(X, 2) || !aligned(Y, 2))
+        return TL_ERR_MISALIGNED;
+    DeviceState *d = nullptr;
+    tl_status st = device_state(&d);
+    if (st != TL_OK)
+        return st;
+    const bool vec = cols % 8 == 0 && aligned(X, 16) && aligned(Y, 16);
+    const uint16_t *x = static_cast<const uint16_t *>(X);
+    uint16_t *y = static_cast<uint16_t *>(Y);
+    const int c = static_cast<int>(cols);
+    if (cols <= 1024) {
+        int64_t blocks = ceil_div(rows, 8);
+        const int64_t cap = static_cast<int64_t>(d->num_sms) * 16;
+        if (blocks > cap)
+            blocks = cap;
+        const dim3 g(static_cast<unsigned>(blocks)), b(256);
+#define TL_SOFTMAX_WARP(DT)                                                                         \
+    do {                                                                                            \
+        if (cols <= 256)                                                                            \
+            vec ? softmax_rows_warp_kernel<DT, 8, true><<<g, b, 0, stream>>>(x, y, rows, c)         \
+                : softmax_rows_warp_kernel<DT, 8, false><<<g, b, 0, stream>>>(x, y, rows, c);       \
+        else                                                                                        \
+            vec ? softmax_rows_warp_kernel<DT, 32, true><<<g, b, 0, stream>>>(x, y, rows, c)        \
+                : softmax_rows_warp_kernel<DT, 32, false><<<g, b, 0, stream>>>(x, y, rows, c);      \
+    } while (0)
+        if (dtype == TL_BF16)
+            TL_SOFTMAX_WARP(1);
+        else
+            TL_SOFTMAX_WARP(0);
+#undef TL_SOFTMAX_WARP
+    } else {
+        int64_t blocks = rows;
+        const int64_t cap = static_cast<int64_t>(d->num_sms) * 4;
+        if (blocks > cap)
+            blocks = cap;
+        const dim3 g(static_cast<unsigned>(blocks)), b(cols <= 8192 ? 256 : 512);
+        if (dtype == TL_BF16)
+            vec ? softmax_rows_block_kernel<1, true><<<g, b, 0, stream>>>(x, y, rows, cols)
+                : softmax_rows_block_kernel<1, false><<<g, b, 0, stream>>>(x, y, rows, cols);
+        else
+            vec ? softmax_rows_block_kernel<0, true><<<g, b, 0, stream>>>(x, y, rows, cols)
+                : softmax_rows_block_kernel<0, false><<<g, b, 0, stream>>>(x, y, rows, cols);
+    }
+    return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ERR_CUDA;
+}
+
+tl_status vector_add_impl(const float *A, const float *B, float *C, int64_t n, cudaStream_t stream)
+{
+    if (!A || !B || !C || n < 1)
+        return TL_ERR_INVALID_ARG;
+    if (!aligned(A, 4) || !aligned(B, 4) || !aligned(C, 4))
+        return TL_ERR_MISALIGNED;
+    DeviceState *d = nullptr;
+    tl_status st = device_state(&d);
+    if (st != TL_OK)
+        return st;
+    const int vec = aligned(A, 16) && aligned(B, 16) && aligned(C, 16);
+    int64_t blocks = ceil_div(vec ? ceil_div(n, 4) : n, 256);
+    const int64_t cap = static_cast<int64_t>(d->num_sms) * 8;
+    if (blocks > cap)
+        blocks = cap;
+    vector_add_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(A, B, C, n, vec);
+    return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ allocation-free entry point
 // The scratch area of tl_gemm_noalloc: file scope, one per device, reserved
 // when the module is loaded.  Host code may only use the address that
@@ -851,6 +926,16 @@ tl_status tl_attention_fwd(const void *Q, const void *K, const void *V, void *O,
 {
     return tl::attention_impl(Q, K, V, O, lse, batch, heads, seq_q, seq_k, head_dim, dtype, causal, softmax_scale,
                               static_cast<cudaStream_t>(stream));
+}
+
+tl_status tl_softmax_rows(const void *X, void *Y, int64_t rows, int64_t cols, tl_dtype dtype, tl_stream stream)
+{
+    return tl::softmax_impl(X, Y, rows, cols, dtype, static_cast<cudaStream_t>(stream));
+}
+
+tl_status tl_vector_add(const float *A, const float *B, float *C, int64_t n, tl_stream stream)
+{
+    return tl::vector_add_impl(A, B, C, n, static_cast<cudaStream_t>(stream));
 }
 
 tl_status tl_check_device(tl_stream stream, uint32_t *detail)

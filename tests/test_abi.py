@@ -232,3 +232,14 @@ def test_attention_validation_before_any_cuda_call(args, status):
     st = tg.tl_attention_fwd(a["Q"], a["K"], a["V"], a["O"], a["lse"], a["batch"], a["heads"], a["seq_q"],
                              a["seq_k"], a["head_dim"], a["dtype"], False, a["scale"], 0)
     assert st == status
+
+
+def test_softmax_and_vector_add_validation():
+    assert tg.tl_softmax_rows(0, P, 4, 4, 0, 0) == tg.Status.INVALID_ARG
+    assert tg.tl_softmax_rows(P, P, 0, 4, 0, 0) == tg.Status.INVALID_ARG
+    assert tg.tl_softmax_rows(P, P, 4, 0, 0, 0) == tg.Status.INVALID_ARG
+    assert tg.tl_softmax_rows(P, P, 4, 4, 9, 0) == tg.Status.INVALID_ARG
+    assert tg.tl_softmax_rows(P + 1, P, 4, 4, 0, 0) == tg.Status.MISALIGNED
+    assert tg.tl_vector_add(P, 0, P, 4, 0) == tg.Status.INVALID_ARG
+    assert tg.tl_vector_add(P, P, P, 0, 0) == tg.Status.INVALID_ARG
+    assert tg.tl_vector_add(P + 2, P, P, 4, 0) == tg.Status.MISALIGNED
