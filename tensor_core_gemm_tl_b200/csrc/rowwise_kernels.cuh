@@ -120,19 +120,109 @@ __global__ void __launch_bounds__(256) softmax_rows_warp_kernel(const uint16_t *
     }
 }
 
+// ------------------------------------------------------------------ row softmax, one CTA per row, in registers
+// Rows of up to THREADS * PER_THREAD values (16-byte aligned, a multiple of 8
+// long) are read once into registers; block reductions through shared memory.
+template <int DT, int PER_THREAD>
+__global__ void __launch_bounds__(512) softmax_rows_cta_regs_kernel(const uint16_t *__restrict__ X,
+                                                                    uint16_t *__restrict__ Y, int64_t rows, int cols)
+{
+    __shared__ float red[16];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    const int step = blockDim.x * 8;
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+        const uint16_t *x = X + row * cols;
+        uint16_t *y = Y + row * cols;
+        float v[PER_THREAD];
+        float m = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < PER_THREAD / 8; ++s) {
+            const int c = s * step + tid * 8;
+            if (c < cols) {
+                const uint4 w = __ldg(reinterpret_cast<const uint4 *>(x + c));
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    v[8 * s + 2 * h] = half_to_float<DT>(static_cast<uint16_t>(ww[h] & 0xFFFFu));
+                    v[8 * s + 2 * h + 1] = half_to_float<DT>(static_cast<uint16_t>(ww[h] >> 16));
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    v[8 * s + e] = -INFINITY;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < PER_THREAD; ++i)
+            m = fmaxf(m, v[i]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        if (lane == 0)
+            red[warp] = m;
+        __syncthreads();
+        m = red[0];
+        for (int w = 1; w < nwarps; ++w)
+            m = fmaxf(m, red[w]);
+        __syncthreads();
+        const float mb = m * kLog2e;
+        float sum = 0.0f;
+#pragma unroll
+        for (int i = 0; i < PER_THREAD; ++i) {
+            v[i] = exp2_approx(fmaf(v[i], kLog2e, -mb));
+            sum += v[i];
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (lane == 0)
+            red[warp] = sum;
+        __syncthreads();
+        sum = 0.0f;
+        for (int w = 0; w < nwarps; ++w)
+            sum += red[w];
+        __syncthreads();
+        const float inv = 1.0f / sum;
+#pragma unroll
+        for (int s = 0; s < PER_THREAD / 8; ++s) {
+            const int c = s * step + tid * 8;
+            if (c < cols) {
+                uint32_t o[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+                    o[h] = float_to_half<DT>(v[8 * s + 2 * h] * inv) |
+                           (static_cast<uint32_t>(float_to_half<DT>(v[8 * s + 2 * h + 1] * inv)) << 16);
+                *reinterpret_cast<uint4 *>(y + c) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ row softmax, one CTA per row
 // Any row length: pass 1 keeps a running (max, sum) per thread and merges
 // them across the block; pass 2 reads the row again (from L2 for rows of up
 // to a few hundred kilobytes) and writes y.
-template <int DT, bool VEC>
+template <int DT>
 __global__ void __launch_bounds__(512) softmax_rows_block_kernel(const uint16_t *__restrict__ X,
-                                                                 uint16_t *__restrict__ Y, int64_t rows, int64_t cols)
+                                                                 uint16_t *__restrict__ Y, int64_t rows, int64_t cols,
+                                                                 int peel)
 {
     __shared__ float red_m[16], red_s[16];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
         const uint16_t *x = X + row * cols;
         uint16_t *y = Y + row * cols;
+        // split the row into a head (up to 7 values before the first 16-byte
+        // boundary), a body of 8-value vectors and a tail; without `peel` (x
+        // and y differently aligned) everything is handled value by value
+        int64_t head = 0, nvec = 0;
+        if (peel) {
+            head = ((16 - (reinterpret_cast<uintptr_t>(x) & 15)) & 15) >> 1;
+            if (head > cols)
+                head = cols;
+            nvec = (cols - head) >> 3;
+        }
+        const int64_t body_end = head + (nvec << 3);
         float m = -INFINITY, s = 0.0f;  // in log2 units: s = sum 2^(t - m)
         auto absorb = [&](float t) {
             if (t > m) {
@@ -142,20 +232,31 @@ __global__ void __launch_bounds__(512) softmax_rows_block_kernel(const uint16_t 
                 s += exp2_approx(t - m);
             }
         };
-        if constexpr (VEC) {
-            for (int64_t c = static_cast<int64_t>(tid) * 8; c < cols; c += static_cast<int64_t>(blockDim.x) * 8) {
-                const uint4 w = __ldg(reinterpret_cast<const uint4 *>(x + c));
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int64_t c = tid; c < head; c += blockDim.x)
+            absorb(half_to_float<DT>(x[c]) * kLog2e);
+        for (int64_t i = tid; i < nvec; i += blockDim.x) {
+            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(x + head) + i);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+            float t[8];
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    absorb(half_to_float<DT>(static_cast<uint16_t>(ww[h] & 0xFFFFu)) * kLog2e);
-                    absorb(half_to_float<DT>(static_cast<uint16_t>(ww[h] >> 16)) * kLog2e);
-                }
+            for (int h = 0; h < 4; ++h) {
+                t[2 * h] = half_to_float<DT>(static_cast<uint16_t>(ww[h] & 0xFFFFu)) * kLog2e;
+                t[2 * h + 1] = half_to_float<DT>(static_cast<uint16_t>(ww[h] >> 16)) * kLog2e;
             }
-        } else {
-            for (int64_t c = tid; c < cols; c += blockDim.x)
-                absorb(half_to_float<DT>(x[c]) * kLog2e);
+            float mx = t[0];
+#pragma unroll
+            for (int e = 1; e < 8; ++e)
+                mx = fmaxf(mx, t[e]);
+            if (mx > m) {
+                s = (m == -INFINITY) ? 0.0f : s * exp2_approx(m - mx);
+                m = mx;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                s += exp2_approx(t[e] - m);
         }
+        for (int64_t c = body_end + tid; c < cols; c += blockDim.x)
+            absorb(half_to_float<DT>(x[c]) * kLog2e);
         // merge (m, s) across the warp, then across warps
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
@@ -179,23 +280,22 @@ __global__ void __launch_bounds__(512) softmax_rows_block_kernel(const uint16_t 
                 S += red_s[w] * exp2_approx(red_m[w] - M);
         __syncthreads();  // red_* reused by the next row
         const float inv = 1.0f / S;
-        if constexpr (VEC) {
-            for (int64_t c = static_cast<int64_t>(tid) * 8; c < cols; c += static_cast<int64_t>(blockDim.x) * 8) {
-                const uint4 w = __ldg(reinterpret_cast<const uint4 *>(x + c));
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-                uint32_t o[4];
+        for (int64_t c = tid; c < head; c += blockDim.x)
+            y[c] = float_to_half<DT>(exp2_approx(fmaf(half_to_float<DT>(x[c]), kLog2e, -M)) * inv);
+        for (int64_t i = tid; i < nvec; i += blockDim.x) {
+            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(x + head) + i);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+            uint32_t o[4];
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const float a = exp2_approx(fmaf(half_to_float<DT>(static_cast<uint16_t>(ww[h] & 0xFFFFu)), kLog2e, -M)) * inv;
-                    const float b = exp2_approx(fmaf(half_to_float<DT>(static_cast<uint16_t>(ww[h] >> 16)), kLog2e, -M)) * inv;
-                    o[h] = float_to_half<DT>(a) | (static_cast<uint32_t>(float_to_half<DT>(b)) << 16);
-                }
-                *reinterpret_cast<uint4 *>(y + c) = make_uint4(o[0], o[1], o[2], o[3]);
+            for (int h = 0; h < 4; ++h) {
+                const float a = exp2_approx(fmaf(half_to_float<DT>(static_cast<uint16_t>(ww[h] & 0xFFFFu)), kLog2e, -M)) * inv;
+                const float b = exp2_approx(fmaf(half_to_float<DT>(static_cast<uint16_t>(ww[h] >> 16)), kLog2e, -M)) * inv;
+                o[h] = float_to_half<DT>(a) | (static_cast<uint32_t>(float_to_half<DT>(b)) << 16);
             }
-        } else {
-            for (int64_t c = tid; c < cols; c += blockDim.x)
-                y[c] = float_to_half<DT>(exp2_approx(fmaf(half_to_float<DT>(x[c]), kLog2e, -M)) * inv);
+            reinterpret_cast<uint4 *>(y + head)[i] = make_uint4(o[0], o[1], o[2], o[3]);
         }
+        for (int64_t c = body_end + tid; c < cols; c += blockDim.x)
+            y[c] = float_to_half<DT>(exp2_approx(fmaf(half_to_float<DT>(x[c]), kLog2e, -M)) * inv);
     }
 }
 
@@ -210,7 +310,19 @@ __global__ void __launch_bounds__(256) vector_add_kernel(const float *__restrict
         const float4 *a4 = reinterpret_cast<const float4 *>(A);
         const float4 *b4 = reinterpret_cast<const float4 *>(B);
         float4 *c4 = reinterpret_cast<float4 *>(C);
-        for (int64_t i = t; i < n4; i += stride) {
+        int64_t i = t;
+        for (; i + 3 * stride < n4; i += 4 * stride) {  // four vectors in flight per thread
+            float4 a[4], b[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                a[u] = __ldcs(a4 + i + u * stride);
+                b[u] = __ldcs(b4 + i + u * stride);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                __stcs(c4 + i + u * stride, make_float4(a[u].x + b[u].x, a[u].y + b[u].y, a[u].z + b[u].z, a[u].w + b[u].w));
+        }
+        for (; i < n4; i += stride) {
             const float4 a = __ldcs(a4 + i), b = __ldcs(b4 + i);
             __stcs(c4 + i, make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w));
         }

@@ -755,18 +755,36 @@ tl_status softmax_impl(const void *X, void *Y, int64_t rows, int64_t cols, int d
         else
             TL_SOFTMAX_WARP(0);
 #undef TL_SOFTMAX_WARP
+    } else if (vec && cols <= 16384) {
+        // the row in registers: 512 threads x up to 32 values, one read
+        int64_t blocks = rows;
+        const int64_t cap = static_cast<int64_t>(d->num_sms) * 4;
+        if (blocks > cap)
+            blocks = cap;
+        const dim3 g(static_cast<unsigned>(blocks)), b(cols <= 4096 ? 256 : 512);
+        if (cols <= 8192) {
+            if (dtype == TL_BF16)
+                softmax_rows_cta_regs_kernel<1, 16><<<g, b, 0, stream>>>(x, y, rows, c);
+            else
+                softmax_rows_cta_regs_kernel<0, 16><<<g, b, 0, stream>>>(x, y, rows, c);
+        } else {
+            if (dtype == TL_BF16)
+                softmax_rows_cta_regs_kernel<1, 32><<<g, b, 0, stream>>>(x, y, rows, c);
+            else
+                softmax_rows_cta_regs_kernel<0, 32><<<g, b, 0, stream>>>(x, y, rows, c);
+        }
     } else {
         int64_t blocks = rows;
         const int64_t cap = static_cast<int64_t>(d->num_sms) * 4;
         if (blocks > cap)
             blocks = cap;
-        const dim3 g(static_cast<unsigned>(blocks)), b(cols <= 8192 ? 256 : 512);
+        const dim3 g(static_cast<unsigned>(blocks)), b(512);
+        // vectors in the body of every row when x and y sit equally far from a 16-byte boundary
+        const int peel = ((reinterpret_cast<uintptr_t>(X) - reinterpret_cast<uintptr_t>(Y)) & 15) == 0;
         if (dtype == TL_BF16)
-            vec ? softmax_rows_block_kernel<1, true><<<g, b, 0, stream>>>(x, y, rows, cols)
-                : softmax_rows_block_kernel<1, false><<<g, b, 0, stream>>>(x, y, rows, cols);
+            softmax_rows_block_kernel<1><<<g, b, 0, stream>>>(x, y, rows, cols, peel);
         else
-            vec ? softmax_rows_block_kernel<0, true><<<g, b, 0, stream>>>(x, y, rows, cols)
-                : softmax_rows_block_kernel<0, false><<<g, b, 0, stream>>>(x, y, rows, cols);
+            softmax_rows_block_kernel<0><<<g, b, 0, stream>>>(x, y, rows, cols, peel);
     }
     return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ERR_CUDA;
 }
@@ -783,7 +801,7 @@ tl_status vector_add_impl(const float *A, const float *B, float *C, int64_t n, c
         return st;
     const int vec = aligned(A, 16) && aligned(B, 16) && aligned(C, 16);
     int64_t blocks = ceil_div(vec ? ceil_div(n, 4) : n, 256);
-    const int64_t cap = static_cast<int64_t>(d->num_sms) * 8;
+    const int64_t cap = static_cast<int64_t>(d->num_sms) * 16;
     if (blocks > cap)
         blocks = cap;
     vector_add_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(A, B, C, n, vec);

@@ -33,7 +33,8 @@ def run_softmax(X_bits, dt, offset=0):
 
 
 @pytest.mark.parametrize("rows,cols", [(1, 1), (3, 7), (64, 33), (1000, 256), (257, 1000), (128, 1024),
-                                       (40, 1025), (17, 4096), (8, 50000), (2, 200000)])
+                                       (40, 1025), (17, 4096), (9, 12288), (8, 50000), (3, 50257),
+                                       (2, 200000)])
 @pytest.mark.parametrize("dt", [wl.F16, wl.BF16])
 def test_softmax_vs_oracle(rows, cols, dt):
     rng = np.random.default_rng(rows * 7 + cols)
