@@ -16,7 +16,8 @@ What it computes, and where that is stated:
     exact.
   * TileLang GPU kernel design article, paragraph 5 (fused GEMM epilogue):
     bias add then GELU on the accumulator before the single store; bias is
-    per column, GELU is the exact erf form.
+    per column, GELU is the exact erf form (epilogues 1-3) or the tanh form
+    of the GELU paper (epilogues 4, 5).
   * The same article, paragraph 6 (attention forward with online softmax,
     checked against PyTorch's scaled dot-product attention): the plain
     definition softmax(scale Q K^T) V, causal mask keeping key j <= query i.
@@ -38,6 +39,9 @@ EPI_NONE = 0
 EPI_BIAS_GELU = 1
 EPI_BIAS = 2
 EPI_GELU = 3
+EPI_BIAS_GELU_TANH = 4
+EPI_GELU_TANH = 5
+EPI_WITH_BIAS = (EPI_BIAS_GELU, EPI_BIAS, EPI_BIAS_GELU_TANH)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
@@ -71,6 +75,8 @@ def _bind(path):
     lib.oracle_decode_array.restype = None
     lib.oracle_gelu_array.argtypes = [p, p, i64]
     lib.oracle_gelu_array.restype = None
+    lib.oracle_gelu_tanh_array.argtypes = [p, p, i64]
+    lib.oracle_gelu_tanh_array.restype = None
     lib.oracle_attention_rows.argtypes = [i64, i64, i64, i64, p, p, p, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_double, p, p, i64, p, p]
     lib.oracle_attention_rows.restype = ctypes.c_int
@@ -105,10 +111,10 @@ def _ptr(a):
 def _check_shapes(A, B, bias, epi):
     if A.ndim != 2 or B.ndim != 2 or A.shape[1] != B.shape[0]:
         raise ValueError(f"shapes A{A.shape} B{B.shape} do not chain")
-    if epi in (EPI_BIAS_GELU, EPI_BIAS):
+    if epi in EPI_WITH_BIAS:
         if bias is None or bias.shape != (B.shape[1],):
             raise ValueError("this epilogue needs a bias of length N")
-    elif epi not in (EPI_NONE, EPI_GELU):
+    elif epi not in (EPI_NONE, EPI_GELU, EPI_GELU_TANH):
         raise ValueError(f"unknown epilogue {epi}")
 
 
@@ -167,6 +173,13 @@ class Oracle:
         a = np.ascontiguousarray(x, dtype=np.float64)
         out = np.empty(a.shape, np.float64)
         self._lib.oracle_gelu_array(_ptr(a), _ptr(out), a.size)
+        return out
+
+    def gelu_tanh(self, x) -> np.ndarray:
+        """Tanh-form GELU 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) in fp64."""
+        a = np.ascontiguousarray(x, dtype=np.float64)
+        out = np.empty(a.shape, np.float64)
+        self._lib.oracle_gelu_tanh_array(_ptr(a), _ptr(out), a.size)
         return out
 
     def attention(self, Q, K, V, dtype, causal, scale, rows=None):
@@ -256,6 +269,11 @@ def decode(bits, dtype) -> np.ndarray:
 def gelu(x) -> np.ndarray:
     """Exact GELU x * Phi(x) in fp64, elementwise."""
     return _oracle().gelu(x)
+
+
+def gelu_tanh(x) -> np.ndarray:
+    """Tanh-form GELU in fp64, elementwise."""
+    return _oracle().gelu_tanh(x)
 
 
 def attention(Q, K, V, dtype, causal, scale, rows=None):

@@ -2,6 +2,7 @@
  * oracle.c -- plain fp64 CPU oracle for the fused tensor-core GEMM
  *
  *     C = epilogue(A . B),   epilogue(x)[i,j] = GELU(x[i,j] + bias[j])  or  identity
+ *     (or bias only, GELU only, and the tanh form of GELU with or without bias)
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check of the build
  * entry point and the CPU-baseline leg of the benchmark may load this file.
@@ -32,12 +33,18 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+#ifndef M_PI
+#define M_PI 3.14159265358979323846
+#endif
+
 #define ORACLE_F16 0
 #define ORACLE_BF16 1
 #define ORACLE_EPI_NONE 0
 #define ORACLE_EPI_BIAS_GELU 1
 #define ORACLE_EPI_BIAS 2
 #define ORACLE_EPI_GELU 3
+#define ORACLE_EPI_BIAS_GELU_TANH 4
+#define ORACLE_EPI_GELU_TANH 5
 
 /* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits.
  * Normal: (1024 + f) * 2^(e - 25).  Subnormal (e = 0): f * 2^-24.          */
@@ -87,6 +94,45 @@ double oracle_gelu(double x)
     return 0.5 * x * erfc(-x / sqrt(2.0));
 }
 
+/* Tanh form of GELU (Hendrycks and Gimpel, "Gaussian Error Linear Units",
+ * the approximation of Phi by the logistic-tanh curve):
+ *     g(x) = 0.5 x (1 + tanh(u)),   u = sqrt(2 / pi) (x + 0.044715 x^3).
+ * Computed through the identity 0.5 (1 + tanh u) = 1 / (1 + exp(-2u))
+ * = exp(2u) / (1 + exp(2u)), the same function, taking the form whose
+ * exponential is at most 1: for negative x the 1 + tanh form subtracts two
+ * numbers close to 1 (in fp64 it is already 0 at x = -7, where g is about
+ * -1e-19), and exp(-2u) alone overflows before g leaves the subnormals.     */
+double oracle_gelu_tanh(double x)
+{
+    const double u = sqrt(2.0 / M_PI) * (x + 0.044715 * x * x * x);
+    const double e = exp(-2.0 * fabs(u));
+    return u >= 0.0 ? x / (1.0 + e) : x * e / (1.0 + e);
+}
+
+void oracle_gelu_tanh_array(const double *x, double *y, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        y[i] = oracle_gelu_tanh(x[i]);
+}
+
+static int epi_has_bias(int epi)
+{
+    return epi == ORACLE_EPI_BIAS_GELU || epi == ORACLE_EPI_BIAS || epi == ORACLE_EPI_BIAS_GELU_TANH;
+}
+
+/* The epilogue on one accumulated value s of column j: bias first, then the
+ * activation (article, paragraph 5: bias add, then GELU). */
+static double epilogue(double s, const uint16_t *bias, int64_t j, int dtype, int epi)
+{
+    if (epi_has_bias(epi))
+        s = s + decode(bias[j], dtype);
+    if (epi == ORACLE_EPI_BIAS_GELU || epi == ORACLE_EPI_GELU)
+        s = oracle_gelu(s);
+    else if (epi == ORACLE_EPI_BIAS_GELU_TANH || epi == ORACLE_EPI_GELU_TANH)
+        s = oracle_gelu_tanh(s);
+    return s;
+}
+
 void oracle_gelu_array(const double *x, double *y, int64_t n)
 {
     for (int64_t i = 0; i < n; ++i)
@@ -109,7 +155,7 @@ int oracle_gemm_rows(int64_t M, int64_t N, int64_t K,
     for (int64_t r = 0; r < nrows; ++r)
         if (rows[r] < 0 || rows[r] >= M)
             return -1;
-    if ((epi == ORACLE_EPI_BIAS_GELU || epi == ORACLE_EPI_BIAS) && bias == NULL)
+    if (epi < ORACLE_EPI_NONE || epi > ORACLE_EPI_GELU_TANH || (epi_has_bias(epi) && bias == NULL))
         return -1;
 
     /* B decoded once; every row reads all of it. */
@@ -132,15 +178,8 @@ int oracle_gemm_rows(int64_t M, int64_t N, int64_t K,
             for (int64_t j = 0; j < N; ++j)
                 c[j] += a * b[j];
         }
-        if (epi == ORACLE_EPI_BIAS_GELU)
-            for (int64_t j = 0; j < N; ++j)
-                c[j] = oracle_gelu(c[j] + decode(bias[j], dtype));
-        else if (epi == ORACLE_EPI_BIAS)
-            for (int64_t j = 0; j < N; ++j)
-                c[j] = c[j] + decode(bias[j], dtype);
-        else if (epi == ORACLE_EPI_GELU)
-            for (int64_t j = 0; j < N; ++j)
-                c[j] = oracle_gelu(c[j]);
+        for (int64_t j = 0; j < N; ++j)
+            c[j] = epilogue(c[j], bias, j, dtype, epi);
     }
     free(Bd);
     return 0;
@@ -170,7 +209,7 @@ int oracle_gemm_points(int64_t M, int64_t N, int64_t K,
     for (int64_t p = 0; p < npts; ++p)
         if (ii[p] < 0 || ii[p] >= M || jj[p] < 0 || jj[p] >= N)
             return -1;
-    if ((epi == ORACLE_EPI_BIAS_GELU || epi == ORACLE_EPI_BIAS) && bias == NULL)
+    if (epi < ORACLE_EPI_NONE || epi > ORACLE_EPI_GELU_TANH || (epi_has_bias(epi) && bias == NULL))
         return -1;
     int64_t p;
 #pragma omp parallel for schedule(static)
@@ -179,13 +218,7 @@ int oracle_gemm_points(int64_t M, int64_t N, int64_t K,
         double s = 0.0;
         for (int64_t k = 0; k < K; ++k)
             s += decode(A[i * K + k], dtype) * decode(B[k * N + j], dtype);
-        if (epi == ORACLE_EPI_BIAS_GELU)
-            s = oracle_gelu(s + decode(bias[j], dtype));
-        else if (epi == ORACLE_EPI_BIAS)
-            s = s + decode(bias[j], dtype);
-        else if (epi == ORACLE_EPI_GELU)
-            s = oracle_gelu(s);
-        out[p] = s;
+        out[p] = epilogue(s, bias, j, dtype, epi);
     }
     return 0;
 }

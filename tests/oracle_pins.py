@@ -263,7 +263,8 @@ def pin_rows_and_points(orc, seed=19):
         A = rand_bits(rng, (M, K), dt, 1.0)
         B = rand_bits(rng, (K, N), dt, 1.0)
         bias = rand_bits(rng, (N,), dt, 0.5, "normal")
-        for epi, b in ((EPI_NONE, None), (EPI_BIAS_GELU, bias), (wl.EPI_BIAS, bias), (wl.EPI_GELU, None)):
+        for epi, b in ((EPI_NONE, None), (EPI_BIAS_GELU, bias), (wl.EPI_BIAS, bias), (wl.EPI_GELU, None),
+                       (wl.EPI_BIAS_GELU_TANH, bias), (wl.EPI_GELU_TANH, None)):
             full = orc.gemm(A, B, b, dt, epi)
             rows = np.array([22, 0, 5, 5, 17])
             assert np.array_equal(orc.gemm(A, B, b, dt, epi, rows=rows), full[rows])
@@ -336,10 +337,81 @@ def pin_gelu_tail_relative(orc):
         assert abs(g - ref) <= (1e-15 + 4e-16 * x * x) * abs(ref), (x, g, ref)
 
 
+# ---------------------------------------------------------------- tanh-form GELU
+def _mp_gelu_tanh(x):
+    """0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), the GELU paper's tanh
+    approximation, in mpmath (the caller sets the precision)."""
+    import mpmath
+    # 1 + tanh(u) loses about 0.87 |u| digits for u << 0: carry that many more
+    u = abs(0.7978845608028654 * (x + 0.044715 * x ** 3))
+    with mpmath.workdps(mpmath.mp.dps + int(0.87 * u) + 10):
+        xm = mpmath.mpf(x)
+        return +(xm / 2 * (1 + mpmath.tanh(mpmath.sqrt(2 / mpmath.pi) * (xm + mpmath.mpf("0.044715") * xm ** 3))))
+
+
+def pin_gelu_tanh_mpmath(orc):
+    """Relative accuracy over [-30, 30], tails included: mpmath at 40 digits."""
+    import mpmath
+    mpmath.mp.dps = 40
+    xs = np.concatenate([np.linspace(-30, -1, 300), np.linspace(-1, 1, 41), np.linspace(1, 30, 100)])
+    got = orc.gelu_tanh(xs)
+    for x, g in zip(xs, got):
+        ref = float(_mp_gelu_tanh(x))
+        # exp(-2u) carries the rounding of u: about |2u| u53 relative
+        u2 = abs(2 * 0.7978845608028654 * (x + 0.044715 * x ** 3))
+        assert abs(g - ref) <= (2e-15 + 4e-16 * u2) * abs(ref) + 1e-320, (x, g, ref)
+
+
+def pin_gelu_tanh_invariants(orc, seed=37):
+    """g(0) = 0; g(x) - g(-x) = x; and the approximation stays within its known
+    distance of the erf form (largest gap 4.7e-4, near x = -2.7)."""
+    rng = np.random.default_rng(seed)
+    assert orc.gelu_tanh(np.array([0.0]))[0] == 0.0
+    x = rng.normal(0, 3, 1000)
+    d = orc.gelu_tanh(x) - orc.gelu_tanh(-x)
+    assert np.all(np.abs(d - x) <= 1e-15 * (np.abs(x) + 1)), "odd part"
+    xs = np.linspace(-8, 8, 3201)
+    gap = np.max(np.abs(orc.gelu_tanh(xs) - orc.gelu(xs)))
+    assert 4.5e-4 < gap < 5.0e-4, gap
+
+
+def pin_exact_bruteforce_tanh_epilogue(orc, cases=16, seed=101):
+    """Bias + tanh GELU on tiny shapes: exact sum + bias (Fractions), then the
+    tanh form in mpmath; and tanh GELU alone with A = I: C = g(B)."""
+    import mpmath
+    mpmath.mp.dps = 40
+    rng = np.random.default_rng(seed)
+    for t in range(cases):
+        dt = (F16, BF16)[t % 2]
+        M, N, K = (int(v) for v in rng.integers(1, 9, size=3))
+        A = rand_bits(rng, (M, K), dt, 1.0)
+        B = rand_bits(rng, (K, N), dt, 1.0)
+        bias = rand_bits(rng, (N,), dt, 1.0, "normal")
+        C = orc.gemm(A, B, bias, dt, wl.EPI_BIAS_GELU_TANH)
+        Ae, Be = exact_values(A, dt), exact_values(B, dt)
+        be = exact_values(bias, dt)[0]
+        for i in range(M):
+            for j in range(N):
+                x = sum((Ae[i][k] * Be[k][j] for k in range(K)), Fraction(0)) + be[j]
+                ref = float(_mp_gelu_tanh(mpmath.mpf(x.numerator) / x.denominator))
+                assert abs(C[i, j] - ref) <= 1e-14 * (abs(ref) + abs(float(x))) + 1e-300, (t, i, j)
+    for dt in (F16, BF16):
+        n = 12
+        A = wl.round_to_bits(np.eye(n, dtype=np.float32), dt)
+        B = rand_bits(rng, (n, n), dt, 4.0, "normal")
+        C = orc.gemm(A, B, None, dt, wl.EPI_GELU_TANH)
+        Bf = wl.bits_to_float32(B, dt)
+        for i in range(n):
+            for j in range(n):
+                ref = float(_mp_gelu_tanh(float(Bf[i, j])))
+                assert abs(C[i, j] - ref) <= 1e-14 * (abs(ref) + 1e-3), (i, j)
+
+
 ALL_PINS = [
     pin_decode_all_patterns, pin_hand_example, pin_exact_bruteforce,
     pin_exact_bruteforce_epilogue, pin_vs_numpy_matmul, pin_identity, pin_row_sums,
     pin_all_ones, pin_zero_B_gelu_table, pin_bias_then_gelu, pin_transpose,
     pin_power_of_two_scaling, pin_rows_and_points, pin_gelu_table, pin_gelu_invariants,
     pin_gelu_tail_relative, pin_bias_only_and_gelu_only,
+    pin_gelu_tanh_mpmath, pin_gelu_tanh_invariants, pin_exact_bruteforce_tanh_epilogue,
 ]

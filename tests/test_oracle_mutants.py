@@ -28,13 +28,28 @@ MUTANTS = [
     ("gelu_cancelling_form", "return 0.5 * x * erfc(-x / sqrt(2.0));",
      "return 0.5 * x * (1.0 + erf(x / sqrt(2.0)));"),
     ("gelu_wrong_sign_in_erfc", "erfc(-x / sqrt(2.0))", "erfc(x / sqrt(2.0))"),
-    ("bias_after_gelu", "c[j] = oracle_gelu(c[j] + decode(bias[j], dtype));",
-     "c[j] = oracle_gelu(c[j]) + decode(bias[j], dtype);"),
-    ("bias_by_row", "c[j] = oracle_gelu(c[j] + decode(bias[j], dtype));",
-     "c[j] = oracle_gelu(c[j] + decode(bias[i % N], dtype));"),
-    ("bias_only_drops_bias", "c[j] = c[j] + decode(bias[j], dtype);", "c[j] = c[j];"),
-    ("gelu_only_adds_bias", "            s = oracle_gelu(s);", "            s = oracle_gelu(s + 1.0);"),
-    ("gelu_only_rows_skip_gelu", "                c[j] = oracle_gelu(c[j]);", "                c[j] = c[j];"),
+    ("bias_after_gelu",
+     "    if (epi_has_bias(epi))\n        s = s + decode(bias[j], dtype);\n"
+     "    if (epi == ORACLE_EPI_BIAS_GELU || epi == ORACLE_EPI_GELU)\n        s = oracle_gelu(s);",
+     "    if (epi == ORACLE_EPI_BIAS_GELU || epi == ORACLE_EPI_GELU)\n        s = oracle_gelu(s);\n"
+     "    if (epi_has_bias(epi))\n        s = s + decode(bias[j], dtype);"),
+    ("bias_by_row", "c[j] = epilogue(c[j], bias, j, dtype, epi);", "c[j] = epilogue(c[j], bias, i % N, dtype, epi);"),
+    ("bias_only_drops_bias", "return epi == ORACLE_EPI_BIAS_GELU || epi == ORACLE_EPI_BIAS || ",
+     "return epi == ORACLE_EPI_BIAS_GELU || "),
+    ("gelu_only_adds_bias", "        s = oracle_gelu(s);", "        s = oracle_gelu(epi == ORACLE_EPI_GELU ? s + 1.0 : s);"),
+    ("gelu_only_skips_gelu", "if (epi == ORACLE_EPI_BIAS_GELU || epi == ORACLE_EPI_GELU)", "if (epi == ORACLE_EPI_BIAS_GELU)"),
+    ("tanh_epilogue_uses_erf", "s = oracle_gelu_tanh(s);", "s = oracle_gelu(s);"),
+    ("tanh_without_cubic", "(x + 0.044715 * x * x * x)", "(x)"),
+    ("tanh_wrong_cubic_coefficient", "0.044715 * x * x * x", "0.04715 * x * x * x"),
+    ("tanh_wrong_scale", "sqrt(2.0 / M_PI)", "sqrt(1.0 / M_PI)"),
+    ("tanh_cancelling_form", "return u >= 0.0 ? x / (1.0 + e) : x * e / (1.0 + e);",
+     "return 0.5 * x * (1.0 + tanh(u));"),
+    ("tanh_overflowing_form", "return u >= 0.0 ? x / (1.0 + e) : x * e / (1.0 + e);",
+     "return x / (1.0 + exp(-2.0 * u));"),
+    ("tanh_branches_swapped", "return u >= 0.0 ? x / (1.0 + e)", "return u < 0.0 ? x / (1.0 + e)"),
+    ("tanh_bias_dropped", " || epi == ORACLE_EPI_BIAS_GELU_TANH;", ";"),
+    ("tanh_only_skips_gelu", "else if (epi == ORACLE_EPI_BIAS_GELU_TANH || epi == ORACLE_EPI_GELU_TANH)",
+     "else if (epi == ORACLE_EPI_BIAS_GELU_TANH)"),
     ("attn_mask_wrong_direction", "const int64_t nkeys = causal ? (i + 1 < Sk ? i + 1 : Sk) : Sk;",
      "const int64_t nkeys = causal ? (i < Sk ? i : Sk) + (i == 0) : Sk;"),
     ("attn_scale_ignored", "s[j] = scale * acc;", "s[j] = acc;"),

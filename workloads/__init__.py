@@ -27,6 +27,8 @@ import numpy as np
 
 F16, BF16 = 0, 1
 EPI_NONE, EPI_BIAS_GELU, EPI_BIAS, EPI_GELU = 0, 1, 2, 3
+EPI_BIAS_GELU_TANH, EPI_GELU_TANH = 4, 5
+EPI_WITH_BIAS = (EPI_BIAS_GELU, EPI_BIAS, EPI_BIAS_GELU_TANH)
 DTYPE_NAMES = {F16: "f16", BF16: "bf16"}
 
 
@@ -152,7 +154,7 @@ def make_inputs(w: Workload, seed: int = 0):
     """(A_bits, B_bits, bias_bits|None) for workload `w`, as uint16 arrays."""
     A = round_to_bits(draw(w.a, (w.M, w.K), seed), w.dtype)
     B = round_to_bits(draw(w.b, (w.K, w.N), seed + 1), w.dtype)
-    bias = round_to_bits(draw(w.bias, (w.N,), seed + 2), w.dtype) if w.epi in (EPI_BIAS_GELU, EPI_BIAS) else None
+    bias = round_to_bits(draw(w.bias, (w.N,), seed + 2), w.dtype) if w.epi in EPI_WITH_BIAS else None
     return A, B, bias
 
 
@@ -160,4 +162,4 @@ def custom(name, M, N, K, dtype, epi, a=None, b=None, bias=None) -> Workload:
     """A workload of any shape with the given (or default unit-normal-ish) laws."""
     s = 1.0 / np.sqrt(max(K, 1))
     return Workload(name, M, N, K, dtype, epi, a or _u(1.0), b or _n(s),
-                    (bias or _n(0.1)) if epi in (EPI_BIAS_GELU, EPI_BIAS) else None)
+                    (bias or _n(0.1)) if epi in EPI_WITH_BIAS else None)
