@@ -196,6 +196,23 @@ __device__ __forceinline__ float exp2_approx(float x)
     return r;
 }
 
+// 2^x with subnormal results flushed to zero (a single MUFU op): for softmax
+// weights, where anything below 2^-126 of the row maximum is negligible.
+__device__ __forceinline__ float exp2_approx_ftz(float x)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// max(a, b, c) in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor (tcgen05), 128-byte swizzle:
 //   bits  0-13 start address >> 4     bits 16-29 leading byte offset >> 4
@@ -231,6 +248,23 @@ __host__ __device__ constexpr uint32_t mma_idesc_f16(int bf16, int m, int n, int
 // Wait until the grids this one depends on (the previous kernels on the
 // stream) have completed and their memory is visible; a no-op when the launch
 // did not allow overlap.
+// Per-warpgroup register budget (every warp of the warpgroup executes it).
+// The block's total stays the one it was launched with: the increases have to
+// fit in what the decreases give back.
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease()
+{
+    static_assert(N >= 24 && N <= 256 && N % 8 == 0, "setmaxnreg count");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase()
+{
+    static_assert(N >= 24 && N <= 256 && N % 8 == 0, "setmaxnreg count");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ void grid_dependency_wait()
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");

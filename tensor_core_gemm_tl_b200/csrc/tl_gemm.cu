@@ -613,6 +613,8 @@ using AttnFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, AttnParams);
 
 struct AttnEntry {
     int smem_bytes;
+    int threads;
+    int launch_regs;  // registers a thread the warpgroup register split needs at launch
     AttnFn fn[2];  // [dtype]
 };
 
@@ -622,6 +624,8 @@ AttnEntry make_attn_entry()
     using CF = AttnConfig<D>;
     AttnEntry e;
     e.smem_bytes = CF::SMEM_BYTES;
+    e.threads = CF::THREADS;
+    e.launch_regs = CF::LAUNCH_REGS;
     e.fn[0] = attention_fwd_kernel<CF, 0>;
     e.fn[1] = attention_fwd_kernel<CF, 1>;
     return e;
@@ -682,6 +686,15 @@ tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, f
         return TL_ERR_UNSUPPORTED;
     const AttnEntry &e = head_dim == 64 ? kAttn64 : kAttn128;
     AttnFn fn = e.fn[dtype];
+    {
+        // the kernel moves registers between warpgroups; that only fits if
+        // it is launched with at least launch_regs a thread
+        cudaFuncAttributes fa{};
+        if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess)
+            return TL_ERR_CUDA;
+        if (fa.numRegs < e.launch_regs)
+            return TL_ERR_UNSUPPORTED;
+    }
     if ((st = raise_smem_limit(d, reinterpret_cast<KernelFn>(fn), e.smem_bytes)) != TL_OK)
         return st;
     const int64_t BH = batch * heads;
@@ -704,7 +717,7 @@ tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, f
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];
     cfg.gridDim = dim3(static_cast<unsigned>(ap.num_qtiles), static_cast<unsigned>(BH), 1);
-    cfg.blockDim = dim3(192, 1, 1);
+    cfg.blockDim = dim3(static_cast<unsigned>(e.threads), 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(e.smem_bytes);
     cfg.stream = stream;
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
