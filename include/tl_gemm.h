@@ -36,7 +36,7 @@
 extern "C" {
 #endif
 
-#define TL_VERSION 1000 /* major * 1000 + minor */
+#define TL_VERSION 1001 /* major * 1000 + minor */
 
 #if defined(__GNUC__)
 #define TL_API __attribute__((visibility("default")))
@@ -46,11 +46,18 @@ extern "C" {
 
 typedef enum { TL_F16 = 0, TL_BF16 = 1 } tl_dtype;
 
+/* The epilogue applied to the fp32 accumulator before C's only store (the
+ * TileLang GPU kernel design article, paragraph 5: bias add, then GELU).
+ * GELU is the exact form x Phi(x) = 0.5 x (1 + erf(x / sqrt 2)); GELU_TANH is
+ * the tanh approximation 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) of
+ * the GELU paper (Hendrycks and Gimpel), PyTorch's approximate="tanh".      */
 typedef enum {
-    TL_EPI_NONE = 0,       /* C = A.B                                   */
-    TL_EPI_BIAS_GELU = 1,  /* C = GELU(A.B + bias[col]), exact erf GELU */
-    TL_EPI_BIAS = 2,       /* C = A.B + bias[col]                       */
-    TL_EPI_GELU = 3        /* C = GELU(A.B)                             */
+    TL_EPI_NONE = 0,            /* C = A.B                                   */
+    TL_EPI_BIAS_GELU = 1,       /* C = GELU(A.B + bias[col]), exact erf GELU */
+    TL_EPI_BIAS = 2,            /* C = A.B + bias[col]                       */
+    TL_EPI_GELU = 3,            /* C = GELU(A.B)                             */
+    TL_EPI_BIAS_GELU_TANH = 4,  /* C = GELU_TANH(A.B + bias[col])            */
+    TL_EPI_GELU_TANH = 5        /* C = GELU_TANH(A.B)                        */
 } tl_epilogue;
 
 typedef enum {
@@ -73,9 +80,11 @@ typedef void *tl_stream;
  *   A     device pointer, M x K, row-major (leading dimension K), `dtype`
  *   B     device pointer, K x N, row-major (leading dimension N), `dtype`
  *   bias  device pointer to N values of `dtype`; required when epi is
- *         TL_EPI_BIAS_GELU or TL_EPI_BIAS, ignored (may be NULL) otherwise
- *   C     device pointer, M x N, row-major (leading dimension N), `dtype`;
- *         written, never read.  C must not overlap A, B or bias (not checked).
+ *         TL_EPI_BIAS_GELU, TL_EPI_BIAS or TL_EPI_BIAS_GELU_TANH, ignored (may
+ *         be NULL) otherwise
+ *   C     device pointer, M x N, row-major (leading dimension N), `dtype`
+ *         (float32 with tl_gemm_ex's c_float32 option); written, never read.
+ *         C must not overlap A, B or bias (not checked).
  *   M, N, K   sizes, each in [1, 2^31 - 1]
  *
  * Layout requirements: every pointer must be aligned to 2 bytes.  Nothing
@@ -199,6 +208,10 @@ typedef struct {
     int32_t b_layout;     /* 0: B is K x N row-major (leading dimension N);
                              1: B is given transposed, N x K row-major (leading
                              dimension K) -- the layout of a weight W in A.W^T */
+    int32_t c_float32;    /* 0: C has the inputs' type, rounded once from fp32;
+                             1: C is float32, the epilogue's fp32 result itself
+                             (4-byte aligned; 16-byte aligned rows take vector
+                             stores).  C is then stored without the TMA unit.  */
 } tl_gemm_options;
 
 /* tl_gemm with options (NULL options == tl_gemm).  Same arguments and errors;

@@ -14,7 +14,7 @@ from __future__ import annotations
 
 from ._binding import (  # noqa: F401
     LIB_PATH, Options, Plan, Status, TLError, TL_BF16, TL_EPI_BIAS, TL_EPI_BIAS_GELU, TL_EPI_GELU,
-    TL_EPI_NONE, TL_F16,
+    TL_EPI_NONE, TL_EPI_BIAS_GELU_TANH, TL_EPI_GELU_TANH, TL_EPI_WITH_BIAS, TL_F16,
     SIGNATURES, tl_attention_fwd, tl_check_device, tl_config_name, tl_gemm, tl_gemm_ex, tl_gemm_noalloc,
     tl_gemm_plan, tl_num_configs, tl_softmax_rows, tl_vector_add,
     tl_status_string, tl_version,
@@ -25,7 +25,7 @@ __all__ = [
     "tl_softmax_rows", "tl_vector_add", "Options", "Plan", "Status", "TLError",
     "tl_gemm", "tl_gemm_ex", "tl_gemm_noalloc", "tl_check_device", "tl_gemm_plan", "tl_num_configs", "tl_config_name",
     "tl_status_string", "tl_version", "TL_F16", "TL_BF16", "TL_EPI_NONE", "TL_EPI_BIAS_GELU",
-    "TL_EPI_BIAS", "TL_EPI_GELU",
+    "TL_EPI_BIAS", "TL_EPI_GELU", "TL_EPI_BIAS_GELU_TANH", "TL_EPI_GELU_TANH",
 ]
 
 
@@ -39,11 +39,12 @@ def _dtype_code(t):
 
 
 _EPILOGUES = {None: TL_EPI_NONE, "none": TL_EPI_NONE, "bias_gelu": TL_EPI_BIAS_GELU,
-              "bias+gelu": TL_EPI_BIAS_GELU, "bias": TL_EPI_BIAS, "gelu": TL_EPI_GELU}
+              "bias+gelu": TL_EPI_BIAS_GELU, "bias": TL_EPI_BIAS, "gelu": TL_EPI_GELU,
+              "bias_gelu_tanh": TL_EPI_BIAS_GELU_TANH, "gelu_tanh": TL_EPI_GELU_TANH}
 
 
 def _epi_code(epilogue):
-    if isinstance(epilogue, int) and epilogue in (TL_EPI_NONE, TL_EPI_BIAS_GELU, TL_EPI_BIAS, TL_EPI_GELU):
+    if isinstance(epilogue, int) and TL_EPI_NONE <= epilogue <= TL_EPI_GELU_TANH:
         return epilogue
     if epilogue in _EPILOGUES:
         return _EPILOGUES[epilogue]
@@ -51,16 +52,19 @@ def _epi_code(epilogue):
 
 
 def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0, timeout_ns: int = 0,
-         no_split: bool = False, b_transposed: bool = False):
+         no_split: bool = False, b_transposed: bool = False, out_dtype=None):
     """C = epilogue(A @ B) for row-major CUDA tensors A (M x K) and B (K x N),
     or B given as N x K (``b_transposed=True``: C = epilogue(A @ B.T), the
     layout of a linear layer's weight).
 
-    ``epilogue`` is None / "none", "bias_gelu", "bias" or "gelu" (``bias`` of
-    length N for the first two; default "bias_gelu" when a bias is given).
-    ``out`` (M x N, same dtype) is written if given, else allocated.  Runs
-    asynchronously on ``stream`` (default: torch's current stream).
-    ``config`` = k > 0 forces kernel configuration k - 1.
+    ``epilogue`` is None / "none", "bias_gelu", "bias", "gelu",
+    "bias_gelu_tanh" or "gelu_tanh" (``bias`` of length N for the ones that
+    name it; default "bias_gelu" when a bias is given).  C has A's dtype, or
+    float32 with ``out_dtype=torch.float32`` (or a float32 ``out``): the
+    epilogue's fp32 result without rounding to 16 bits.  ``out`` (M x N) is
+    written if given, else allocated.  Runs asynchronously on ``stream``
+    (default: torch's current stream).  ``config`` = k > 0 forces kernel
+    configuration k - 1.
     """
     import torch
     epi = _epi_code(epilogue if epilogue is not None else ("bias_gelu" if bias is not None else None))
@@ -75,23 +79,28 @@ def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0,
         raise TypeError("A and B must have the same dtype")
     M, K = A.shape
     N = B.shape[0] if b_transposed else B.shape[1]
-    if epi in (TL_EPI_BIAS_GELU, TL_EPI_BIAS):
+    if epi in TL_EPI_WITH_BIAS:
         if bias is None or bias.shape != (N,) or bias.dtype != A.dtype or not bias.is_cuda or not bias.is_contiguous():
             raise ValueError("this epilogue needs a contiguous CUDA bias of length N in the input dtype")
+    if out_dtype is None:
+        out_dtype = out.dtype if out is not None else A.dtype
+    if out_dtype not in (A.dtype, torch.float32):
+        raise TypeError("C is either A's dtype or float32")
+    c_f32 = out_dtype == torch.float32
     if out is None:
-        out = torch.empty((M, N), dtype=A.dtype, device=A.device)
-    elif out.shape != (M, N) or out.dtype != A.dtype or not out.is_contiguous() or not out.is_cuda:
-        raise ValueError("out must be a contiguous CUDA tensor of shape (M, N) and the input dtype")
+        out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    elif out.shape != (M, N) or out.dtype != out_dtype or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous CUDA tensor of shape (M, N) and C's dtype")
     s = stream if stream is not None else torch.cuda.current_stream(A.device)
+    bias_ptr = bias.data_ptr() if bias is not None and epi in TL_EPI_WITH_BIAS else 0
     with torch.cuda.device(A.device):
-        if config or timeout_ns or no_split or b_transposed:
+        if config or timeout_ns or no_split or b_transposed or c_f32:
             opt = Options(config=config, inject_fault=0, timeout_ns=timeout_ns, no_split=int(no_split),
-                          b_layout=int(bool(b_transposed)))
-            st = tl_gemm_ex(A.data_ptr(), B.data_ptr(), bias.data_ptr() if bias is not None and epi in (1, 2) else 0,
-                            out.data_ptr(), M, N, K, dt, epi, s.cuda_stream, opt)
+                          b_layout=int(bool(b_transposed)), c_float32=int(c_f32))
+            st = tl_gemm_ex(A.data_ptr(), B.data_ptr(), bias_ptr, out.data_ptr(), M, N, K, dt, epi,
+                            s.cuda_stream, opt)
         else:
-            st = tl_gemm(A.data_ptr(), B.data_ptr(), bias.data_ptr() if bias is not None and epi in (1, 2) else 0,
-                         out.data_ptr(), M, N, K, dt, epi, s.cuda_stream)
+            st = tl_gemm(A.data_ptr(), B.data_ptr(), bias_ptr, out.data_ptr(), M, N, K, dt, epi, s.cuda_stream)
     if st != 0:
         raise TLError(st, "tl_gemm")
     return out
@@ -168,13 +177,13 @@ def check_device(stream=None) -> int:
 
 
 def plan(M, N, K, dtype=TL_F16, epilogue=None, num_sms=148, config=0, ptrs=(256, 256, 256, 256),
-         b_transposed=False, no_split=False) -> dict:
+         b_transposed=False, no_split=False, c_float32=False) -> dict:
     """The host plan for a call (no GPU needed): config, grid, padding, store path."""
     a, b, bias, c = ptrs
     epi = _epi_code(epilogue)
-    opt = Options(config=config, b_layout=int(b_transposed), no_split=int(no_split)) \
-        if (config or b_transposed or no_split) else None
-    st, p = tl_gemm_plan(a, b, bias if epi in (1, 2) else 0, c, M, N, K, dtype, epi, num_sms, opt)
+    opt = Options(config=config, b_layout=int(b_transposed), no_split=int(no_split), c_float32=int(c_float32)) \
+        if (config or b_transposed or no_split or c_float32) else None
+    st, p = tl_gemm_plan(a, b, bias if epi in TL_EPI_WITH_BIAS else 0, c, M, N, K, dtype, epi, num_sms, opt)
     if st != 0:
         raise TLError(st, "tl_gemm_plan")
     d = p.as_dict()

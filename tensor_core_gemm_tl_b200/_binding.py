@@ -15,6 +15,8 @@ LIB_PATH = os.path.join(_HERE, "libtlgemm.so")
 
 TL_F16, TL_BF16 = 0, 1
 TL_EPI_NONE, TL_EPI_BIAS_GELU, TL_EPI_BIAS, TL_EPI_GELU = 0, 1, 2, 3
+TL_EPI_BIAS_GELU_TANH, TL_EPI_GELU_TANH = 4, 5
+TL_EPI_WITH_BIAS = (TL_EPI_BIAS_GELU, TL_EPI_BIAS, TL_EPI_BIAS_GELU_TANH)
 
 
 class Status(enum.IntEnum):
@@ -36,9 +38,11 @@ class TLError(RuntimeError):
 class Options(ctypes.Structure):
     """tl_gemm_options: config (0 = library's choice, k = configuration k-1),
     inject_fault (test hook), timeout_ns (0 = 10 s), no_split (1 = never split
-    the tiles of a short last round), b_layout (1 = B given as N x K)."""
+    the tiles of a short last round), b_layout (1 = B given as N x K),
+    c_float32 (1 = C is float32)."""
     _fields_ = [("config", ctypes.c_int32), ("inject_fault", ctypes.c_int32),
-                ("timeout_ns", ctypes.c_uint64), ("no_split", ctypes.c_int32), ("b_layout", ctypes.c_int32)]
+                ("timeout_ns", ctypes.c_uint64), ("no_split", ctypes.c_int32), ("b_layout", ctypes.c_int32),
+                ("c_float32", ctypes.c_int32)]
 
 
 class Plan(ctypes.Structure):

@@ -55,11 +55,13 @@ struct GemmParams {
     int32_t group_m;         // output-tile rows per rasterisation group
     const uint16_t *bias;    // N values of the input dtype (epilogue only)
     int32_t epi_bias;        // fused epilogue: add bias[col]
-    int32_t epi_gelu;        // fused epilogue: apply exact GELU
+    int32_t epi_gelu;        // fused epilogue: 0 no GELU, 1 exact (erf) GELU, 2 tanh-form GELU
     int32_t bias_vec16;      // bias is 16-byte aligned: load 8 values per access
     int32_t inject_fault;    // test hook: skip the first stage's copy
-    uint16_t *C;             // direct-store path only
-    int64_t ldc;             // direct-store path only (elements)
+    uint16_t *C;             // 16-bit element-store path only
+    float *C32;              // float32 output only
+    int32_t c32_vec16;       // float32 output: base 16-byte aligned and ldc % 4 == 0
+    int64_t ldc;             // element-store and float32 paths (elements)
     uint64_t timeout_ns;
     // Work items: tiles [0, full_tiles) whole, then each remaining tile split
     // along K into `split` parts, item = full_tiles + r * split + part.  Parts
@@ -280,10 +282,34 @@ __device__ __forceinline__ float gelu_erf(float x)
     return x * (x >= 0.0f ? 1.0f - q : q);
 }
 
+// Tanh form of GELU (the GELU paper's approximation):
+//     g(x) = 0.5 x (1 + tanh(u)),   u = sqrt(2 / pi) (x + 0.044715 x^3),
+// through 0.5 (1 + tanh u) = 1 / (1 + 2^-a) for x >= 0 and 2^-a / (1 + 2^-a)
+// for x < 0, a = |2u| log2(e): the exponential never exceeds 1, so nothing
+// overflows or cancels.  u has the sign of x.  Relative error about
+// 3e-7 + 1.2e-7 a (the rounding of a, carried through 2^-a): below 1e-5
+// for x >= -10, where g is 1e-37.  NaN stays NaN.
+__device__ __forceinline__ float gelu_tanh(float x)
+{
+    constexpr float K0 = 2.3022081983f;       // 2 sqrt(2 / pi) log2(e)
+    constexpr float K1 = 0.044715f * K0;
+    const float a = fabsf(x) * fmaf(K1, x * x, K0);
+    const float e = exp2_approx(-a);
+    const float s = rcp_approx(1.0f + e);
+    return x * (x >= 0.0f ? s : e * s);
+}
+
+// How C leaves the epilogue.
+enum StoreMode : int {
+    STORE_ELEMENTS = 0,  // 16-bit C, element stores (rows not 16-byte aligned)
+    STORE_TMA = 1,       // 16-bit C, swizzled shared-memory staging and TMA stores
+    STORE_F32 = 2,       // float32 C (no rounding to 16 bits), vector or element stores
+};
+
 // EPI = 0: C = A.B.  EPI = 1: the fused epilogue, its steps chosen at run
-// time (bias add and/or GELU).  BT: B is given as N x K row-major (K-major
-// operand) instead of K x N.
-template <class CF, int DT, int EPI, bool TMA_STORE, bool BT>
+// time (bias add and/or a GELU form).  BT: B is given as N x K row-major
+// (K-major operand) instead of K x N.
+template <class CF, int DT, int EPI, int STORE, bool BT>
 __global__ void __launch_bounds__(CF::THREADS, 1)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_c, const GemmParams p)
@@ -330,7 +356,7 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_map(&tmap_a);
         tma_prefetch_map(&tmap_b);
-        if constexpr (TMA_STORE)
+        if constexpr (STORE == STORE_TMA)
             tma_prefetch_map(&tmap_c);
     }
     if (warp == 1) {
@@ -584,7 +610,7 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                     }
                 }
 
-                if constexpr (TMA_STORE) {
+                if constexpr (STORE == STORE_TMA) {
                     // this warp's staging box: its previous store must have read it
                     if (lane == 0)
                         bulk_wait_group_read<0>();
@@ -619,18 +645,41 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                                     v[j] += to_float<DT>(__ldg(p.bias + colh + j));
                         }
                       }
-                      if (p.epi_gelu) {
+                      if (p.epi_gelu == 1) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
                             v[j] = gelu_erf(v[j]);
+                      } else if (p.epi_gelu == 2) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            v[j] = gelu_tanh(v[j]);
                       }
+                    }
+                    if constexpr (STORE == STORE_F32) {
+                        // row `lane`: 32 consecutive floats (128 bytes)
+                        const int m = row0 + lane;
+                        if (m < p.M) {
+                            float *crow = p.C32 + static_cast<int64_t>(m) * p.ldc + colh;
+                            if (p.c32_vec16 && colh + 32 <= p.N) {
+#pragma unroll
+                                for (int i = 0; i < 8; ++i)
+                                    reinterpret_cast<float4 *>(crow)[i] =
+                                        make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j)
+                                    if (colh + j < p.N)
+                                        crow[j] = v[j];
+                            }
+                        }
+                        continue;
                     }
                     uint32_t packed[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         packed[j] = pack2<DT>(v[2 * j], v[2 * j + 1]);
 
-                    if constexpr (TMA_STORE) {
+                    if constexpr (STORE == STORE_TMA) {
                         // row `lane` of the 32 x 64 box; 16-byte chunk i lands at i ^ (lane & 7)
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
@@ -653,7 +702,7 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                         }
                     }
                 }
-                if constexpr (TMA_STORE) {
+                if constexpr (STORE == STORE_TMA) {
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
@@ -667,7 +716,7 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                 acc_phase ^= 1u;
             }
         }
-        if constexpr (TMA_STORE) {
+        if constexpr (STORE == STORE_TMA) {
             if (lane == 0)
                 bulk_wait_group<0>();
             __syncwarp();

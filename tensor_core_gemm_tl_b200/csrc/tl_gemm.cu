@@ -33,8 +33,23 @@ struct ConfigEntry {
     int ctas;                // 1, or 2 for a CTA pair (cluster of two, cta_group::2 MMA)
     int threads;             // threads per CTA
     int smem_bytes;
-    KernelFn fn[2][2][2][2];  // [dtype][fused epilogue][tma_store][B given transposed]
+    KernelFn fn[2][2][3][2];  // [dtype][fused epilogue][store mode][B given transposed]
 };
+
+template <class CF, int DT, int EPI, int STORE>
+void fill_entry(ConfigEntry &e)
+{
+    e.fn[DT][EPI][STORE][0] = gemm_sm100_kernel<CF, DT, EPI, STORE, false>;
+    e.fn[DT][EPI][STORE][1] = gemm_sm100_kernel<CF, DT, EPI, STORE, true>;
+}
+
+template <class CF, int DT, int EPI>
+void fill_entry_stores(ConfigEntry &e)
+{
+    fill_entry<CF, DT, EPI, STORE_ELEMENTS>(e);
+    fill_entry<CF, DT, EPI, STORE_TMA>(e);
+    fill_entry<CF, DT, EPI, STORE_F32>(e);
+}
 
 template <class CF>
 ConfigEntry make_entry(const char *name)
@@ -49,22 +64,10 @@ ConfigEntry make_entry(const char *name)
     e.bk = CF::BK;
     e.stages = CF::STAGES;
     e.smem_bytes = CF::SMEM_BYTES;
-    e.fn[0][0][0][0] = gemm_sm100_kernel<CF, 0, 0, false, false>;
-    e.fn[0][0][1][0] = gemm_sm100_kernel<CF, 0, 0, true, false>;
-    e.fn[0][1][0][0] = gemm_sm100_kernel<CF, 0, 1, false, false>;
-    e.fn[0][1][1][0] = gemm_sm100_kernel<CF, 0, 1, true, false>;
-    e.fn[1][0][0][0] = gemm_sm100_kernel<CF, 1, 0, false, false>;
-    e.fn[1][0][1][0] = gemm_sm100_kernel<CF, 1, 0, true, false>;
-    e.fn[1][1][0][0] = gemm_sm100_kernel<CF, 1, 1, false, false>;
-    e.fn[1][1][1][0] = gemm_sm100_kernel<CF, 1, 1, true, false>;
-    e.fn[0][0][0][1] = gemm_sm100_kernel<CF, 0, 0, false, true>;
-    e.fn[0][0][1][1] = gemm_sm100_kernel<CF, 0, 0, true, true>;
-    e.fn[0][1][0][1] = gemm_sm100_kernel<CF, 0, 1, false, true>;
-    e.fn[0][1][1][1] = gemm_sm100_kernel<CF, 0, 1, true, true>;
-    e.fn[1][0][0][1] = gemm_sm100_kernel<CF, 1, 0, false, true>;
-    e.fn[1][0][1][1] = gemm_sm100_kernel<CF, 1, 0, true, true>;
-    e.fn[1][1][0][1] = gemm_sm100_kernel<CF, 1, 1, false, true>;
-    e.fn[1][1][1][1] = gemm_sm100_kernel<CF, 1, 1, true, true>;
+    fill_entry_stores<CF, 0, 0>(e);
+    fill_entry_stores<CF, 0, 1>(e);
+    fill_entry_stores<CF, 1, 0>(e);
+    fill_entry_stores<CF, 1, 1>(e);
     return e;
 }
 
@@ -173,6 +176,29 @@ struct Plan {
     int32_t num_kb;
 };
 
+bool epi_has_bias(int epi)
+{
+    return epi == TL_EPI_BIAS_GELU || epi == TL_EPI_BIAS || epi == TL_EPI_BIAS_GELU_TANH;
+}
+
+// GELU form of an epilogue: 0 none, 1 exact (erf), 2 tanh
+int epi_gelu_form(int epi)
+{
+    if (epi == TL_EPI_BIAS_GELU || epi == TL_EPI_GELU)
+        return 1;
+    if (epi == TL_EPI_BIAS_GELU_TANH || epi == TL_EPI_GELU_TANH)
+        return 2;
+    return 0;
+}
+
+// Store mode of the kernel for this call (see StoreMode)
+int store_mode(const tl_plan &q, const tl_gemm_options *opt)
+{
+    if (opt && opt->c_float32)
+        return STORE_F32;
+    return q.direct_store ? STORE_ELEMENTS : STORE_TMA;
+}
+
 tl_status validate(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N,
                    int64_t K, int dtype, int epi, const tl_gemm_options *opt)
 {
@@ -182,23 +208,25 @@ tl_status validate(const void *A, const void *B, const void *bias, void *C, int6
         return TL_ERR_INVALID_ARG;
     if (dtype != TL_F16 && dtype != TL_BF16)
         return TL_ERR_INVALID_ARG;
-    if (epi < TL_EPI_NONE || epi > TL_EPI_GELU)
+    if (epi < TL_EPI_NONE || epi > TL_EPI_GELU_TANH)
         return TL_ERR_INVALID_ARG;
-    const bool needs_bias = epi == TL_EPI_BIAS_GELU || epi == TL_EPI_BIAS;
+    const bool needs_bias = epi_has_bias(epi);
     if (needs_bias && !bias)
         return TL_ERR_INVALID_ARG;
     if (opt && (opt->config < 0 || opt->config > num_configs()))
         return TL_ERR_INVALID_ARG;
     if (opt && (opt->inject_fault != 0 && opt->inject_fault != 1))
         return TL_ERR_INVALID_ARG;
-    if (opt && ((opt->no_split != 0 && opt->no_split != 1) || (opt->b_layout != 0 && opt->b_layout != 1)))
+    if (opt && ((opt->no_split != 0 && opt->no_split != 1) || (opt->b_layout != 0 && opt->b_layout != 1) ||
+                (opt->c_float32 != 0 && opt->c_float32 != 1)))
         return TL_ERR_INVALID_ARG;
     if (opt && opt->inject_fault && opt->config > 0 && kConfigs[opt->config - 1].ctas != 1)
         return TL_ERR_UNSUPPORTED;  // the fault hook exists for single-CTA configurations only
     const int64_t lim = 0x7FFFFFFFll;
     if (M > lim || N > lim || K > lim)
         return TL_ERR_UNSUPPORTED;
-    if (!aligned(A, 2) || !aligned(B, 2) || !aligned(C, 2) || (needs_bias && !aligned(bias, 2)))
+    const bool c_f32 = opt && opt->c_float32;
+    if (!aligned(A, 2) || !aligned(B, 2) || !aligned(C, c_f32 ? 4 : 2) || (needs_bias && !aligned(bias, 2)))
         return TL_ERR_MISALIGNED;
     return TL_OK;
 }
@@ -275,7 +303,7 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
     const int64_t b_rows = bt ? N : K;
     q.pad_a = !(aligned(A, 16) && K % 8 == 0);
     q.pad_b = !(aligned(B, 16) && b_cols % 8 == 0);
-    q.direct_store = !(aligned(C, 16) && N % 8 == 0);
+    q.direct_store = (opt && opt->c_float32) || !(aligned(C, 16) && N % 8 == 0);
     p.lda = q.pad_a ? ceil_div(K, 8) * 8 : K;
     p.ldb = q.pad_b ? ceil_div(b_cols, 8) * 8 : b_cols;
     int64_t ws = 0;
@@ -457,9 +485,10 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
                       const tl_gemm_options *opt, void *workspace)
 {
     const ConfigEntry &c = kConfigs[p.pub.config];
-    const bool tma_store = !p.pub.direct_store;
+    const int store = store_mode(p.pub, opt);
+    const bool tma_store = store == STORE_TMA;
     const int bt = (opt && opt->b_layout == 1) ? 1 : 0;
-    KernelFn fn = c.fn[dtype][epi != 0][tma_store ? 1 : 0][bt];
+    KernelFn fn = c.fn[dtype][epi != 0][store][bt];
     tl_status st = raise_smem_limit(d, fn, c.smem_bytes);
     if (st != TL_OK)
         return st;
@@ -485,12 +514,14 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
     gp.group_m = 8;
     gp.bias = static_cast<const uint16_t *>(bias);
     gp.bias_vec16 = bias && aligned(bias, 16);
-    gp.epi_bias = epi == TL_EPI_BIAS_GELU || epi == TL_EPI_BIAS;
-    gp.epi_gelu = epi == TL_EPI_BIAS_GELU || epi == TL_EPI_GELU;
+    gp.epi_bias = epi_has_bias(epi);
+    gp.epi_gelu = epi_gelu_form(epi);
     if (!gp.epi_bias)
         gp.bias = nullptr;
     gp.inject_fault = opt ? opt->inject_fault : 0;
     gp.C = static_cast<uint16_t *>(C);
+    gp.C32 = store == STORE_F32 ? static_cast<float *>(C) : nullptr;
+    gp.c32_vec16 = store == STORE_F32 && aligned(C, 16) && N % 4 == 0;
     gp.ldc = N;
     gp.timeout_ns = (opt && opt->timeout_ns) ? opt->timeout_ns : kDefaultTimeoutNs;
     gp.split = p.pub.split;
@@ -542,7 +573,7 @@ tl_status device_plan(DeviceState *d, const void *A, const void *B, const void *
     const ConfigEntry &c = kConfigs[p->pub.config];
     if (c.ctas != 2)
         return TL_OK;
-    KernelFn fn = c.fn[dtype][epi != 0][p->pub.direct_store ? 0 : 1][(opt && opt->b_layout == 1) ? 1 : 0];
+    KernelFn fn = c.fn[dtype][epi != 0][store_mode(p->pub, opt)][(opt && opt->b_layout == 1) ? 1 : 0];
     if ((st = raise_smem_limit(d, fn, c.smem_bytes)) != TL_OK)
         return st;
     cudaLaunchConfig_t cfg{};

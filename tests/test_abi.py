@@ -32,7 +32,8 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_strings():
-    assert tg.tl_version() == 1000
+    declared = int(re.search(r"#define TL_VERSION (\d+)", open(HEADER).read()).group(1))
+    assert tg.tl_version() == declared
     for s in tg.Status:
         assert tg.tl_status_string(int(s)) == "TL_" + ("OK" if s.name == "OK" else "ERR_" + s.name)
     assert tg.tl_status_string(99) == "TL_ERR_UNKNOWN"
@@ -51,10 +52,12 @@ def test_version_and_strings():
     (dict(N=-1), tg.Status.INVALID_ARG),
     (dict(K=0), tg.Status.INVALID_ARG),
     (dict(dtype=2), tg.Status.INVALID_ARG),
-    (dict(epi=7), tg.Status.INVALID_ARG),
+    (dict(epi=6), tg.Status.INVALID_ARG),
     (dict(epi=-1), tg.Status.INVALID_ARG),
     (dict(epi=1, bias=0), tg.Status.INVALID_ARG),
     (dict(epi=2, bias=0), tg.Status.INVALID_ARG),
+    (dict(epi=4, bias=0), tg.Status.INVALID_ARG),
+    (dict(epi=4, bias=P + 1), tg.Status.MISALIGNED),
     (dict(epi=2, bias=P + 1), tg.Status.MISALIGNED),
     (dict(M=1 << 31), tg.Status.UNSUPPORTED),
     (dict(K=1 << 40), tg.Status.UNSUPPORTED),
@@ -200,6 +203,23 @@ def test_gelu_only_needs_no_bias_and_b_layout_is_validated():
     st, _ = tg.tl_gemm_plan(P, P, 0, P, 256, 256, 256, 0, tg.TL_EPI_GELU, 148)
     assert st == 0
     assert tg.tl_gemm_ex(P, P, 0, P, 8, 8, 8, 0, 0, 0, tg.Options(b_layout=2)) == tg.Status.INVALID_ARG
+
+
+def test_tanh_epilogues_and_float32_output_options():
+    # tanh GELU alone needs no bias; with bias it does
+    st, _ = tg.tl_gemm_plan(P, P, 0, P, 256, 256, 256, 0, tg.TL_EPI_GELU_TANH, 148)
+    assert st == 0
+    st, _ = tg.tl_gemm_plan(P, P, P, P, 256, 256, 256, 1, tg.TL_EPI_BIAS_GELU_TANH, 148)
+    assert st == 0
+    # float32 C: 4-byte alignment, never the TMA store, same tiles and padding
+    f32 = tg.Options(c_float32=1)
+    st, p = tg.tl_gemm_plan(P, P, 0, P, 4096, 4096, 4096, 0, 0, 148, f32)
+    assert st == 0 and p.direct_store == 1 and p.pad_a == 0 and p.pad_b == 0
+    st, p16 = tg.tl_gemm_plan(P, P, 0, P, 4096, 4096, 4096, 0, 0, 148)
+    assert st == 0 and p16.direct_store == 0 and p16.config == p.config and p16.grid == p.grid
+    assert tg.tl_gemm_ex(P, P, 0, P + 2, 8, 8, 8, 0, 0, 0, f32) == tg.Status.MISALIGNED
+    assert tg.tl_gemm_ex(P, P, 0, P, 8, 8, 8, 0, 0, 0, tg.Options(c_float32=2)) == tg.Status.INVALID_ARG
+    assert tg.plan(512, 1000, 2048, tg.TL_BF16, "gelu_tanh", c_float32=True)["direct_store"] == 1
 
 
 def test_plan_transposed_b_pads_on_k():

@@ -1,6 +1,7 @@
-"""The epilogue's GELU: the kernel's float32 formula and constants checked on
-the CPU against mpmath, and on the GPU the fused epilogue over every finite
-fp16 and bf16 input value against the oracle."""
+"""The epilogue's GELU (exact erf form and tanh form): the kernel's float32
+formulas and constants checked on the CPU against mpmath, and on the GPU the
+fused epilogue over every finite fp16 and bf16 input value against the
+oracle, with 16-bit and with float32 output."""
 import os
 import re
 import sys
@@ -58,6 +59,101 @@ def test_kernel_gelu_formula_accuracy():
     assert rel[small & (np.abs(ref) > 1e-37)].max() < 3e-6
     assert rel[np.abs(ref) > 1e-37].max() < 2e-5
     assert np.isnan(gelu_like_kernel(np.float32([np.nan]))[0])
+
+
+def kernel_tanh_constant():
+    src = open(KERNEL).read()
+    body = src[src.index("__device__ __forceinline__ float gelu_tanh"):]
+    body = body[:body.index("\n}\n")]
+    k0 = np.float32(re.search(r"constexpr float K0 = ([0-9.eE+-]+)f;", body).group(1))
+    k1c = np.float32(re.search(r"constexpr float K1 = ([0-9.eE+-]+)f \* K0;", body).group(1))
+    return k0, np.float32(k1c * k0)
+
+
+def gelu_tanh_like_kernel(x):
+    """The kernel's float32 tanh-GELU sequence in numpy float32 (2^x and the
+    reciprocal correctly rounded here; the device's add about 2^-22 each)."""
+    K0, K1 = kernel_tanh_constant()
+    f = np.float32
+    x = np.asarray(x, dtype=np.float32)
+    with np.errstate(over="ignore", under="ignore"):
+        # fmaf(K1, x * x, K0): one rounding of the exact K1 x^2 + K0
+        a = np.abs(x) * (np.float64(K1) * (x * x).astype(np.float64) + np.float64(K0)).astype(np.float32)
+        e = np.exp2(-a.astype(np.float64)).astype(np.float32)
+        s = (1.0 / (f(1) + e).astype(np.float64)).astype(np.float32)
+        return x * np.where(x >= 0, s, e * s)
+
+
+def tanh_rel_bound(x):
+    """Relative error allowed for the float32 tanh GELU at x: the rounding of
+    a = |2u| log2(e) (about 2 ulps) carried through 2^-a, plus the device's
+    approximate 2^x and reciprocal."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x) * (2.3022082 + 0.10294 * x * x)
+    return 1e-6 + 2.5e-7 * a
+
+
+def _mp_gelu_tanh(x):
+    import mpmath as mp
+    # for x < 0, 1 + tanh(u) loses about 0.87 |u| digits: carry that many more
+    u = abs(0.7978845608028654 * (x + 0.044715 * x ** 3)) if x < 0 else 0.0
+    with mp.workdps(30 + int(0.87 * u)):
+        xm = mp.mpf(x)
+        return float(xm / 2 * (1 + mp.tanh(mp.sqrt(2 / mp.pi) * (xm + mp.mpf("0.044715") * xm ** 3))))
+
+
+def test_kernel_gelu_tanh_formula_accuracy():
+    import mpmath as mp
+    mp.mp.dps = 30
+    xs = np.concatenate([np.linspace(-12, 12, 4801), np.geomspace(1e-20, 1, 200),
+                         -np.geomspace(1e-20, 1, 200), [0.0, 25.0, -25.0, 1e30]]).astype(np.float32)
+    got = gelu_tanh_like_kernel(xs).astype(np.float64)
+    ref = np.array([_mp_gelu_tanh(float(x)) for x in xs])
+    keep = np.abs(ref) > 1e-37
+    rel = np.abs(got - ref)[keep] / np.abs(ref[keep])
+    assert np.all(rel < tanh_rel_bound(xs[keep]) - 5e-7), rel.max()  # room for the device's MUFU ops
+    assert np.isnan(gelu_tanh_like_kernel(np.float32([np.nan]))[0])
+
+
+def _finite_patterns(dt):
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    expo = (allbits >> 10) & 0x1F if dt == wl.F16 else (allbits >> 7) & 0xFF
+    return allbits[expo != (0x1F if dt == wl.F16 else 0xFF)]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dt", [wl.F16, wl.BF16])
+@pytest.mark.parametrize("form", ["erf", "tanh"])
+@pytest.mark.parametrize("out_f32", [False, True])
+def test_fused_gelu_forms_every_finite_input(dt, form, out_f32):
+    """Both GELU forms, 16-bit and float32 output: C = GELU(0 + bias) for bias
+    = every finite 16-bit value, against the oracle's fp64 GELU."""
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import oracle
+    from gpu_util import F32, run_library, ulp
+    finite = _finite_patterns(dt)
+    N, M, K = finite.size, 256, 16
+    A = np.zeros((M, K), np.uint16)
+    B = np.zeros((K, N), np.uint16)
+    epi = wl.EPI_BIAS_GELU if form == "erf" else wl.EPI_BIAS_GELU_TANH
+    C = run_library(A, B, finite, dt, epi, out_f32=out_f32)
+    assert np.array_equal(C, np.repeat(C[:1], M, axis=0)), "rows differ"
+    got = C[0].astype(np.float64) if out_f32 else wl.bits_to_float32(C[0], dt).astype(np.float64)
+    x = oracle.decode(finite, dt)
+    ref = oracle.gelu(x) if form == "erf" else oracle.gelu_tanh(x)
+    assert np.all(np.isfinite(got))
+    if form == "erf":
+        rel = np.where(np.abs(x) <= 9, 4e-6, 2e-5)
+    else:
+        rel = tanh_rel_bound(x)
+    # a result below the smallest normal float32 (2^-126) has fewer significant
+    # bits, and so do the kernel's intermediates on the way to it: the relative
+    # allowance applies to max(|ref|, 2^-126) there
+    bound = 0.5 * ulp(np.abs(ref), F32 if out_f32 else dt) + rel * np.maximum(np.abs(ref), 2.0 ** -126) + 1e-45
+    bad = np.abs(got - ref) > bound
+    assert not bad.any(), (x[bad][:5], got[bad][:5], ref[bad][:5])
 
 
 @pytest.mark.gpu

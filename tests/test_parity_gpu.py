@@ -12,7 +12,7 @@ sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 
 import oracle  # noqa: E402
 import workloads as wl  # noqa: E402
-from gpu_util import accumulation_bound, compare, run_library, to_device  # noqa: E402
+from gpu_util import accumulation_bound, compare, compare_f32, run_library, to_device  # noqa: E402
 
 torch = pytest.importorskip("torch")
 pytestmark = [pytest.mark.gpu,
@@ -202,6 +202,55 @@ def test_bias_only_and_gelu_only_vs_oracle(epi, dt, M, N, K):
     ref = oracle.gemm(A, B, bias, dt, epi)
     C = run_library(A, B, bias, dt, epi)
     compare(C, ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
+
+
+TANH_F32_SHAPES = [(256, 512, 256), (300, 520, 200), (129, 1001, 2050), (4096, 1024, 512)]
+
+
+@pytest.mark.parametrize("epi", [wl.EPI_BIAS_GELU_TANH, wl.EPI_GELU_TANH])
+@pytest.mark.parametrize("dt", [wl.F16, wl.BF16])
+@pytest.mark.parametrize("M,N,K", TANH_F32_SHAPES)
+def test_tanh_gelu_epilogues_vs_oracle(epi, dt, M, N, K):
+    A, B, bias = inputs(M, N, K, dt, epi, seed=K + epi)
+    ref = oracle.gemm(A, B, bias, dt, epi)
+    C = run_library(A, B, bias, dt, epi)
+    compare(C, ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
+
+
+@pytest.mark.parametrize("epi", [wl.EPI_NONE, wl.EPI_BIAS_GELU, wl.EPI_BIAS, wl.EPI_GELU, wl.EPI_BIAS_GELU_TANH])
+@pytest.mark.parametrize("dt", [wl.F16, wl.BF16])
+@pytest.mark.parametrize("M,N,K", TANH_F32_SHAPES)
+def test_float32_output_vs_oracle(epi, dt, M, N, K):
+    """C in float32: the epilogue's fp32 value, never rounded to 16 bits (N = 1001
+    takes the element-store tail, the others the vector stores)."""
+    A, B, bias = inputs(M, N, K, dt, epi, seed=M + epi)
+    ref = oracle.gemm(A, B, bias, dt, epi)
+    C = run_library(A, B, bias, dt, epi, out_f32=True)
+    compare_f32(C, ref, accumulation_bound(A, B, bias, dt, epi, ref, out_f32=True))
+
+
+@pytest.mark.parametrize("config", ALL_CONFIGS)
+def test_float32_output_every_config_and_unaligned(config):
+    M, N, K = 520, 700, 264
+    dt, epi = wl.BF16, wl.EPI_BIAS_GELU
+    A, B, bias = inputs(M, N, K, dt, epi, seed=config)
+    ref = oracle.gemm(A, B, bias, dt, epi)
+    bound = accumulation_bound(A, B, bias, dt, epi, ref, out_f32=True)
+    compare_f32(run_library(A, B, bias, dt, epi, config=config, out_f32=True), ref, bound)
+    # C's base 4-byte but not 16-byte aligned: element stores throughout
+    compare_f32(run_library(A, B, bias, dt, epi, config=config, out_f32=True, offsets=(0, 0, 0, 1)), ref, bound)
+
+
+def test_float32_output_is_the_unrounded_16bit_result():
+    """Rounding the float32 C once to the input type gives the 16-bit C bit for
+    bit (the same accumulator, the same epilogue, one rounding moved out)."""
+    M, N, K = 384, 512, 320
+    for dt in (wl.F16, wl.BF16):
+        for epi in (wl.EPI_NONE, wl.EPI_BIAS_GELU, wl.EPI_GELU_TANH):
+            A, B, bias = inputs(M, N, K, dt, epi, seed=3)
+            C16 = run_library(A, B, bias, dt, epi)
+            C32 = run_library(A, B, bias, dt, epi, out_f32=True)
+            assert np.array_equal(wl.round_to_bits(C32, dt), C16), (dt, epi)
 
 
 # ------------------------------------------------------------------ the named workloads
