@@ -120,3 +120,45 @@ def test_attention_deterministic():
     a, la = run_attention(Q, K, V, dt, True, 0.1)
     b, lb = run_attention(Q, K, V, dt, True, 0.1)
     assert np.array_equal(a, b) and np.array_equal(la, lb)
+
+
+def weighted_abs_rows(Q, K, V, dt, causal, scale, bh, qi):
+    """sum_j w_j |v_j| for the listed (batch*head, query) rows only, one row
+    at a time (a head's K and V are read per row, not gathered for all)."""
+    B, H, Sq, D = Q.shape
+    Sk = K.shape[2]
+    Qr, Kr, Vr = Q.reshape(B * H, Sq, D), K.reshape(B * H, Sk, D), V.reshape(B * H, Sk, D)
+    out = np.empty((bh.size, D))
+    for n, (h, i) in enumerate(zip(bh, qi)):
+        q = wl.bits_to_float32(Qr[h, i], dt).astype(np.float64)
+        k = wl.bits_to_float32(Kr[h], dt).astype(np.float64)
+        v = np.abs(wl.bits_to_float32(Vr[h], dt).astype(np.float64))
+        s = k @ q * scale
+        if causal:
+            s[i + 1:] = -np.inf
+        w = np.exp(s - s.max())
+        out[n] = (w / w.sum()) @ v
+    return out
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_benchmark_size_sampled_rows(causal):
+    """The timed shape, B 4 H 16 Sq = Sk = 4096 D 128 bf16, computed whole on
+    the GPU; 256 sampled rows (every query tile's first and last row included
+    for a few heads) checked against the oracle's rows, same bar as above."""
+    dt, B, H, S, D = wl.BF16, 4, 16, 4096, 128
+    Q, K, V = make_qkv(B, H, S, S, D, dt, seed=11)
+    scale = 1.0 / math.sqrt(D)
+    O, lse = run_attention(Q, K, V, dt, causal, scale)
+    rng = np.random.default_rng(12)
+    bh = np.concatenate([np.repeat([0, 37, 63], 2 * (S // 128)), rng.integers(0, B * H, 64)])
+    edge = np.tile(np.concatenate([np.arange(0, S, 128), np.arange(127, S, 128)]), 3)
+    qi = np.concatenate([edge, rng.integers(0, S, 64)])
+    ref, ref_lse = oracle.attention(Q, K, V, dt, causal, scale, rows=(bh, qi))
+    got = wl.bits_to_float32(O.reshape(B * H, S, D)[bh, qi], dt).astype(np.float64)
+    u = 2.0 ** -9
+    bound = 2 * u * (weighted_abs_rows(Q, K, V, dt, causal, scale, bh, qi) + np.abs(ref)) \
+        + 0.5 * ulp(np.abs(ref), dt) + 1e-7
+    assert np.all(np.abs(got - ref) <= bound), (np.abs(got - ref) - bound).max()
+    l_got = lse.reshape(B * H, S)[bh, qi]
+    assert np.all(np.abs(l_got - ref_lse) <= 1e-4 * (1 + np.abs(ref_lse)))

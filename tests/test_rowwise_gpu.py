@@ -45,6 +45,20 @@ def test_softmax_vs_oracle(rows, cols, dt):
     assert np.all(np.abs(Y - ref) <= bound), np.max(np.abs(Y - ref) - bound)
 
 
+@pytest.mark.parametrize("rows,cols", [(16384, 8192), (4096, 50257), (262144, 128)])
+def test_softmax_benchmark_sizes_sampled_rows(rows, cols):
+    """The timed shapes, computed whole on the GPU; sampled rows (first, last
+    and random) checked against the oracle."""
+    dt = wl.BF16
+    rng = np.random.default_rng(cols)
+    X = wl.round_to_bits(rng.normal(size=(rows, cols)).astype(np.float32), dt)
+    Y = run_softmax(X, dt)
+    pick = np.unique(np.concatenate([[0, rows - 1], rng.integers(0, rows, 200)]))
+    ref = oracle.softmax_rows(np.ascontiguousarray(X[pick]), dt)
+    got = wl.bits_to_float32(Y[pick], dt).astype(np.float64)
+    assert np.all(np.abs(got - ref) <= 0.5 * ulp(ref, dt) + 1e-5 * ref + 1e-40)
+
+
 @pytest.mark.parametrize("offset", [1, 3])
 def test_softmax_unaligned(offset):
     dt = wl.BF16
