@@ -7,7 +7,8 @@
 //                 3, and the blog retelling's Step 3)
 //
 // Both read each input once and write each output once; their roofline is
-// HBM bandwidth.  16-byte vector accesses when the rows / arrays allow them,
+// HBM bandwidth.  The softmax weights use the flush-to-zero 2^x (one MUFU
+// op): a probability below 2^-126 (1.2e-38) comes out as 0.  16-byte vector accesses when the rows / arrays allow them,
 // element accesses otherwise; grids are sized in multiples of the SM count.
 #pragma once
 
@@ -16,6 +17,7 @@
 #include <cstdint>
 
 #include "sm100.cuh"
+#include "gemm_kernel.cuh"  // the library's device error word (g_device_error)
 
 namespace tl {
 
@@ -39,80 +41,126 @@ __device__ __forceinline__ uint16_t float_to_half(float f)
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// ------------------------------------------------------------------ row softmax, one warp per row
-// Rows of up to 32 * PER_LANE values live in registers: one read, one write.
-template <int DT, int PER_LANE, bool VEC>
-__global__ void __launch_bounds__(256) softmax_rows_warp_kernel(const uint16_t *__restrict__ X,
+// 8 16-bit values of one 16-byte word, widened to float
+template <int DT>
+__device__ __forceinline__ void unpack8(const uint4 &w, float *v)
+{
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        v[2 * h] = half_to_float<DT>(static_cast<uint16_t>(ww[h] & 0xFFFFu));
+        v[2 * h + 1] = half_to_float<DT>(static_cast<uint16_t>(ww[h] >> 16));
+    }
+}
+
+// 8 floats, rounded to 16 bits, as one 16-byte word
+template <int DT>
+__device__ __forceinline__ uint4 pack8(const float *v, float scale)
+{
+    uint32_t o[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+        o[h] = pack2<DT>(v[2 * h] * scale, v[2 * h + 1] * scale);  // one paired conversion
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// ------------------------------------------------------------------ row softmax, LPR lanes per row
+// Rows of up to LPR * PER_LANE values live in registers: one read, one write.
+// A warp serves 32 / LPR rows at a time (short rows do not leave lanes idle)
+// and loads its next rows before reducing the current ones, so a load is in
+// flight while the previous rows are reduced and written.
+template <int DT, int PER_LANE, bool VEC, int LPR>
+__global__ void __launch_bounds__(256, VEC ? 4 : 2) softmax_rows_warp_kernel(const uint16_t *__restrict__ X,
                                                                 uint16_t *__restrict__ Y, int64_t rows, int cols)
 {
+    static_assert(LPR == 8 || LPR == 16 || LPR == 32, "lanes per row");
+    constexpr int RPW = 32 / LPR;                   // rows per warp
+    constexpr int NW = VEC ? PER_LANE / 8 : 1;      // 16-byte words a lane holds
     const int lane = threadIdx.x & 31;
+    const int sub = lane % LPR;                     // lane within its row
     const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-    for (int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
-         row += warps_total) {
+    const int64_t warp0 = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t group_stride = warps_total * RPW;
+
+    uint4 w[NW];                                    // raw words (VEC)
+    uint16_t e[VEC ? 1 : PER_LANE];                 // raw values (scalar path)
+    auto load = [&](int64_t row) {
+        if (row >= rows)
+            return;
         const uint16_t *x = X + row * cols;
-        uint16_t *y = Y + row * cols;
-        float v[PER_LANE];
-        float m = -INFINITY;
         if constexpr (VEC) {
-            // lane reads 8 consecutive values per step; a step covers 256 columns
 #pragma unroll
-            for (int s = 0; s < PER_LANE / 8; ++s) {
-                const int c = s * 256 + lane * 8;
-                if (c < cols) {
-                    const uint4 w = __ldg(reinterpret_cast<const uint4 *>(x + c));
-                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        v[8 * s + 2 * h] = half_to_float<DT>(static_cast<uint16_t>(ww[h] & 0xFFFFu));
-                        v[8 * s + 2 * h + 1] = half_to_float<DT>(static_cast<uint16_t>(ww[h] >> 16));
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        v[8 * s + e] = -INFINITY;
-                }
+            for (int s = 0; s < NW; ++s) {
+                const int c = s * LPR * 8 + sub * 8;
+                if (c < cols)
+                    w[s] = __ldg(reinterpret_cast<const uint4 *>(x + c));
             }
         } else {
 #pragma unroll
             for (int s = 0; s < PER_LANE; ++s) {
-                const int c = s * 32 + lane;
-                v[s] = c < cols ? half_to_float<DT>(x[c]) : -INFINITY;
+                const int c = s * LPR + sub;
+                if (c < cols)
+                    e[s] = __ldg(x + c);
             }
         }
+    };
+    int64_t row = warp0 * RPW + lane / LPR;
+    load(row);
+    // the loop runs while any row of the warp is live (shuffles need every lane)
+    for (int64_t base = warp0 * RPW; base < rows; base += group_stride, row += group_stride) {
+        const bool live = row < rows;
+        float v[PER_LANE];
+        if constexpr (VEC) {
 #pragma unroll
-        for (int s = 0; s < PER_LANE; ++s)
-            m = fmaxf(m, v[s]);
+            for (int s = 0; s < NW; ++s) {
+                const int c = s * LPR * 8 + sub * 8;
+                if (live && c < cols) {
+                    unpack8<DT>(w[s], v + 8 * s);
+                } else {
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
+                    for (int k = 0; k < 8; ++k)
+                        v[8 * s + k] = -INFINITY;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int s = 0; s < PER_LANE; ++s)
+                v[s] = (live && s * LPR + sub < cols) ? half_to_float<DT>(e[s]) : -INFINITY;
+        }
+        load(row + group_stride);  // next rows: in flight during this row's work
+        float m = -INFINITY;
+        static_assert(PER_LANE % 2 == 0, "pairs for the three-way max");
+#pragma unroll
+        for (int s = 0; s < PER_LANE; s += 2)
+            m = fmax3(m, v[s], v[s + 1]);
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1)
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        const float mb = m * kLog2e;
+        const float mb = live ? m * kLog2e : 0.0f;
         float sum = 0.0f;
 #pragma unroll
         for (int s = 0; s < PER_LANE; ++s) {
-            v[s] = exp2_approx(fmaf(v[s], kLog2e, -mb));  // -inf (padding) -> 0
+            v[s] = exp2_approx_ftz(fmaf(v[s], kLog2e, -mb));  // -inf (padding) -> 0
             sum += v[s];
         }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
+        for (int off = LPR / 2; off > 0; off >>= 1)
             sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (!live)
+            continue;
         const float inv = 1.0f / sum;
+        uint16_t *y = Y + row * cols;
         if constexpr (VEC) {
 #pragma unroll
-            for (int s = 0; s < PER_LANE / 8; ++s) {
-                const int c = s * 256 + lane * 8;
-                if (c < cols) {
-                    uint4 w;
-                    w.x = float_to_half<DT>(v[8 * s] * inv) | (static_cast<uint32_t>(float_to_half<DT>(v[8 * s + 1] * inv)) << 16);
-                    w.y = float_to_half<DT>(v[8 * s + 2] * inv) | (static_cast<uint32_t>(float_to_half<DT>(v[8 * s + 3] * inv)) << 16);
-                    w.z = float_to_half<DT>(v[8 * s + 4] * inv) | (static_cast<uint32_t>(float_to_half<DT>(v[8 * s + 5] * inv)) << 16);
-                    w.w = float_to_half<DT>(v[8 * s + 6] * inv) | (static_cast<uint32_t>(float_to_half<DT>(v[8 * s + 7] * inv)) << 16);
-                    *reinterpret_cast<uint4 *>(y + c) = w;
-                }
+            for (int s = 0; s < NW; ++s) {
+                const int c = s * LPR * 8 + sub * 8;
+                if (c < cols)
+                    *reinterpret_cast<uint4 *>(y + c) = pack8<DT>(v + 8 * s, inv);
             }
         } else {
 #pragma unroll
             for (int s = 0; s < PER_LANE; ++s) {
-                const int c = s * 32 + lane;
+                const int c = s * LPR + sub;
                 if (c < cols)
                     y[c] = float_to_half<DT>(v[s] * inv);
             }
@@ -123,78 +171,261 @@ __global__ void __launch_bounds__(256) softmax_rows_warp_kernel(const uint16_t *
 // ------------------------------------------------------------------ row softmax, one CTA per row, in registers
 // Rows of up to THREADS * PER_THREAD values (16-byte aligned, a multiple of 8
 // long) are read once into registers; block reductions through shared memory.
+// The CTA's next row is loaded (as raw words) before the current one is
+// reduced, so its loads are in flight during the reductions.
 template <int DT, int PER_THREAD>
-__global__ void __launch_bounds__(512) softmax_rows_cta_regs_kernel(const uint16_t *__restrict__ X,
+__global__ void __launch_bounds__(512, PER_THREAD <= 16 ? 3 : 2) softmax_rows_cta_regs_kernel(const uint16_t *__restrict__ X,
                                                                     uint16_t *__restrict__ Y, int64_t rows, int cols)
 {
-    __shared__ float red[16];
+    constexpr int NW = PER_THREAD / 8;
+    __shared__ float red[2][16];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     const int step = blockDim.x * 8;
-    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    uint4 w[NW];
+    auto load = [&](int64_t row) {
+        if (row >= rows)
+            return;
         const uint16_t *x = X + row * cols;
-        uint16_t *y = Y + row * cols;
-        float v[PER_THREAD];
-        float m = -INFINITY;
 #pragma unroll
-        for (int s = 0; s < PER_THREAD / 8; ++s) {
+        for (int s = 0; s < NW; ++s) {
+            const int c = s * step + tid * 8;
+            if (c < cols)
+                w[s] = __ldg(reinterpret_cast<const uint4 *>(x + c));
+        }
+    };
+    load(blockIdx.x);
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+        float v[PER_THREAD];
+#pragma unroll
+        for (int s = 0; s < NW; ++s) {
             const int c = s * step + tid * 8;
             if (c < cols) {
-                const uint4 w = __ldg(reinterpret_cast<const uint4 *>(x + c));
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    v[8 * s + 2 * h] = half_to_float<DT>(static_cast<uint16_t>(ww[h] & 0xFFFFu));
-                    v[8 * s + 2 * h + 1] = half_to_float<DT>(static_cast<uint16_t>(ww[h] >> 16));
-                }
+                unpack8<DT>(w[s], v + 8 * s);
             } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    v[8 * s + e] = -INFINITY;
+                for (int k = 0; k < 8; ++k)
+                    v[8 * s + k] = -INFINITY;
             }
         }
+        load(row + gridDim.x);
+        float m = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < PER_THREAD; ++i)
-            m = fmaxf(m, v[i]);
+        for (int i = 0; i < PER_THREAD; i += 2)
+            m = fmax3(m, v[i], v[i + 1]);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1)
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        // red[0] holds maxima, red[1] sums: the barrier after the sums orders
+        // this row's reads of red[0] before the next row's writes
         if (lane == 0)
-            red[warp] = m;
+            red[0][warp] = m;
         __syncthreads();
-        m = red[0];
-        for (int w = 1; w < nwarps; ++w)
-            m = fmaxf(m, red[w]);
-        __syncthreads();
+        m = red[0][0];
+        for (int k = 1; k < nwarps; ++k)
+            m = fmaxf(m, red[0][k]);
         const float mb = m * kLog2e;
         float sum = 0.0f;
 #pragma unroll
         for (int i = 0; i < PER_THREAD; ++i) {
-            v[i] = exp2_approx(fmaf(v[i], kLog2e, -mb));
+            v[i] = exp2_approx_ftz(fmaf(v[i], kLog2e, -mb));
             sum += v[i];
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1)
             sum += __shfl_xor_sync(0xffffffffu, sum, off);
         if (lane == 0)
-            red[warp] = sum;
+            red[1][warp] = sum;
         __syncthreads();
         sum = 0.0f;
-        for (int w = 0; w < nwarps; ++w)
-            sum += red[w];
-        __syncthreads();
+        for (int k = 0; k < nwarps; ++k)
+            sum += red[1][k];
         const float inv = 1.0f / sum;
+        uint16_t *y = Y + row * cols;
 #pragma unroll
-        for (int s = 0; s < PER_THREAD / 8; ++s) {
+        for (int s = 0; s < NW; ++s) {
             const int c = s * step + tid * 8;
-            if (c < cols) {
-                uint32_t o[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h)
-                    o[h] = float_to_half<DT>(v[8 * s + 2 * h] * inv) |
-                           (static_cast<uint32_t>(float_to_half<DT>(v[8 * s + 2 * h + 1] * inv)) << 16);
-                *reinterpret_cast<uint4 *>(y + c) = make_uint4(o[0], o[1], o[2], o[3]);
-            }
+            if (c < cols)
+                *reinterpret_cast<uint4 *>(y + c) = pack8<DT>(v + 8 * s, inv);
         }
+    }
+}
+
+// ------------------------------------------------------------------ row softmax, one CTA per row, in shared memory
+// Rows too long for registers but short enough for shared memory (up to
+// ~110,000 values).  One thread streams the row's 16-byte-aligned body into
+// shared memory with bulk copies (the TMA engine, completion counted on an
+// mbarrier); the few values before the first and after the last 16-byte
+// boundary are loaded by plain loads.  The row sits in shared memory at the
+// same offset from a 16-byte boundary as in global memory.  With two row
+// buffers (rows up to ~55,000 values) the next row's copy runs while the
+// current row is reduced and written, so HBM reads one row ahead.
+// The wait for a copy is bounded; on expiry the kernel records
+// ERR_ROW_COPY in the device error word and carries on (the row's output is
+// then wrong, which tl_check_device reports), so no thread ever hangs.
+constexpr unsigned ERR_ROW_COPY = 64u;
+
+struct RowSplit {
+    int mis;   // byte offset of the row start from a 16-byte boundary (even)
+    int head;  // values before the first 16-byte boundary
+    int nvec;  // 8-value words in the aligned body
+};
+
+__device__ __forceinline__ RowSplit split_row(const uint16_t *x, int cols)
+{
+    RowSplit r;
+    r.mis = static_cast<int>(reinterpret_cast<uintptr_t>(x) & 15);
+    r.head = min(((16 - r.mis) & 15) >> 1, cols);
+    r.nvec = (cols - r.head) >> 3;
+    return r;
+}
+
+template <int DT>
+__global__ void __launch_bounds__(512) softmax_rows_smem_kernel(const uint16_t *__restrict__ X,
+                                                                uint16_t *__restrict__ Y, int64_t rows, int cols,
+                                                                int y_vec, int nbuf, int buf_bytes,
+                                                                uint64_t timeout_ns)
+{
+    extern __shared__ __align__(128) uint8_t smem_dyn[];
+    // row buffers from the first 128-byte boundary (the launch adds 128 bytes)
+    uint8_t *srow_raw = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 127) &
+                                                    ~static_cast<uintptr_t>(127));
+    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ float red_m[16], red_s[16];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    if (tid == 0) {
+        mbar_init(smem_addr(&bars[0]), 1);
+        mbar_init(smem_addr(&bars[1]), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // one thread: start the copy of `row`'s body into buffer `buf`
+    auto issue = [&](int64_t row, int buf) {
+        const uint16_t *x = X + row * cols;
+        const RowSplit sp = split_row(x, cols);
+        const uint32_t bar = smem_addr(&bars[buf]);
+        if (sp.nvec == 0) {
+            mbar_arrive(bar);
+            return;
+        }
+        const uint32_t bytes = static_cast<uint32_t>(sp.nvec) * 16u;
+        const uint32_t dst = smem_addr(srow_raw + buf * buf_bytes + sp.mis + 2 * sp.head);
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(x + sp.head);
+        fence_proxy_async_smem();  // earlier generic reads of this buffer come first
+        mbar_arrive_expect_tx(bar, bytes);
+        constexpr uint32_t CHUNK = 32768;
+        for (uint32_t off = 0; off < bytes; off += CHUNK)
+            bulk_load_g2s(dst + off, src + off, min(CHUNK, bytes - off), bar);
+    };
+
+    int it = 0;
+    uint32_t phases = 0u;  // bit b: parity of buffer b's next phase
+    if (tid == 0 && static_cast<int64_t>(blockIdx.x) < rows)
+        issue(blockIdx.x, 0);
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x, ++it) {
+        const int buf = nbuf == 2 ? (it & 1) : 0;
+        const int64_t next = row + gridDim.x;
+        if (nbuf == 2 && tid == 0 && next < rows)
+            issue(next, buf ^ 1);  // its buffer was released by the barrier that ended the previous row
+        const uint16_t *x = X + row * cols;
+        uint16_t *y = Y + row * cols;
+        const RowSplit sp = split_row(x, cols);
+        uint16_t *sr = reinterpret_cast<uint16_t *>(srow_raw + buf * buf_bytes + sp.mis);
+        const int body_end = sp.head + (sp.nvec << 3);
+        for (int c = tid; c < sp.head; c += blockDim.x)
+            sr[c] = x[c];
+        for (int c = body_end + tid; c < cols; c += blockDim.x)
+            sr[c] = x[c];
+        {
+            // bounded wait for the body (every thread)
+            const uint32_t bar = smem_addr(&bars[buf]);
+            const uint32_t parity = (phases >> buf) & 1u;
+            if (!mbar_try_wait(bar, parity)) {
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(bar, parity)) {
+                    if (global_timer_ns() - t0 > timeout_ns) {
+                        atomicOr(&g_device_error, ERR_ROW_COPY);
+                        break;
+                    }
+                }
+            }
+            phases ^= 1u << buf;
+        }
+        __syncthreads();  // head and tail visible to every thread
+
+        // running (max, sum) in log2 units over the row in shared memory
+        float m = -INFINITY, s = 0.0f;
+        auto absorb = [&](float t) {
+            if (t > m) {
+                s = s * exp2_approx_ftz(m - t) + 1.0f;
+                m = t;
+            } else {
+                s += exp2_approx_ftz(t - m);
+            }
+        };
+        for (int c = tid; c < sp.head; c += blockDim.x)
+            absorb(half_to_float<DT>(sr[c]) * kLog2e);
+        const uint4 *body = reinterpret_cast<const uint4 *>(sr + sp.head);
+        for (int i = tid; i < sp.nvec; i += blockDim.x) {
+            float t[8];
+            unpack8<DT>(body[i], t);
+            float mx = t[0];
+#pragma unroll
+            for (int e = 1; e < 8; ++e)
+                mx = fmaxf(mx, t[e]);
+            mx *= kLog2e;
+            if (mx > m) {
+                s = (m == -INFINITY) ? 0.0f : s * exp2_approx_ftz(m - mx);
+                m = mx;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                s += exp2_approx_ftz(fmaf(t[e], kLog2e, -m));
+        }
+        for (int c = body_end + tid; c < cols; c += blockDim.x)
+            absorb(half_to_float<DT>(sr[c]) * kLog2e);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+            const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
+            const float mm = fmaxf(m, m2);
+            s = (m == -INFINITY ? 0.0f : s * exp2_approx_ftz(m - mm)) + (m2 == -INFINITY ? 0.0f : s2 * exp2_approx_ftz(m2 - mm));
+            m = mm;
+        }
+        if (lane == 0) {
+            red_m[warp] = m;
+            red_s[warp] = s;
+        }
+        __syncthreads();
+        float M = -INFINITY;
+        for (int k = 0; k < nwarps; ++k)
+            M = fmaxf(M, red_m[k]);
+        float S = 0.0f;
+        for (int k = 0; k < nwarps; ++k)
+            if (red_m[k] != -INFINITY)
+                S += red_s[k] * exp2_approx_ftz(red_m[k] - M);
+        const float inv = 1.0f / S;
+        if (y_vec) {
+            // y lies as far from a 16-byte boundary as x: whole words for the body
+            for (int c = tid; c < sp.head; c += blockDim.x)
+                y[c] = float_to_half<DT>(exp2_approx_ftz(fmaf(half_to_float<DT>(sr[c]), kLog2e, -M)) * inv);
+            for (int i = tid; i < sp.nvec; i += blockDim.x) {
+                float t[8];
+                unpack8<DT>(body[i], t);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    t[e] = exp2_approx_ftz(fmaf(t[e], kLog2e, -M));
+                __stcs(reinterpret_cast<uint4 *>(y + sp.head) + i, pack8<DT>(t, inv));
+            }
+            for (int c = body_end + tid; c < cols; c += blockDim.x)
+                y[c] = float_to_half<DT>(exp2_approx_ftz(fmaf(half_to_float<DT>(sr[c]), kLog2e, -M)) * inv);
+        } else {
+            for (int c = tid; c < cols; c += blockDim.x)
+                y[c] = float_to_half<DT>(exp2_approx_ftz(fmaf(half_to_float<DT>(sr[c]), kLog2e, -M)) * inv);
+        }
+        __syncthreads();  // the row buffer and red_* are free for the next row
+        if (nbuf == 1 && tid == 0 && next < rows)
+            issue(next, 0);
     }
 }
 
@@ -226,10 +457,10 @@ __global__ void __launch_bounds__(512) softmax_rows_block_kernel(const uint16_t 
         float m = -INFINITY, s = 0.0f;  // in log2 units: s = sum 2^(t - m)
         auto absorb = [&](float t) {
             if (t > m) {
-                s = s * exp2_approx(m - t) + 1.0f;
+                s = s * exp2_approx_ftz(m - t) + 1.0f;
                 m = t;
             } else {
-                s += exp2_approx(t - m);
+                s += exp2_approx_ftz(t - m);
             }
         };
         for (int64_t c = tid; c < head; c += blockDim.x)
@@ -248,12 +479,12 @@ __global__ void __launch_bounds__(512) softmax_rows_block_kernel(const uint16_t 
             for (int e = 1; e < 8; ++e)
                 mx = fmaxf(mx, t[e]);
             if (mx > m) {
-                s = (m == -INFINITY) ? 0.0f : s * exp2_approx(m - mx);
+                s = (m == -INFINITY) ? 0.0f : s * exp2_approx_ftz(m - mx);
                 m = mx;
             }
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                s += exp2_approx(t[e] - m);
+                s += exp2_approx_ftz(t[e] - m);
         }
         for (int64_t c = body_end + tid; c < cols; c += blockDim.x)
             absorb(half_to_float<DT>(x[c]) * kLog2e);
@@ -263,7 +494,7 @@ __global__ void __launch_bounds__(512) softmax_rows_block_kernel(const uint16_t 
             const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
             const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
             const float mm = fmaxf(m, m2);
-            s = (m == -INFINITY ? 0.0f : s * exp2_approx(m - mm)) + (m2 == -INFINITY ? 0.0f : s2 * exp2_approx(m2 - mm));
+            s = (m == -INFINITY ? 0.0f : s * exp2_approx_ftz(m - mm)) + (m2 == -INFINITY ? 0.0f : s2 * exp2_approx_ftz(m2 - mm));
             m = mm;
         }
         if (lane == 0) {
@@ -277,25 +508,25 @@ __global__ void __launch_bounds__(512) softmax_rows_block_kernel(const uint16_t 
         float S = 0.0f;
         for (int w = 0; w < nwarps; ++w)
             if (red_m[w] != -INFINITY)
-                S += red_s[w] * exp2_approx(red_m[w] - M);
+                S += red_s[w] * exp2_approx_ftz(red_m[w] - M);
         __syncthreads();  // red_* reused by the next row
         const float inv = 1.0f / S;
         for (int64_t c = tid; c < head; c += blockDim.x)
-            y[c] = float_to_half<DT>(exp2_approx(fmaf(half_to_float<DT>(x[c]), kLog2e, -M)) * inv);
+            y[c] = float_to_half<DT>(exp2_approx_ftz(fmaf(half_to_float<DT>(x[c]), kLog2e, -M)) * inv);
         for (int64_t i = tid; i < nvec; i += blockDim.x) {
             const uint4 w = __ldg(reinterpret_cast<const uint4 *>(x + head) + i);
             const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
             uint32_t o[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-                const float a = exp2_approx(fmaf(half_to_float<DT>(static_cast<uint16_t>(ww[h] & 0xFFFFu)), kLog2e, -M)) * inv;
-                const float b = exp2_approx(fmaf(half_to_float<DT>(static_cast<uint16_t>(ww[h] >> 16)), kLog2e, -M)) * inv;
+                const float a = exp2_approx_ftz(fmaf(half_to_float<DT>(static_cast<uint16_t>(ww[h] & 0xFFFFu)), kLog2e, -M)) * inv;
+                const float b = exp2_approx_ftz(fmaf(half_to_float<DT>(static_cast<uint16_t>(ww[h] >> 16)), kLog2e, -M)) * inv;
                 o[h] = float_to_half<DT>(a) | (static_cast<uint32_t>(float_to_half<DT>(b)) << 16);
             }
             reinterpret_cast<uint4 *>(y + head)[i] = make_uint4(o[0], o[1], o[2], o[3]);
         }
         for (int64_t c = body_end + tid; c < cols; c += blockDim.x)
-            y[c] = float_to_half<DT>(exp2_approx(fmaf(half_to_float<DT>(x[c]), kLog2e, -M)) * inv);
+            y[c] = float_to_half<DT>(exp2_approx_ftz(fmaf(half_to_float<DT>(x[c]), kLog2e, -M)) * inv);
     }
 }
 

@@ -761,6 +761,22 @@ tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, f
 }
 
 // ------------------------------------------------------------------ row softmax and vector add
+// Largest dynamic shared memory the row-in-shared-memory softmax takes (one
+// row of 16-bit values plus 16 bytes of alignment slack).
+constexpr int64_t kSoftmaxSmemMax = 220 * 1024;
+
+// Persistent grid for a row kernel: one CTA per row, at most as many as can
+// be resident at once on every SM (so no CTA waits for a second wave).
+template <class Fn>
+int64_t resident_grid(DeviceState *d, Fn fn, int threads, size_t smem, int64_t work_blocks)
+{
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    const int64_t cap = static_cast<int64_t>(d->num_sms) * per_sm;
+    return work_blocks < cap ? work_blocks : cap;
+}
+
 tl_status softmax_impl(const void *X, void *Y, int64_t rows, int64_t cols, int dtype, cudaStream_t stream)
 {
     if (!X || !Y || rows < 1 || cols < 1)
@@ -780,43 +796,72 @@ tl_status softmax_impl(const void *X, void *Y, int64_t rows, int64_t cols, int d
     uint16_t *y = static_cast<uint16_t *>(Y);
     const int c = static_cast<int>(cols);
     if (cols <= 1024) {
-        int64_t blocks = ceil_div(rows, 8);
-        const int64_t cap = static_cast<int64_t>(d->num_sms) * 16;
-        if (blocks > cap)
-            blocks = cap;
-        const dim3 g(static_cast<unsigned>(blocks)), b(256);
-#define TL_SOFTMAX_WARP(DT)                                                                         \
-    do {                                                                                            \
-        if (cols <= 256)                                                                            \
-            vec ? softmax_rows_warp_kernel<DT, 8, true><<<g, b, 0, stream>>>(x, y, rows, c)         \
-                : softmax_rows_warp_kernel<DT, 8, false><<<g, b, 0, stream>>>(x, y, rows, c);       \
-        else                                                                                        \
-            vec ? softmax_rows_warp_kernel<DT, 32, true><<<g, b, 0, stream>>>(x, y, rows, c)        \
-                : softmax_rows_warp_kernel<DT, 32, false><<<g, b, 0, stream>>>(x, y, rows, c);      \
+        // lanes per row: short rows share a warp
+        const int lpr = cols <= 64 ? 8 : cols <= 128 ? 16 : 32;
+        const int64_t work = ceil_div(rows, 8 * (32 / lpr));
+        const dim3 b(256);
+#define TL_SOFTMAX_WARP_LAUNCH(DT, P, V, L)                                                          \
+    do {                                                                                             \
+        auto fn = softmax_rows_warp_kernel<DT, P, V, L>;                                             \
+        const dim3 g(static_cast<unsigned>(resident_grid(d, fn, 256, 0, work)));                     \
+        fn<<<g, b, 0, stream>>>(x, y, rows, c);                                                      \
     } while (0)
-        if (dtype == TL_BF16)
-            TL_SOFTMAX_WARP(1);
-        else
-            TL_SOFTMAX_WARP(0);
-#undef TL_SOFTMAX_WARP
-    } else if (vec && cols <= 16384) {
-        // the row in registers: 512 threads x up to 32 values, one read
-        int64_t blocks = rows;
-        const int64_t cap = static_cast<int64_t>(d->num_sms) * 4;
-        if (blocks > cap)
-            blocks = cap;
-        const dim3 g(static_cast<unsigned>(blocks)), b(cols <= 4096 ? 256 : 512);
-        if (cols <= 8192) {
-            if (dtype == TL_BF16)
-                softmax_rows_cta_regs_kernel<1, 16><<<g, b, 0, stream>>>(x, y, rows, c);
+#define TL_SOFTMAX_WARP(DT, V)                                                                       \
+    do {                                                                                             \
+        if (cols <= 64)                                                                              \
+            TL_SOFTMAX_WARP_LAUNCH(DT, 8, V, 8);                                                     \
+        else if (cols <= 128)                                                                        \
+            TL_SOFTMAX_WARP_LAUNCH(DT, 8, V, 16);                                                    \
+        else if (cols <= 256)                                                                        \
+            TL_SOFTMAX_WARP_LAUNCH(DT, 8, V, 32);                                                    \
+        else                                                                                         \
+            TL_SOFTMAX_WARP_LAUNCH(DT, 32, V, 32);                                                   \
+    } while (0)
+        if (dtype == TL_BF16) {
+            if (vec)
+                TL_SOFTMAX_WARP(1, true);
             else
-                softmax_rows_cta_regs_kernel<0, 16><<<g, b, 0, stream>>>(x, y, rows, c);
+                TL_SOFTMAX_WARP(1, false);
         } else {
-            if (dtype == TL_BF16)
-                softmax_rows_cta_regs_kernel<1, 32><<<g, b, 0, stream>>>(x, y, rows, c);
+            if (vec)
+                TL_SOFTMAX_WARP(0, true);
             else
-                softmax_rows_cta_regs_kernel<0, 32><<<g, b, 0, stream>>>(x, y, rows, c);
+                TL_SOFTMAX_WARP(0, false);
         }
+#undef TL_SOFTMAX_WARP
+#undef TL_SOFTMAX_WARP_LAUNCH
+    } else if (vec && cols <= 16384) {
+        // the row in registers: 256 or 512 threads x up to 32 values, one read
+        const int threads = cols <= 4096 ? 256 : 512;
+        const dim3 b(threads);
+        auto launch = [&](auto fn) {
+            const dim3 g(static_cast<unsigned>(resident_grid(d, fn, threads, 0, rows)));
+            fn<<<g, b, 0, stream>>>(x, y, rows, c);
+        };
+        if (cols <= 8192)
+            dtype == TL_BF16 ? launch(softmax_rows_cta_regs_kernel<1, 16>) : launch(softmax_rows_cta_regs_kernel<0, 16>);
+        else
+            dtype == TL_BF16 ? launch(softmax_rows_cta_regs_kernel<1, 32>) : launch(softmax_rows_cta_regs_kernel<0, 32>);
+    } else if (ceil_div(2 * cols + 16, 128) * 128 + 128 <= kSoftmaxSmemMax) {
+        // the row in shared memory, read from HBM once by bulk copies; two
+        // row buffers when they fit, so the next row streams in meanwhile
+        const int buf_bytes = static_cast<int>(ceil_div(2 * cols + 16, 128) * 128);
+        const int nbuf = 2 * static_cast<int64_t>(buf_bytes) + 128 <= kSoftmaxSmemMax ? 2 : 1;
+        const int smem = nbuf * buf_bytes + 128;  // + slack to a 128-byte boundary
+        const dim3 b(512);
+        // y's body takes whole words when y lies as far from a 16-byte
+        // boundary as x (then every row's x and y do)
+        const int y_vec = ((reinterpret_cast<uintptr_t>(X) - reinterpret_cast<uintptr_t>(Y)) & 15) == 0;
+        auto launch = [&](auto fn) -> tl_status {
+            tl_status r = raise_smem_limit(d, reinterpret_cast<KernelFn>(fn), static_cast<int>(kSoftmaxSmemMax));
+            if (r != TL_OK)
+                return r;
+            const dim3 g(static_cast<unsigned>(resident_grid(d, fn, 512, static_cast<size_t>(smem), rows)));
+            fn<<<g, b, smem, stream>>>(x, y, rows, c, y_vec, nbuf, buf_bytes, kDefaultTimeoutNs);
+            return TL_OK;
+        };
+        if ((st = dtype == TL_BF16 ? launch(softmax_rows_smem_kernel<1>) : launch(softmax_rows_smem_kernel<0>)) != TL_OK)
+            return st;
     } else {
         int64_t blocks = rows;
         const int64_t cap = static_cast<int64_t>(d->num_sms) * 4;

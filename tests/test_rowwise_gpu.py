@@ -1,7 +1,8 @@
 """Row softmax and vector add on the GPU (through the C ABI) against the
 oracle.  Softmax: every element within half an output ulp plus 1e-5
-relative (float32 evaluation with the hardware exp2) of the fp64 softmax.
-Vector add: bit for bit."""
+relative (float32 evaluation with the hardware exp2) of the fp64 softmax;
+probabilities below 2^-126 may come out as 0 (the flush-to-zero exp2), which
+the bound allows by adding |ref| there.  Vector add: bit for bit."""
 import os
 import sys
 
@@ -14,17 +15,23 @@ import oracle  # noqa: E402
 import workloads as wl  # noqa: E402
 from gpu_util import from_device, to_device, ulp  # noqa: E402
 
+
+def softmax_bound(ref, dt):
+    """Half an output ulp + 1e-5 relative, and below 2^-126 the value itself."""
+    return 0.5 * ulp(ref, dt) + 1e-5 * ref + np.where(ref < 2.0 ** -126, ref, 0.0) + 1e-40
+
 torch = pytest.importorskip("torch")
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 
-def run_softmax(X_bits, dt, offset=0):
+def run_softmax(X_bits, dt, offset=0, y_offset=None):
     import tensor_core_gemm_tl_b200 as tg
     x = to_device(X_bits, dt, offset)
-    if offset:
-        buf = torch.empty(x.numel() + offset, dtype=x.dtype, device="cuda")
-        y = buf[offset:].view(x.shape)
+    y_offset = offset if y_offset is None else y_offset
+    if y_offset:
+        buf = torch.empty(x.numel() + y_offset, dtype=x.dtype, device="cuda")
+        y = buf[y_offset:].view(x.shape)
     else:
         y = torch.empty_like(x)
     tg.softmax(x, out=y)
@@ -32,8 +39,9 @@ def run_softmax(X_bits, dt, offset=0):
     return from_device(y)
 
 
-@pytest.mark.parametrize("rows,cols", [(1, 1), (3, 7), (64, 33), (1000, 256), (257, 1000), (128, 1024),
-                                       (40, 1025), (17, 4096), (9, 12288), (8, 50000), (3, 50257),
+@pytest.mark.parametrize("rows,cols", [(1, 1), (3, 7), (64, 33), (333, 64), (1001, 100), (1000, 128),
+                                       (1000, 256), (257, 1000), (128, 1024), (40, 1025), (17, 4096),
+                                       (9, 12288), (11, 16385), (8, 50000), (3, 50257), (5, 112000),
                                        (2, 200000)])
 @pytest.mark.parametrize("dt", [wl.F16, wl.BF16])
 def test_softmax_vs_oracle(rows, cols, dt):
@@ -41,7 +49,7 @@ def test_softmax_vs_oracle(rows, cols, dt):
     X = wl.round_to_bits((rng.normal(size=(rows, cols)) * 3).astype(np.float32), dt)
     ref = oracle.softmax_rows(X, dt)
     Y = wl.bits_to_float32(run_softmax(X, dt), dt).astype(np.float64)
-    bound = 0.5 * ulp(ref, dt) + 1e-5 * ref + 1e-40
+    bound = softmax_bound(ref, dt)
     assert np.all(np.abs(Y - ref) <= bound), np.max(np.abs(Y - ref) - bound)
 
 
@@ -56,7 +64,7 @@ def test_softmax_benchmark_sizes_sampled_rows(rows, cols):
     pick = np.unique(np.concatenate([[0, rows - 1], rng.integers(0, rows, 200)]))
     ref = oracle.softmax_rows(np.ascontiguousarray(X[pick]), dt)
     got = wl.bits_to_float32(Y[pick], dt).astype(np.float64)
-    assert np.all(np.abs(got - ref) <= 0.5 * ulp(ref, dt) + 1e-5 * ref + 1e-40)
+    assert np.all(np.abs(got - ref) <= softmax_bound(ref, dt))
 
 
 @pytest.mark.parametrize("offset", [1, 3])
@@ -67,7 +75,20 @@ def test_softmax_unaligned(offset):
         X = wl.round_to_bits(rng.normal(size=(rows, cols)).astype(np.float32), dt)
         ref = oracle.softmax_rows(X, dt)
         Y = wl.bits_to_float32(run_softmax(X, dt, offset), dt).astype(np.float64)
-        assert np.all(np.abs(Y - ref) <= 0.5 * ulp(ref, dt) + 1e-5 * ref + 1e-40)
+        assert np.all(np.abs(Y - ref) <= softmax_bound(ref, dt))
+
+
+@pytest.mark.parametrize("x_off,y_off", [(1, 2), (0, 3), (5, 0)])
+@pytest.mark.parametrize("cols", [600, 3000, 20001, 70000])
+def test_softmax_input_and_output_differently_aligned(x_off, y_off, cols):
+    """X and Y at different distances from a 16-byte boundary: no row body can
+    move as whole words on both sides (element path throughout)."""
+    dt = wl.F16
+    rng = np.random.default_rng(cols + x_off)
+    X = wl.round_to_bits(rng.normal(size=(6, cols)).astype(np.float32), dt)
+    ref = oracle.softmax_rows(X, dt)
+    Y = wl.bits_to_float32(run_softmax(X, dt, x_off, y_off), dt).astype(np.float64)
+    assert np.all(np.abs(Y - ref) <= softmax_bound(ref, dt))
 
 
 def test_softmax_constant_and_dominant_rows():
