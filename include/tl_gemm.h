@@ -181,8 +181,11 @@ TL_API tl_status tl_attention_fwd(const void *Q, const void *K, const void *V, v
  * row-wise softmax with max and sum reductions).  X and Y are device pointers
  * to rows x cols row-major `dtype` values (2-byte aligned; 16-byte aligned with
  * cols a multiple of 8 for the vectorised path); Y may equal X.  Computed in
- * fp32 with the row maximum subtracted, rounded once to `dtype`.  rows, cols
- * >= 1.  Asynchronous on `stream`; allocates nothing.
+ * fp32 with the row maximum subtracted, rounded once to `dtype`;
+ * probabilities below 2^-126 are returned as 0.  rows, cols >= 1.
+ * Asynchronous on `stream`; allocates nothing.  Rows of up to ~110,000 values
+ * are read into shared memory by bulk copies whose wait is bounded; a wait
+ * that runs out is reported by tl_check_device (bit 6).
  */
 TL_API tl_status tl_softmax_rows(const void *X, void *Y, int64_t rows, int64_t cols, tl_dtype dtype,
                          tl_stream stream);
@@ -229,7 +232,8 @@ TL_API tl_status tl_gemm_ex(const void *A, const void *B, const void *bias, void
  * otherwise.  `detail`, if not NULL, receives the raw error word (which waits
  * gave up: bit 0 copy warp, bit 1 MMA warp on data, bit 2 MMA warp on the
  * accumulator, bit 3 epilogue warps, bit 4 final drain, bit 5 the last K part
- * of a split tile waiting for an earlier part).
+ * of a split tile waiting for an earlier part, bit 6 the row softmax waiting
+ * for a row's copy into shared memory).
  */
 TL_API tl_status tl_check_device(tl_stream stream, uint32_t *detail);
 
