@@ -17,6 +17,7 @@
 #include "tl_gemm.h"
 #include "gemm_kernel.cuh"
 #include "attention_kernel.cuh"
+#include "attention_pp_kernel.cuh"
 #include "rowwise_kernels.cuh"
 
 namespace tl {
@@ -645,20 +646,23 @@ using AttnFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, AttnParams);
 struct AttnEntry {
     int smem_bytes;
     int threads;
-    int launch_regs;  // registers a thread the warpgroup register split needs at launch
-    AttnFn fn[2];  // [dtype]
+    int launch_regs;     // registers a thread the warpgroup register split needs at launch
+    int tiles_per_cta;   // 128-row query tiles one CTA computes
+    AttnFn fn[2];        // [dtype]
 };
 
+// Two query tiles per CTA in ping-pong (attention_pp_kernel.cuh)
 template <int D>
 AttnEntry make_attn_entry()
 {
-    using CF = AttnConfig<D>;
+    using CF = AttnPPConfig<D>;
     AttnEntry e;
     e.smem_bytes = CF::SMEM_BYTES;
     e.threads = CF::THREADS;
     e.launch_regs = CF::LAUNCH_REGS;
-    e.fn[0] = attention_fwd_kernel<CF, 0>;
-    e.fn[1] = attention_fwd_kernel<CF, 1>;
+    e.tiles_per_cta = CF::TILES;
+    e.fn[0] = attention_fwd_pp_kernel<CF, 0>;
+    e.fn[1] = attention_fwd_pp_kernel<CF, 1>;
     return e;
 }
 
@@ -747,7 +751,7 @@ tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, f
 
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];
-    cfg.gridDim = dim3(static_cast<unsigned>(ap.num_qtiles), static_cast<unsigned>(BH), 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(ceil_div(ap.num_qtiles, e.tiles_per_cta)), static_cast<unsigned>(BH), 1);
     cfg.blockDim = dim3(static_cast<unsigned>(e.threads), 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(e.smem_bytes);
     cfg.stream = stream;
