@@ -17,7 +17,6 @@
 #include "tl_gemm.h"
 #include "gemm_kernel.cuh"
 #include "attention_kernel.cuh"
-#include "attention_pp_kernel.cuh"
 #include "rowwise_kernels.cuh"
 
 namespace tl {
@@ -651,18 +650,18 @@ struct AttnEntry {
     AttnFn fn[2];        // [dtype]
 };
 
-// Two query tiles per CTA in ping-pong (attention_pp_kernel.cuh)
+// Two query tiles per CTA in ping-pong (attention_kernel.cuh)
 template <int D>
 AttnEntry make_attn_entry()
 {
-    using CF = AttnPPConfig<D>;
+    using CF = AttnConfig<D>;
     AttnEntry e;
     e.smem_bytes = CF::SMEM_BYTES;
     e.threads = CF::THREADS;
     e.launch_regs = CF::LAUNCH_REGS;
     e.tiles_per_cta = CF::TILES;
-    e.fn[0] = attention_fwd_pp_kernel<CF, 0>;
-    e.fn[1] = attention_fwd_pp_kernel<CF, 1>;
+    e.fn[0] = attention_fwd_kernel<CF, 0>;
+    e.fn[1] = attention_fwd_kernel<CF, 1>;
     return e;
 }
 
