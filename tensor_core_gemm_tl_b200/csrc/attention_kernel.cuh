@@ -17,14 +17,17 @@
 //
 //   S_i = Q_i K_j^T       tcgen05.mma (A, B from shared memory) into S_i
 //   P_i = 2^(S_i' - m_i)  the tile's softmax warpgroup, one query row per
-//                         thread: 16-bit weights written back over S_i's first
-//                         64 columns with tcgen05.st
+//                         thread: 16-bit weights written with tcgen05.st over
+//                         S_i's first 64 columns (head_dim 128) or into
+//                         columns of their own (head_dim 64)
 //   O_i += P_i V_j        tcgen05.mma with A = P_i read from Tensor Memory
 //
-// The MMA thread issues PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ...: while one
-// warpgroup turns S into P, the tensor core works on the other tile.  S_i(j+1)
-// overwrites the columns PV_i(j) reads, so it is issued only once PV_i(j) has
-// completed.  The running maximum m_i used for P only moves when a row's new
+// With head_dim 128 the MMA thread issues PV_0(j), S_0(j+1), PV_1(j),
+// S_1(j+1), ...: while one warpgroup turns S into P, the tensor core works on
+// the other tile; S_i(j+1) overwrites the columns PV_i(j) reads, so it is
+// issued only once PV_i(j) has completed.  With head_dim 64 it issues
+// S_0(j+1), S_1(j+1) as soon as the softmax has read S_i(j), then PV_0(j),
+// PV_1(j); the softmax writes P_i(j+1) once PV_i(j) has completed.  The running maximum m_i used for P only moves when a row's new
 // maximum exceeds it by more than 2^8: then (rarely, after the first blocks)
 // the warp multiplies its rows of O_i by 2^(m_old - m_new) in Tensor Memory
 // before P_i(j) is released; otherwise the weights stay below 256.
@@ -69,15 +72,24 @@ struct AttnConfig {
     static constexpr int BAR_SF = 1 + 4 * KS;   // [tile]: S_i(j) in Tensor Memory
     static constexpr int BAR_PF = BAR_SF + 2;   // [tile]: P_i(j) in Tensor Memory (4 warps arrive)
     static constexpr int BAR_PV = BAR_PF + 2;   // [tile]: O_i += P_i(j) V_j completed
-    static constexpr int BAR_DRAIN = BAR_PV + 2;
+    static constexpr int BAR_SE = BAR_PV + 2;   // [tile]: S_i(j) read into registers (4 warps; separate P only)
+    static constexpr int BAR_DRAIN = BAR_SE + 2;
     static constexpr int NUM_BARS = BAR_DRAIN + 1;
     static constexpr int SMEM_USED = OFF_BAR + NUM_BARS * 8 + 16;
     static constexpr int SMEM_BYTES = SMEM_USED + 1024;
     static constexpr int THREADS = 384;
     static constexpr int FIRST_SOFTMAX_WARP = 4;
-    static constexpr int REGS_CONTROL = 72, REGS_SOFTMAX = 208;
+    static constexpr int REGS_CONTROL = 64, REGS_SOFTMAX = 216;
     static constexpr int LAUNCH_REGS = (128 * REGS_CONTROL + 256 * REGS_SOFTMAX + THREADS - 1) / THREADS;
     static constexpr int TMEM_S = 0, TMEM_O = 256;  // S_i at 128 i, O_i at 256 + D i
+    // With D = 64 Tensor Memory has room for P_i in columns of its own (at
+    // 384 + 64 i): S_i(j+1) can then be computed as soon as the softmax has
+    // read S_i(j), while P_i(j) waits for its P V.  With D = 128, P_i(j) is
+    // written over the first 64 columns of S_i.
+    static constexpr bool SEPARATE_P = D == 64;
+    static constexpr int TMEM_P = 256 + 2 * D;
+    __host__ __device__ static constexpr int p_col(int i) { return SEPARATE_P ? TMEM_P + 64 * i : TMEM_S + 128 * i; }
+    static_assert(!SEPARATE_P || TMEM_P + 128 <= 512, "Tensor Memory columns");
     static constexpr float RESCALE_LOG2 = 8.0f;     // m moves when a row maximum exceeds it by 2^8
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -130,6 +142,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(bar(CF::BAR_SF + i), 1);
             mbar_init(bar(CF::BAR_PF + i), 4);
             mbar_init(bar(CF::BAR_PV + i), 1);
+            mbar_init(bar(CF::BAR_SE + i), 4);
         }
         mbar_init(bar(CF::BAR_DRAIN), 1);
         *abort_flag = 0;
@@ -224,7 +237,7 @@ __global__ void __launch_bounds__(384, 1)
                 };
                 auto issue_pv = [&](int i, int j) {  // O_i (+)= P_i V from the current V slot
                     const uint32_t d_o = tmem_base + static_cast<uint32_t>(CF::TMEM_O + i * D);
-                    const uint32_t a_p = tmem_base + static_cast<uint32_t>(CF::TMEM_S + i * 128);
+                    const uint32_t a_p = tmem_base + static_cast<uint32_t>(CF::p_col(i));
                     const uint64_t vd = v_desc0 + ((vst * CF::KV_BYTES) >> 4);
 #pragma unroll
                     for (int k = 0; k < CF::BN / 16; ++k)  // 16 keys: 8 columns of P, 2048 B down V
@@ -249,37 +262,73 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 for (int j = 0; ok && j < nbmax; ++j) {
                     const uint32_t jp = static_cast<uint32_t>(j) & 1u;
-                    if (!wait_bounded(bar(CF::BAR_VF + vst), vph, abort_flag, timeout, ERR_MMA_DATA)) {
-                        ok = false;
-                        break;
-                    }
                     bool k_ready = false;  // K(j + 1) waited for
-                    for (int i = 0; ok && i < 2; ++i) {
-                        if (j < nbt(i)) {
-                            if (!wait_bounded(bar(CF::BAR_PF + i), jp, abort_flag, timeout, ERR_MMA_DATA)) {
-                                ok = false;
-                                break;
+                    if constexpr (CF::SEPARATE_P) {
+                        // S_i(j + 1) as soon as the softmax holds S_i(j) in registers
+                        for (int i = 0; ok && i < 2; ++i) {
+                            if (j + 1 < nbt(i)) {
+                                if ((!k_ready && !wait_bounded(bar(CF::BAR_KF + kst), kph, abort_flag, timeout,
+                                                               ERR_MMA_DATA)) ||
+                                    !wait_bounded(bar(CF::BAR_SE + i), jp, abort_flag, timeout, ERR_MMA_ACC)) {
+                                    ok = false;
+                                    break;
+                                }
+                                k_ready = true;
+                                tc_fence_after_sync();
+                                issue_s(i);
                             }
-                            tc_fence_after_sync();
-                            issue_pv(i, j);
                         }
-                        if (i == 1)
-                            tc_commit(bar(CF::BAR_VE + vst));  // V(j) free once the last P V of block j is done
-                        if (j + 1 < nbt(i)) {
-                            // S_i(j + 1) overwrites the P_i(j) that PV_i(j) reads: wait for it
-                            if ((!k_ready && !wait_bounded(bar(CF::BAR_KF + kst), kph, abort_flag, timeout,
-                                                           ERR_MMA_DATA)) ||
-                                !wait_bounded(bar(CF::BAR_PV + i), jp, abort_flag, timeout, ERR_MMA_ACC)) {
-                                ok = false;
-                                break;
+                        if (!ok)
+                            break;
+                        if (!wait_bounded(bar(CF::BAR_VF + vst), vph, abort_flag, timeout, ERR_MMA_DATA)) {
+                            ok = false;
+                            break;
+                        }
+                        for (int i = 0; ok && i < 2; ++i) {
+                            if (j < nbt(i)) {
+                                if (!wait_bounded(bar(CF::BAR_PF + i), jp, abort_flag, timeout, ERR_MMA_DATA)) {
+                                    ok = false;
+                                    break;
+                                }
+                                tc_fence_after_sync();
+                                issue_pv(i, j);
                             }
-                            k_ready = true;
-                            tc_fence_after_sync();
-                            issue_s(i);
                         }
+                        if (!ok)
+                            break;
+                        tc_commit(bar(CF::BAR_VE + vst));  // V(j) free once the P V of block j are done
+                    } else {
+                        if (!wait_bounded(bar(CF::BAR_VF + vst), vph, abort_flag, timeout, ERR_MMA_DATA)) {
+                            ok = false;
+                            break;
+                        }
+                        for (int i = 0; ok && i < 2; ++i) {
+                            if (j < nbt(i)) {
+                                if (!wait_bounded(bar(CF::BAR_PF + i), jp, abort_flag, timeout, ERR_MMA_DATA)) {
+                                    ok = false;
+                                    break;
+                                }
+                                tc_fence_after_sync();
+                                issue_pv(i, j);
+                            }
+                            if (i == 1)
+                                tc_commit(bar(CF::BAR_VE + vst));  // V(j) free once the last P V of block j is done
+                            if (j + 1 < nbt(i)) {
+                                // S_i(j + 1) overwrites the P_i(j) that PV_i(j) reads: wait for it
+                                if ((!k_ready && !wait_bounded(bar(CF::BAR_KF + kst), kph, abort_flag, timeout,
+                                                               ERR_MMA_DATA)) ||
+                                    !wait_bounded(bar(CF::BAR_PV + i), jp, abort_flag, timeout, ERR_MMA_ACC)) {
+                                    ok = false;
+                                    break;
+                                }
+                                k_ready = true;
+                                tc_fence_after_sync();
+                                issue_s(i);
+                            }
+                        }
+                        if (!ok)
+                            break;
                     }
-                    if (!ok)
-                        break;
                     if (++vst == KS) {
                         vst = 0;
                         vph ^= 1u;
@@ -307,6 +356,8 @@ __global__ void __launch_bounds__(384, 1)
         const int nb = nbt(tile);
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const uint32_t s_addr = tmem_base + lane_base + static_cast<uint32_t>(CF::TMEM_S + tile * 128);
+        const uint32_t p_addr =
+            CF::SEPARATE_P ? tmem_base + lane_base + static_cast<uint32_t>(CF::p_col(tile)) : s_addr;
         const uint32_t o_addr = tmem_base + lane_base + static_cast<uint32_t>(CF::TMEM_O + tile * D);
         auto wait_warp = [&](int id, uint32_t parity) -> bool {
             const bool w = wait_bounded(bar(id), parity, abort_flag, timeout, ERR_EPILOGUE);
@@ -326,6 +377,13 @@ __global__ void __launch_bounds__(384, 1)
             for (int c = 0; c < 4; ++c)
                 tmem_load_32cols(s_addr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * c]));
             tmem_load_wait();
+            if constexpr (CF::SEPARATE_P) {
+                // S_i(j) is in registers: its columns may take S_i(j + 1)
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar(CF::BAR_SE + tile));
+            }
             const int key0 = j * CF::BN;
             int nvalid = min(p.Sk, key0 + CF::BN) - key0;
             if (p.causal)
@@ -355,6 +413,12 @@ __global__ void __launch_bounds__(384, 1)
             const float m_new = resc ? mx : m;
             const float m_ref = m_new == -INFINITY ? 0.0f : m_new;  // no visible key yet: all weights 0
             const float alpha = resc ? exp2_approx_ftz(m - m_ref) : 1.0f;  // 0 when m is -inf
+            if constexpr (CF::SEPARATE_P) {
+                // P_i's columns are free once PV_i(j - 1) has read them
+                if (j > 0 && !(ok = wait_warp(CF::BAR_PV + tile, jp ^ 1u)))
+                    break;
+                tc_fence_after_sync();
+            }
             float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -367,14 +431,14 @@ __global__ void __launch_bounds__(384, 1)
                     part[e2 & 3] += w0 + w1;
                     pk[e2] = pack2<DT>(w0, w1);  // keys 2 e2, 2 e2 + 1 of this half: one 32-bit column
                 }
-                tmem_store_32cols(s_addr + 32 * h, pk);
+                tmem_store_32cols(p_addr + 32 * h, pk);
             }
             l = l * alpha + ((part[0] + part[1]) + (part[2] + part[3]));
             m = m_new;
             // the rows whose maximum moved take O_i down by alpha (O_i holds
             // blocks 0 .. j-1, so PV_i(j - 1) has to be complete)
             if (j > 0 && __any_sync(0xffffffffu, resc)) {
-                if (!(ok = wait_warp(CF::BAR_PV + tile, jp ^ 1u)))
+                if (!CF::SEPARATE_P && !(ok = wait_warp(CF::BAR_PV + tile, jp ^ 1u)))
                     break;
                 tc_fence_after_sync();
 #pragma unroll 1
