@@ -849,7 +849,11 @@ tl_status softmax_impl(const void *X, void *Y, int64_t rows, int64_t cols, int d
         // the row in shared memory, read from HBM once by bulk copies; two
         // row buffers when they fit, so the next row streams in meanwhile
         const int buf_bytes = static_cast<int>(ceil_div(2 * cols + 16, 128) * 128);
-        const int nbuf = 2 * static_cast<int64_t>(buf_bytes) + 128 <= kSoftmaxSmemMax ? 2 : 1;
+        // two CTAs of one row buffer each when both fit on an SM (two rows'
+        // reductions overlap), else one CTA with two buffers when they fit
+        // (the next row streams in during the reductions), else one buffer
+        const bool two_ctas = 2 * (static_cast<int64_t>(buf_bytes) + 128 + 1024) <= kSoftmaxSmemMax;
+        const int nbuf = !two_ctas && 2 * static_cast<int64_t>(buf_bytes) + 128 <= kSoftmaxSmemMax ? 2 : 1;
         const int smem = nbuf * buf_bytes + 128;  // + slack to a 128-byte boundary
         const dim3 b(512);
         // y's body takes whole words when y lies as far from a 16-byte
