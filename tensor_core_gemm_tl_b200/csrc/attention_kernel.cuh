@@ -54,6 +54,30 @@ struct AttnParams {
     uint64_t timeout_ns;
 };
 
+// Two fp32 lanes per instruction (sm_100): d = a * b + c and d = a + b, each
+// lane rounded as its scalar form.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    uint64_t d;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\tmov.b64 rc, {%5, %6};\n\t"
+        "fma.rn.f32x2 %0, ra, rb, rc;\n\t}"
+        : "=l"(d)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return make_float2(__uint_as_float(static_cast<uint32_t>(d)), __uint_as_float(static_cast<uint32_t>(d >> 32)));
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
+{
+    uint64_t d;
+    asm("{\n\t.reg .b64 ra, rb;\n\t"
+        "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\t"
+        "add.rn.f32x2 %0, ra, rb;\n\t}"
+        : "=l"(d)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return make_float2(__uint_as_float(static_cast<uint32_t>(d)), __uint_as_float(static_cast<uint32_t>(d >> 32)));
+}
+
 template <int D_>
 struct AttnConfig {
     static constexpr int D = D_;
@@ -419,21 +443,27 @@ __global__ void __launch_bounds__(384, 1)
                     break;
                 tc_fence_after_sync();
             }
-            float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            // keys in pairs: the exponent argument and the running sums two
+            // lanes per instruction
+            const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
+            const float2 negm2 = make_float2(-m_ref, -m_ref);
+            float2 part[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                              make_float2(0.0f, 0.0f)};
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int e2 = 0; e2 < 32; ++e2) {
                     const int e = 64 * h + 2 * e2;
-                    const float w0 = exp2_approx_ftz(fmaf(__uint_as_float(sv[e]), p.scale_log2, -m_ref));
-                    const float w1 = exp2_approx_ftz(fmaf(__uint_as_float(sv[e + 1]), p.scale_log2, -m_ref));
-                    part[e2 & 3] += w0 + w1;
-                    pk[e2] = pack2<DT>(w0, w1);  // keys 2 e2, 2 e2 + 1 of this half: one 32-bit column
+                    const float2 x = ffma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), scale2, negm2);
+                    const float2 w = make_float2(exp2_approx_ftz(x.x), exp2_approx_ftz(x.y));
+                    part[e2 & 3] = fadd2(part[e2 & 3], w);
+                    pk[e2] = pack2<DT>(w.x, w.y);  // keys 2 e2, 2 e2 + 1 of this half: one 32-bit column
                 }
                 tmem_store_32cols(p_addr + 32 * h, pk);
             }
-            l = l * alpha + ((part[0] + part[1]) + (part[2] + part[3]));
+            const float2 ps = fadd2(fadd2(part[0], part[1]), fadd2(part[2], part[3]));
+            l = l * alpha + (ps.x + ps.y);
             m = m_new;
             // the rows whose maximum moved take O_i down by alpha (O_i holds
             // blocks 0 .. j-1, so PV_i(j - 1) has to be complete)
