@@ -205,7 +205,12 @@ typedef struct {
     int32_t inject_fault; /* test hook, 0 in production: 1 makes the copy warp
                              skip its first stage without issuing the copy, so
                              the consumer's bounded wait runs out and the kernel
-                             returns with TL_ERR_DEVICE_TIMEOUT recorded          */
+                             returns with TL_ERR_DEVICE_TIMEOUT recorded; 2 makes
+                             the host treat the encoding of A's tensor map as
+                             failed: the call returns TL_ERR_CUDA and the GEMM
+                             kernel is not launched (padding copies the shape
+                             needs may already be enqueued; their temporary is
+                             released on the stream)                             */
     uint64_t timeout_ns;  /* bound on every wait inside the kernel; 0 = 10 s     */
     int32_t no_split;     /* 1: never split the tiles of a short last round      */
     int32_t b_layout;     /* 0: B is K x N row-major (leading dimension N);
@@ -233,7 +238,8 @@ TL_API tl_status tl_gemm_ex(const void *A, const void *B, const void *bias, void
  * gave up: bit 0 copy warp, bit 1 MMA warp on data, bit 2 MMA warp on the
  * accumulator, bit 3 epilogue warps, bit 4 final drain, bit 5 the last K part
  * of a split tile waiting for an earlier part, bit 6 the row softmax waiting
- * for a row's copy into shared memory).
+ * for a row's copy into shared memory, bit 7 -- in the checked build
+ * libtlgemm_checked.so only -- an index invariant of the GEMM kernel failed).
  */
 TL_API tl_status tl_check_device(tl_stream stream, uint32_t *detail);
 

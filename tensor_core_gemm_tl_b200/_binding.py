@@ -37,7 +37,7 @@ class TLError(RuntimeError):
 
 class Options(ctypes.Structure):
     """tl_gemm_options: config (0 = library's choice, k = configuration k-1),
-    inject_fault (test hook), timeout_ns (0 = 10 s), no_split (1 = never split
+    inject_fault (test hook: 1 device-side stall, 2 host-side encode failure), timeout_ns (0 = 10 s), no_split (1 = never split
     the tiles of a short last round), b_layout (1 = B given as N x K),
     c_float32 (1 = C is float32)."""
     _fields_ = [("config", ctypes.c_int32), ("inject_fault", ctypes.c_int32),

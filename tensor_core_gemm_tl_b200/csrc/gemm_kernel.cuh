@@ -47,7 +47,27 @@ enum : unsigned {
     ERR_EPILOGUE = 8u,
     ERR_DRAIN = 16u,
     ERR_SPLIT = 32u,   // the last part of a split tile gave up waiting for an earlier part
+    ERR_CHECK = 128u,  // checked build only: an index invariant failed (the access was skipped)
 };
+
+// The checked build (compiled with -DTL_CHECKED, libtlgemm_checked.so) tests
+// the kernel's index invariants at run time: a violation sets ERR_CHECK in the
+// device error word and the access it guards is skipped, never a trap.  In
+// the product build check_ok() is the constant true and costs nothing.
+#ifdef TL_CHECKED
+constexpr bool kCheckedBuild = true;
+#else
+constexpr bool kCheckedBuild = false;
+#endif
+
+__device__ __forceinline__ bool check_ok(bool cond)
+{
+    if (kCheckedBuild && !cond) {
+        atomicOr(&g_device_error, ERR_CHECK);
+        return false;
+    }
+    return true;
+}
 
 struct GemmParams {
     int32_t M, N, K;
@@ -69,6 +89,7 @@ struct GemmParams {
     // with `epoch`; the last part adds them, in part order, to its own sum and
     // runs the epilogue.
     int32_t full_tiles, split, num_items;
+    int32_t num_slabs;       // 128-row fp32 partial slabs the workspace holds
     float *partials;
     unsigned long long *flags;
     unsigned long long epoch;  // unique per launch
@@ -396,6 +417,8 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                 const WorkItem w = work_item(item, p);
                 int tm, tn;
                 tile_coords(w.tile, p, tm, tn);
+                check_ok(w.tile < p.num_tiles && w.part < p.split && w.kb0 <= w.kb1 && w.kb1 <= p.num_kb &&
+                         tm < p.tiles_m && tn < p.tiles_n);  // TMA clips anything outside: record only
                 const int a_row = tm * CF::TILE_M + static_cast<int>(rank) * CF::BM;
                 const int b_col = tn * CF::BN + static_cast<int>(rank) * CF::BN_LOCAL;
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
@@ -532,6 +555,7 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
             const WorkItem w = work_item(item, p);
             int tm, tn;
             tile_coords(w.tile, p, tm, tn);
+            check_ok(w.tile < p.num_tiles && w.part < p.split && tm < p.tiles_m && tn < p.tiles_n);
             const int n0 = tn * CF::BN;
             const bool split_tile = w.tile >= p.full_tiles;
             const int r_tail = w.tile - p.full_tiles;
@@ -555,6 +579,8 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
 #pragma unroll 1
             for (int c = half; c < CHUNKS; c += 2) {
                 uint32_t r[64];
+                if (!check_ok(acc * CF::ACC_COLS + c * 64 + 64 <= CF::TMEM_COLS))
+                    continue;  // outside this CTA's Tensor Memory
                 const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(acc * CF::ACC_COLS + c * 64);
                 tmem_load_32cols(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
                 tmem_load_32cols(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
@@ -572,6 +598,8 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                     const size_t slab_step = CF::CTAS;  // from part to part + 1
                     const size_t row_off = (static_cast<size_t>(q) * 32 + lane) * CF::BN + c * 64;
                     const size_t flag_off = static_cast<size_t>(q) * CHUNKS + c;
+                    if (!check_ok(slab0 + (p.split - 2) * slab_step < static_cast<size_t>(p.num_slabs)))
+                        continue;  // outside the workspace
                     if (w.part < p.split - 1) {
                         const size_t slab = slab0 + w.part * slab_step;
                         float4 *dst = reinterpret_cast<float4 *>(p.partials + slab * CF::BM * CF::BN + row_off);

@@ -215,12 +215,12 @@ tl_status validate(const void *A, const void *B, const void *bias, void *C, int6
         return TL_ERR_INVALID_ARG;
     if (opt && (opt->config < 0 || opt->config > num_configs()))
         return TL_ERR_INVALID_ARG;
-    if (opt && (opt->inject_fault != 0 && opt->inject_fault != 1))
+    if (opt && (opt->inject_fault < 0 || opt->inject_fault > 2))
         return TL_ERR_INVALID_ARG;
     if (opt && ((opt->no_split != 0 && opt->no_split != 1) || (opt->b_layout != 0 && opt->b_layout != 1) ||
                 (opt->c_float32 != 0 && opt->c_float32 != 1)))
         return TL_ERR_INVALID_ARG;
-    if (opt && opt->inject_fault && opt->config > 0 && kConfigs[opt->config - 1].ctas != 1)
+    if (opt && opt->inject_fault == 1 && opt->config > 0 && kConfigs[opt->config - 1].ctas != 1)
         return TL_ERR_UNSUPPORTED;  // the fault hook exists for single-CTA configurations only
     const int64_t lim = 0x7FFFFFFFll;
     if (M > lim || N > lim || K > lim)
@@ -268,7 +268,7 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
         return TL_ERR_INVALID_ARG;
     bool table_split = true;  // a forced configuration splits unless told not to
     int ci = (opt && opt->config > 0) ? opt->config - 1 : choose_config(M, N, K, dtype, epi, num_sms, &table_split);
-    if (opt && opt->inject_fault && kConfigs[ci].ctas != 1)
+    if (opt && opt->inject_fault == 1 && kConfigs[ci].ctas != 1)
         ci = model_config_single(M, N, num_sms);
     const ConfigEntry &c = kConfigs[ci];
     Plan p{};
@@ -289,7 +289,7 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
     p.num_kb = static_cast<int32_t>(ceil_div(K, c.bk));
     int64_t full_tiles = tiles;
     int32_t split = 1;
-    if (table_split && !(opt && (opt->inject_fault || opt->no_split)))
+    if (table_split && !(opt && (opt->inject_fault == 1 || opt->no_split)))
         split_tail(tiles, units, p.num_kb, &split, &full_tiles);
     const int64_t items = full_tiles + (tiles - full_tiles) * split;
     q.split = split;
@@ -495,7 +495,9 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
 
     CUtensorMap ta, tb, tc;
     std::memset(&tc, 0, sizeof(tc));
-    if (!encode_2d(&ta, A, dtype, M, K, p.lda, 64, c.cta_m))
+    // test hook 2: the driver "refuses" A's tensor map, as a failing encode would
+    const bool refuse_encode = opt && opt->inject_fault == 2;
+    if (refuse_encode || !encode_2d(&ta, A, dtype, M, K, p.lda, 64, c.cta_m))
         return TL_ERR_CUDA;
     if (bt ? !encode_2d(&tb, B, dtype, N, K, p.ldb, 64, c.bn / c.ctas)   // B^T: BN/CTAS rows of 64 k
            : !encode_2d(&tb, B, dtype, K, N, p.ldb, 64, c.bk))
@@ -518,7 +520,7 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
     gp.epi_gelu = epi_gelu_form(epi);
     if (!gp.epi_bias)
         gp.bias = nullptr;
-    gp.inject_fault = opt ? opt->inject_fault : 0;
+    gp.inject_fault = (opt && opt->inject_fault == 1) ? 1 : 0;
     gp.C = static_cast<uint16_t *>(C);
     gp.C32 = store == STORE_F32 ? static_cast<float *>(C) : nullptr;
     gp.c32_vec16 = store == STORE_F32 && aligned(C, 16) && N % 4 == 0;
@@ -527,6 +529,7 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
     gp.split = p.pub.split;
     gp.full_tiles = p.pub.full_tiles;
     gp.num_items = p.pub.full_tiles + (gp.num_tiles - p.pub.full_tiles) * p.pub.split;
+    gp.num_slabs = (gp.num_tiles - p.pub.full_tiles) * (p.pub.split - 1) * c.ctas;
     gp.partials = nullptr;
     gp.flags = nullptr;
     gp.epoch = 0;

@@ -194,6 +194,14 @@ def test_plan_splits_only_a_short_last_round(M, N, K, config, split, full):
         assert p["workspace_bytes"] == 0 or p["pad_a"] or p["pad_b"]
 
 
+def test_host_fault_hook_is_valid_and_changes_no_plan():
+    # 2: the host-side hook (a refused tensor-map encode) plans like a normal call
+    st, p = tg.tl_gemm_plan(P, P, 0, P, 4096, 4096, 4096, 0, 0, 148, tg.Options(inject_fault=2))
+    st0, p0 = tg.tl_gemm_plan(P, P, 0, P, 4096, 4096, 4096, 0, 0, 148)
+    assert st == 0 and st0 == 0 and p.config == p0.config and p.split == p0.split and p.grid == p0.grid
+    assert tg.tl_gemm_ex(P, P, 0, P, 8, 8, 8, 0, 0, 0, tg.Options(inject_fault=-1)) == tg.Status.INVALID_ARG
+
+
 def test_fault_hook_disables_the_split():
     st, p = tg.tl_gemm_plan(P, P, 0, P, 1024, 1024, 2048, 0, 0, 148, tg.Options(config=1, inject_fault=1))
     assert st == 0 and p.split == 1

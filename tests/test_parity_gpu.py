@@ -310,3 +310,24 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     C = run_library(A, B, None, wl.F16, 0)
     ref = oracle.gemm(A, B, None, wl.F16, 0)
     compare(C, ref, wl.F16, accumulation_bound(A, B, None, wl.F16, 0, ref))
+
+
+def test_host_side_encode_failure_is_reported_and_nothing_runs():
+    """The host treats A's tensor-map encode as failed (test hook 2): the call
+    returns TL_ERR_CUDA before any kernel is launched, C is untouched, no device
+    error is recorded, and the next call on the same context is right."""
+    import tensor_core_gemm_tl_b200 as m
+    M, N, K = 256, 384, 320
+    A, B, bias = inputs(M, N, K, wl.BF16, wl.EPI_BIAS_GELU, seed=9)
+    dA, dB, dbias = to_device(A, wl.BF16), to_device(B, wl.BF16), to_device(bias, wl.BF16)
+    out = torch.full((M, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    st = m.tl_gemm_ex(dA.data_ptr(), dB.data_ptr(), dbias.data_ptr(), out.data_ptr(), M, N, K, wl.BF16,
+                      wl.EPI_BIAS_GELU, stream, m.Options(inject_fault=2))
+    assert st == int(m.Status.CUDA)
+    st, word = m.tl_check_device(stream)
+    assert st == 0 and word == 0
+    assert bool(torch.all(out == 7.0))
+    C = run_library(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU)
+    ref = oracle.gemm(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU)
+    compare(C, ref, wl.BF16, accumulation_bound(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU, ref))
