@@ -14,10 +14,13 @@
  *     optionally add a per-column bias and apply GELU to the float32
  *     accumulator before the single write of C, so no intermediate reaches
  *     global memory.  GELU is the exact form x * Phi(x) =
- *     0.5 x (1 + erf(x / sqrt 2)).
+ *     0.5 x (1 + erf(x / sqrt 2)), or on request its tanh form (see
+ *     tl_epilogue).
  *
  * The result is rounded once, to nearest even, from float32 to the input
- * dtype.  Sums are accumulated in float32 on the tensor cores; the order of
+ * dtype (or kept as float32 with tl_gemm_ex's c_float32 option).  The library
+ * also holds the tutorial's adjacent kernels: tl_attention_fwd,
+ * tl_softmax_rows and tl_vector_add.  Sums are accumulated in float32 on the tensor cores; the order of
  * the sum is fixed by the kernel configuration, so two calls with the same
  * configuration give bit-identical results.
  *

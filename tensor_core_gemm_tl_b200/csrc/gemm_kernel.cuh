@@ -1,5 +1,6 @@
 // gemm_kernel.cuh -- persistent, warp-specialised sm_100a GEMM with a fused
-// bias + exact-GELU epilogue:  C = epilogue(A . B).
+// epilogue:  C = epilogue(A . B), epilogue = optional per-column bias, then
+// optional GELU (exact erf form or tanh form); C 16-bit or float32.
 //
 // What it computes follows "Designing High-Performance GPU Kernels with
 // TileLang" (blog retelling), Step 4 (tiled Tensor-Core GEMM: A tiles
@@ -14,6 +15,8 @@
 //          --tcgen05.mma (one thread)--> fp32 accumulator in Tensor Memory
 //          --tcgen05.ld--> registers: + bias, GELU, round once to fp16/bf16
 //          --st.shared (swizzled)--> TMA store --> global
+// (element stores when C's rows are not 16-byte aligned; with float32 C the
+// fp32 values go straight out in 16-byte stores)
 //
 // Warp roles (320 threads, one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer (one lane)

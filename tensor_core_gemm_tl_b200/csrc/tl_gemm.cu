@@ -1,6 +1,8 @@
-// tl_gemm.cu -- host side of libtlgemm.so: argument validation, the launch
-// plan (kernel configuration, padding, store path), tensor-map encoding and
-// the launches.  The C ABI is declared in include/tl_gemm.h.
+// tl_gemm.cu -- host side of libtlgemm.so: for the GEMM, argument
+// validation, the launch plan (kernel configuration, padding, store path),
+// tensor-map encoding and the launches; the same for the attention forward,
+// the row softmax and the vector add; the device error word's read-out.  The
+// C ABI is declared in include/tl_gemm.h.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
