@@ -281,29 +281,33 @@ __device__ __forceinline__ float to_float(uint16_t bits)
 // avoids the cancellation of 1 + erf(x / sqrt 2) for negative x.  Relative
 // error below 3e-6 for |x| <= 9 (below 1e-5 everywhere; one fp16 ulp is 5e-4,
 // one bf16 ulp 4e-3); NaN stays NaN.
-__device__ __forceinline__ float gelu_erf(float x)
+// Both GELU forms run on pairs of values: their multiply-adds take two lanes
+// per instruction (fma/mul/add .f32x2, each lane rounded as its scalar step).
+__device__ __forceinline__ float2 gelu_erf2(float2 x)
 {
-    constexpr float P_SQRT1_2 = 0.415f * 0.70710678118654752f;  // p / sqrt 2: t = 1 / (1 + p' |x|)
+    constexpr float P_SQRT1_2 = 0.415f * 0.70710678118654752f;
     constexpr float C0 = 4.281122892280109e-05f, C1 = 0.23316948115825653f, C2 = 0.24358120560646057f,
                     C3 = 0.1621198058128357f, C4 = 0.34987202286720276f, C5 = -0.2624722123146057f,
                     C6 = 0.5700822472572327f, C7 = -0.3758394122123718f, C8 = 0.079444020986557f;
-    constexpr float NEG_HALF_LOG2E = -0.72134752044448170f;  // -log2(e) / 2
-    // beyond |x| = 20, Phi is exactly 0 or 1 in float32; the clamp keeps x^2 finite
-    const float a = fminf(fabsf(x), 20.0f);
-    const float t = rcp_approx(fmaf(P_SQRT1_2, a, 1.0f));
-    float h = fmaf(C8, t, C7);
-    h = fmaf(h, t, C6);
-    h = fmaf(h, t, C5);
-    h = fmaf(h, t, C4);
-    h = fmaf(h, t, C3);
-    h = fmaf(h, t, C2);
-    h = fmaf(h, t, C1);
-    h = fmaf(h, t, C0);
-    const float hi = a * a;
-    const float lo = fmaf(a, a, -hi);                                   // a^2 = hi + lo exactly
-    const float e = exp2_approx(hi * NEG_HALF_LOG2E) * fmaf(-0.5f, lo, 1.0f);  // exp(-x^2 / 2)
-    const float q = 0.5f * h * e;                                       // erfc(z) / 2
-    return x * (x >= 0.0f ? 1.0f - q : q);
+    constexpr float NEG_HALF_LOG2E = -0.72134752044448170f;
+    const float2 a = make_float2(fminf(fabsf(x.x), 20.0f), fminf(fabsf(x.y), 20.0f));
+    const float2 d = ffma2(splat2(P_SQRT1_2), a, splat2(1.0f));
+    const float2 t = make_float2(rcp_approx(d.x), rcp_approx(d.y));
+    float2 h = ffma2(splat2(C8), t, splat2(C7));
+    h = ffma2(h, t, splat2(C6));
+    h = ffma2(h, t, splat2(C5));
+    h = ffma2(h, t, splat2(C4));
+    h = ffma2(h, t, splat2(C3));
+    h = ffma2(h, t, splat2(C2));
+    h = ffma2(h, t, splat2(C1));
+    h = ffma2(h, t, splat2(C0));
+    const float2 hi = fmul2(a, a);
+    const float2 lo = ffma2(a, a, make_float2(-hi.x, -hi.y));
+    const float2 m = fmul2(hi, splat2(NEG_HALF_LOG2E));
+    const float2 e = fmul2(make_float2(exp2_approx(m.x), exp2_approx(m.y)), ffma2(splat2(-0.5f), lo, splat2(1.0f)));
+    const float2 q = fmul2(fmul2(splat2(0.5f), h), e);
+    const float2 one_q = fadd2(splat2(1.0f), make_float2(-q.x, -q.y));
+    return fmul2(x, make_float2(x.x >= 0.0f ? one_q.x : q.x, x.y >= 0.0f ? one_q.y : q.y));
 }
 
 // Tanh form of GELU (the GELU paper's approximation):
@@ -313,14 +317,17 @@ __device__ __forceinline__ float gelu_erf(float x)
 // overflows or cancels.  u has the sign of x.  Relative error about
 // 3e-7 + 1.2e-7 a (the rounding of a, carried through 2^-a): below 1e-5
 // for x >= -10, where g is 1e-37.  NaN stays NaN.
-__device__ __forceinline__ float gelu_tanh(float x)
+__device__ __forceinline__ float2 gelu_tanh2(float2 x)
 {
-    constexpr float K0 = 2.3022081983f;       // 2 sqrt(2 / pi) log2(e)
+    constexpr float K0 = 2.3022081983f;
     constexpr float K1 = 0.044715f * K0;
-    const float a = fabsf(x) * fmaf(K1, x * x, K0);
-    const float e = exp2_approx(-a);
-    const float s = rcp_approx(1.0f + e);
-    return x * (x >= 0.0f ? s : e * s);
+    const float2 inner = ffma2(splat2(K1), fmul2(x, x), splat2(K0));
+    const float2 a = fmul2(make_float2(fabsf(x.x), fabsf(x.y)), inner);
+    const float2 e = make_float2(exp2_approx(-a.x), exp2_approx(-a.y));
+    const float2 den = fadd2(splat2(1.0f), e);
+    const float2 s = make_float2(rcp_approx(den.x), rcp_approx(den.y));
+    const float2 es = fmul2(e, s);
+    return fmul2(x, make_float2(x.x >= 0.0f ? s.x : es.x, x.y >= 0.0f ? s.y : es.y));
 }
 
 // How C leaves the epilogue.
@@ -665,8 +672,11 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                                 const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
-                                    v[8 * i + 2 * e] += to_float<DT>(static_cast<uint16_t>(ww[e] & 0xFFFFu));
-                                    v[8 * i + 2 * e + 1] += to_float<DT>(static_cast<uint16_t>(ww[e] >> 16));
+                                    const float2 sum2 = fadd2(make_float2(v[8 * i + 2 * e], v[8 * i + 2 * e + 1]),
+                                                              make_float2(to_float<DT>(static_cast<uint16_t>(ww[e] & 0xFFFFu)),
+                                                                          to_float<DT>(static_cast<uint16_t>(ww[e] >> 16))));
+                                    v[8 * i + 2 * e] = sum2.x;
+                                    v[8 * i + 2 * e + 1] = sum2.y;
                                 }
                             }
                         } else {
@@ -678,12 +688,18 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                       }
                       if (p.epi_gelu == 1) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            v[j] = gelu_erf(v[j]);
+                        for (int j = 0; j < 32; j += 2) {
+                            const float2 g = gelu_erf2(make_float2(v[j], v[j + 1]));
+                            v[j] = g.x;
+                            v[j + 1] = g.y;
+                        }
                       } else if (p.epi_gelu == 2) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            v[j] = gelu_tanh(v[j]);
+                        for (int j = 0; j < 32; j += 2) {
+                            const float2 g = gelu_tanh2(make_float2(v[j], v[j + 1]));
+                            v[j] = g.x;
+                            v[j + 1] = g.y;
+                        }
                       }
                     }
                     if constexpr (STORE == STORE_F32) {

@@ -19,7 +19,7 @@ KERNEL = os.path.join(ROOT, "tensor_core_gemm_tl_b200", "csrc", "gemm_kernel.cuh
 
 def kernel_constants():
     src = open(KERNEL).read()
-    body = src[src.index("__device__ __forceinline__ float gelu_erf"):]
+    body = src[src.index("__device__ __forceinline__ float2 gelu_erf2"):]
     body = body[:body.index("\n}\n")]
     m = re.search(r"constexpr float P_SQRT1_2 = ([0-9.eE+-]+)f \* ([0-9.eE+-]+)f;", body)
     p = np.float32(m.group(1)) * np.float32(m.group(2))          # folded at compile time in float
@@ -63,7 +63,7 @@ def test_kernel_gelu_formula_accuracy():
 
 def kernel_tanh_constant():
     src = open(KERNEL).read()
-    body = src[src.index("__device__ __forceinline__ float gelu_tanh"):]
+    body = src[src.index("__device__ __forceinline__ float2 gelu_tanh2"):]
     body = body[:body.index("\n}\n")]
     k0 = np.float32(re.search(r"constexpr float K0 = ([0-9.eE+-]+)f;", body).group(1))
     k1c = np.float32(re.search(r"constexpr float K1 = ([0-9.eE+-]+)f \* K0;", body).group(1))
