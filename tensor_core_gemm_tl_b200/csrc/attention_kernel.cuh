@@ -354,6 +354,10 @@ __global__ void __launch_bounds__(384, 1)
         const int r = q * 32 + lane;                  // row of the tile (TMEM lane)
         const int row = q0 + tile * CF::BM + r;       // query index
         const int nb = nbt(tile);
+        // checked build: this tile's Tensor Memory columns (S, P, O) inside the
+        // 512 allocated, its key blocks inside K
+        check_ok(CF::TMEM_S + tile * 128 + 128 <= 512 && CF::p_col(tile) + 64 <= 512 &&
+                 CF::TMEM_O + tile * D + D <= 512 && nb <= kblocks_all && bh < p.BH);
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const uint32_t s_addr = tmem_base + lane_base + static_cast<uint32_t>(CF::TMEM_S + tile * 128);
         const uint32_t p_addr =
@@ -476,7 +480,7 @@ __global__ void __launch_bounds__(384, 1)
                 uint32_t o[32];
                 tmem_load_32cols(o_addr + 32 * c, o);
                 tmem_load_wait();
-                if (row < p.Sq) {
+                if (row < p.Sq && check_ok(static_cast<size_t>(bh) * p.Sq + row < static_cast<size_t>(p.BH) * p.Sq)) {
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         uint4 w;

@@ -311,6 +311,13 @@ __global__ void __launch_bounds__(512) softmax_rows_smem_kernel(const uint16_t *
         const uint32_t bytes = static_cast<uint32_t>(sp.nvec) * 16u;
         const uint32_t dst = smem_addr(srow_raw + buf * buf_bytes + sp.mis + 2 * sp.head);
         const uint8_t *src = reinterpret_cast<const uint8_t *>(x + sp.head);
+        // checked build: the copy stays inside its row buffer, starts and ends on
+        // 16-byte boundaries, and reads inside the row
+        if (!check_ok(buf < nbuf && sp.mis + 2 * sp.head + static_cast<int>(bytes) <= buf_bytes && (dst & 15u) == 0 &&
+                      (reinterpret_cast<uintptr_t>(src) & 15u) == 0 && sp.head + 8 * sp.nvec <= cols)) {
+            mbar_arrive(bar);  // complete the phase without the copy
+            return;
+        }
         fence_proxy_async_smem();  // earlier generic reads of this buffer come first
         mbar_arrive_expect_tx(bar, bytes);
         constexpr uint32_t CHUNK = 32768;

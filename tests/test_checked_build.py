@@ -1,11 +1,14 @@
 """The checked build, libtlgemm_checked.so: the same sources compiled with
--DTL_CHECKED, whose GEMM kernel tests its index invariants at run time (work
-items, tile coordinates, Tensor Memory columns, split-tile workspace slabs)
-and sets bit 7 of the device error word on a violation instead of trapping.
+-DTL_CHECKED, whose kernels test their index invariants at run time (GEMM:
+work items, tile coordinates, Tensor Memory columns, split-tile workspace
+slabs; attention: Tensor Memory columns, key blocks, output rows; row
+softmax: every bulk copy inside its row buffer and its row, 16-byte aligned)
+and set bit 7 of the device error word on a violation instead of trapping.
 On the CPU: it loads and exports the ABI.  On the GPU: parity cases covering
 every configuration, split tiles, padding, element stores, B given
-transposed and float32 C run through it against the oracle with no check
-firing."""
+transposed and float32 C, attention of both head sizes and masks, and row
+softmax through every kernel kind run through it against the oracle with no
+check firing."""
 import ctypes
 import os
 import re
@@ -89,3 +92,53 @@ def test_checked_kernel_no_invariant_fires(M, N, K, config, dt, epi, bt, f32):
         compare_f32(out.cpu().numpy(), ref, accumulation_bound(A, B, bias, dt, epi, ref, out_f32=True))
     else:
         compare(from_device(out), ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("D,causal,Sq,Sk", [(64, False, 300, 500), (128, True, 333, 333), (128, False, 1024, 4096)])
+def test_checked_attention_no_invariant_fires(D, causal, Sq, Sk):
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from gpu_util import from_device, to_device
+    lib = checked_lib()
+    dt, B, H = wl.BF16, 1, 2
+    rng = np.random.default_rng(D + Sq)
+    Q, K, V = (wl.round_to_bits(rng.normal(size=(B, H, s, D)).astype(np.float32), dt) for s in (Sq, Sk, Sk))
+    q, k, v = to_device(Q, dt), to_device(K, dt), to_device(V, dt)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream().cuda_stream
+    scale = 1.0 / np.sqrt(D)
+    st = lib.tl_attention_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), None, B, H, Sq, Sk, D,
+                              dt, int(causal), ctypes.c_float(scale), stream or None)
+    assert st == 0
+    word = ctypes.c_uint32(0)
+    assert lib.tl_check_device(stream or None, ctypes.byref(word)) == 0, word.value
+    assert not (word.value & ERR_CHECK)
+    ref, _ = oracle.attention(Q, K, V, dt, causal, scale)
+    got = wl.bits_to_float32(from_device(out), dt).astype(np.float64)
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 1e-2
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("rows,cols,offset", [(64, 8192, 0), (37, 3000, 1), (9, 50257, 0), (5, 112000, 3)])
+def test_checked_softmax_no_invariant_fires(rows, cols, offset):
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from gpu_util import from_device, to_device, ulp
+    lib = checked_lib()
+    dt = wl.BF16
+    rng = np.random.default_rng(cols)
+    X = wl.round_to_bits(rng.normal(size=(rows, cols)).astype(np.float32), dt)
+    x = to_device(X, dt, offset)
+    buf = torch.empty(x.numel() + offset, dtype=x.dtype, device="cuda")
+    y = buf[offset:].view(x.shape)
+    stream = torch.cuda.current_stream().cuda_stream
+    assert lib.tl_softmax_rows(x.data_ptr(), y.data_ptr(), rows, cols, dt, stream or None) == 0
+    word = ctypes.c_uint32(0)
+    assert lib.tl_check_device(stream or None, ctypes.byref(word)) == 0, word.value
+    assert not (word.value & ERR_CHECK)
+    ref = oracle.softmax_rows(X, dt)
+    got = wl.bits_to_float32(from_device(y), dt).astype(np.float64)
+    assert np.all(np.abs(got - ref) <= 0.5 * ulp(ref, dt) + 1e-5 * ref + np.where(ref < 2.0 ** -126, ref, 0) + 1e-40)
