@@ -165,7 +165,8 @@ TL_API tl_status tl_gemm_noalloc(const void *A, const void *B, const void *bias,
  *   O    device pointer, [batch][heads][seq_q][head_dim], `dtype`; written
  *   lse  device pointer to batch*heads*seq_q floats, or NULL; written
  *   head_dim        64 or 128
- *   batch * heads   at most 65535
+ *   batch * heads   at most 65535 (non-causal) or 2^31 - 1 (causal);
+ *   seq_q           at most 65535 * 256 when causal
  *   softmax_scale   > 0, or 0 for 1 / sqrt(head_dim)
  *
  * The products run on 16-bit inputs with fp32 accumulation; the softmax

@@ -108,10 +108,13 @@ __global__ void __launch_bounds__(384, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // CTA pairs of query tiles; heaviest first when causal
+    // CTA pairs of query tiles.  Non-causal: pairs along x, so the CTAs that
+    // start together share a head's K and V in L2.  Causal: heads along x and
+    // the pairs reversed along y, so every head's heaviest pair starts first.
     const int num_pairs = (p.num_qtiles + 1) / 2;
-    const int qp = p.causal ? num_pairs - 1 - static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x);
-    const int bh = static_cast<int>(blockIdx.y);
+    const int pair_idx = static_cast<int>(p.causal ? blockIdx.y : blockIdx.x);
+    const int qp = p.causal ? num_pairs - 1 - pair_idx : pair_idx;
+    const int bh = static_cast<int>(p.causal ? blockIdx.x : blockIdx.y);
     const int q0 = qp * 2 * CF::BM;  // first query row of tile 0
     const int kblocks_all = (p.Sk + CF::BN - 1) / CF::BN;
     // key blocks each tile visits (a tile past the end of the queries visits none)

@@ -691,7 +691,7 @@ bool encode_3d_rows(CUtensorMap *map, const void *base, int dtype, int64_t BH, i
 }
 
 tl_status attention_validate(const void *Q, const void *K, const void *V, void *O, const float *lse, int64_t batch,
-                             int64_t heads, int64_t seq_q, int64_t seq_k, int64_t head_dim, int dtype,
+                             int64_t heads, int64_t seq_q, int64_t seq_k, int64_t head_dim, int dtype, int causal,
                              float softmax_scale)
 {
     if (!Q || !K || !V || !O)
@@ -704,7 +704,10 @@ tl_status attention_validate(const void *Q, const void *K, const void *V, void *
         return TL_ERR_INVALID_ARG;
     if (!(softmax_scale >= 0.0f) || softmax_scale == INFINITY)
         return TL_ERR_INVALID_ARG;
-    if (batch * heads > 65535 || seq_q > 0x7FFFFFFFll || seq_k > 0x7FFFFFFFll)
+    // the grid is (pairs of 128-row query tiles, batch * heads), transposed when causal
+    const int64_t grid_y = causal ? ceil_div(seq_q, 256) : batch * heads;
+    const int64_t grid_x = causal ? batch * heads : ceil_div(seq_q, 256);
+    if (grid_y > 65535 || grid_x > 0x7FFFFFFFll || batch * heads > 0x7FFFFFFFll || seq_k > 0x7FFFFFFFll)
         return TL_ERR_UNSUPPORTED;
     if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || (lse && !aligned(lse, 4)))
         return TL_ERR_MISALIGNED;
@@ -715,7 +718,8 @@ tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, f
                          int64_t heads, int64_t seq_q, int64_t seq_k, int64_t head_dim, int dtype, int causal,
                          float softmax_scale, cudaStream_t stream)
 {
-    tl_status st = attention_validate(Q, K, V, O, lse, batch, heads, seq_q, seq_k, head_dim, dtype, softmax_scale);
+    tl_status st =
+        attention_validate(Q, K, V, O, lse, batch, heads, seq_q, seq_k, head_dim, dtype, causal, softmax_scale);
     if (st != TL_OK)
         return st;
     DeviceState *d = nullptr;
@@ -755,7 +759,12 @@ tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, f
 
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];
-    cfg.gridDim = dim3(static_cast<unsigned>(ceil_div(ap.num_qtiles, e.tiles_per_cta)), static_cast<unsigned>(BH), 1);
+    // blocks start x fastest.  Non-causal: query-tile pairs along x (the CTAs
+    // running together share a head's K and V in L2).  Causal: heads along x,
+    // pairs along y reversed in the kernel, so every head's heaviest pair
+    // starts before any lighter one.
+    const unsigned pairs = static_cast<unsigned>(ceil_div(ap.num_qtiles, e.tiles_per_cta));
+    cfg.gridDim = causal ? dim3(static_cast<unsigned>(BH), pairs, 1) : dim3(pairs, static_cast<unsigned>(BH), 1);
     cfg.blockDim = dim3(static_cast<unsigned>(e.threads), 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(e.smem_bytes);
     cfg.stream = stream;

@@ -250,7 +250,7 @@ def test_plan_transposed_b_pads_on_k():
     (dict(dtype=5), tg.Status.INVALID_ARG),
     (dict(scale=-1.0), tg.Status.INVALID_ARG),
     (dict(scale=float("nan")), tg.Status.INVALID_ARG),
-    (dict(batch=256, heads=256), tg.Status.UNSUPPORTED),
+    (dict(batch=256, heads=256), tg.Status.UNSUPPORTED),   # non-causal: batch * heads beyond 65535
     (dict(K=P + 2), tg.Status.MISALIGNED),
     (dict(lse=P + 2), tg.Status.MISALIGNED),
 ])
@@ -260,6 +260,16 @@ def test_attention_validation_before_any_cuda_call(args, status):
     st = tg.tl_attention_fwd(a["Q"], a["K"], a["V"], a["O"], a["lse"], a["batch"], a["heads"], a["seq_q"],
                              a["seq_k"], a["head_dim"], a["dtype"], False, a["scale"], 0)
     assert st == status
+
+
+def test_attention_causal_grid_limits():
+    # causal launches put batch * heads along x (up to 2^31 - 1) and the
+    # query-tile pairs along y (up to 65535)
+    def st(batch, heads, seq_q):
+        return tg.tl_attention_fwd(P, P, P, P, 0, batch, heads, seq_q, 64, 64, 0, True, 0.0, 0)
+    assert st(1 << 16, 1 << 15, 64) == tg.Status.UNSUPPORTED
+    assert st(1, 2, 65536 * 256) == tg.Status.UNSUPPORTED
+    assert st(256, 256, 64) != tg.Status.UNSUPPORTED  # fine when causal (fails later only for want of a GPU)
 
 
 def test_softmax_and_vector_add_validation():
