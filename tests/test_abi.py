@@ -281,3 +281,42 @@ def test_softmax_and_vector_add_validation():
     assert tg.tl_vector_add(P, 0, P, 4, 0) == tg.Status.INVALID_ARG
     assert tg.tl_vector_add(P, P, P, 0, 0) == tg.Status.INVALID_ARG
     assert tg.tl_vector_add(P + 2, P, P, 4, 0) == tg.Status.MISALIGNED
+
+
+def test_plan_is_total_and_consistent_for_any_shape():
+    """Every shape gets a configuration, and the plan is self-consistent: the
+    tiles cover C, the grid is at most one unit per SM (or pair) and at most
+    the work items, a split only cuts the last round, the shared memory fits
+    and the workspace holds the padded copies (property test over random
+    shapes, dtypes, epilogues and layouts)."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=400, deadline=None)
+    @given(M=st.integers(1, 70000), N=st.integers(1, 70000), K=st.integers(1, 70000),
+           dtype=st.sampled_from([0, 1]), epi=st.integers(0, 5), bt=st.booleans(), f32=st.booleans(),
+           sms=st.sampled_from([148, 132, 8]))
+    def check(M, N, K, dtype, epi, bt, f32, sms):
+        bias = P if epi in (1, 2, 4) else 0
+        opt = tg.Options(b_layout=int(bt), c_float32=int(f32))
+        s, p = tg.tl_gemm_plan(P, P, bias, P, M, N, K, dtype, epi, sms, opt)
+        assert s == 0, (M, N, K, s)
+        assert 0 <= p.config < tg.tl_num_configs()
+        assert p.tiles_m * p.block_m >= M and (p.tiles_m - 1) * p.block_m < M
+        assert p.tiles_n * p.block_n >= N and (p.tiles_n - 1) * p.block_n < N
+        tiles = p.tiles_m * p.tiles_n
+        units = sms // p.cluster_ctas
+        items = p.full_tiles + (tiles - p.full_tiles) * p.split
+        assert 1 <= p.grid // p.cluster_ctas <= min(units, items) and p.grid % p.cluster_ctas == 0
+        assert p.split >= 1 and (p.split == 1) == (p.full_tiles == tiles)
+        assert p.split == 1 or tiles - p.full_tiles < units  # only the short last round is split
+        assert p.smem_bytes <= 232448
+        assert bool(p.direct_store) == (f32 or N % 8 != 0)  # base pointers here are 256-byte aligned
+        need = 0
+        if p.pad_a:
+            need += M * ((K + 7) // 8 * 8) * 2
+        if p.pad_b:
+            rows, cols = (N, K) if bt else (K, N)
+            need += rows * ((cols + 7) // 8 * 8) * 2
+        assert p.workspace_bytes >= need
+
+    check()
