@@ -379,10 +379,20 @@ __global__ void __launch_bounds__(384, 1)
             if (!(ok = wait_warp(CF::BAR_SF + tile, jp)))
                 break;
             tc_fence_after_sync();
+            // S in two waves of 64 columns: the maximum of the first runs while
+            // the second is still arriving
             uint32_t sv[128];
+            tmem_load_32cols(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_load_32cols(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+            tmem_load_wait();
+            tmem_load_32cols(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+            tmem_load_32cols(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+            float t[16];  // maxima of groups of 8 raw scores
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                tmem_load_32cols(s_addr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * c]));
+            for (int g = 0; g < 8; ++g) {
+                const float *f = reinterpret_cast<const float *>(&sv[8 * g]);
+                t[g] = fmax3(fmax3(f[0], f[1], f[2]), fmax3(f[3], f[4], f[5]), fmaxf(f[6], f[7]));
+            }
             tmem_load_wait();
             if constexpr (CF::SEPARATE_P) {
                 // S_i(j) is in registers: its columns may take S_i(j + 1)
@@ -396,16 +406,21 @@ __global__ void __launch_bounds__(384, 1)
             if (p.causal)
                 nvalid = min(nvalid, row + 1 - key0);
             if (!__all_sync(0xffffffffu, nvalid >= CF::BN)) {
+                // masked keys count neither in the maximum nor in the weights
 #pragma unroll
                 for (int e = 0; e < 128; ++e)
                     if (e >= nvalid)
                         sv[e] = __float_as_uint(-INFINITY);
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const float *f = reinterpret_cast<const float *>(&sv[8 * g]);
+                    t[g] = fmax3(fmax3(f[0], f[1], f[2]), fmax3(f[3], f[4], f[5]), fmaxf(f[6], f[7]));
+                }
             }
             float mx;
             {
-                float t[16];
 #pragma unroll
-                for (int g = 0; g < 16; ++g) {
+                for (int g = 8; g < 16; ++g) {
                     const float *f = reinterpret_cast<const float *>(&sv[8 * g]);
                     t[g] = fmax3(fmax3(f[0], f[1], f[2]), fmax3(f[3], f[4], f[5]), fmaxf(f[6], f[7]));
                 }
