@@ -83,6 +83,8 @@ SHAPES = [
     (257, 8, 16),
     (8, 257, 129),
     (1000, 24, 8),
+    (70001, 24, 72),     # many tile rows, one ragged tile column
+    (8, 70001, 40),      # one ragged tile row, many tile columns
 ]
 
 
