@@ -813,8 +813,9 @@ tl_status softmax_impl(const void *X, void *Y, int64_t rows, int64_t cols, int d
     uint16_t *y = static_cast<uint16_t *>(Y);
     const int c = static_cast<int>(cols);
     if (cols <= 1024) {
-        // lanes per row: short rows share a warp
-        const int lpr = cols <= 64 ? 8 : cols <= 128 ? 16 : 32;
+        // lanes per row: short rows share a warp (rows of up to 128 values take
+        // 8 lanes, 16 values each)
+        const int lpr = cols <= 128 ? 8 : 32;
         const int64_t work = ceil_div(rows, 8 * (32 / lpr));
         const dim3 b(256);
 #define TL_SOFTMAX_WARP_LAUNCH(DT, P, V, L)                                                          \
@@ -828,7 +829,7 @@ tl_status softmax_impl(const void *X, void *Y, int64_t rows, int64_t cols, int d
         if (cols <= 64)                                                                              \
             TL_SOFTMAX_WARP_LAUNCH(DT, 8, V, 8);                                                     \
         else if (cols <= 128)                                                                        \
-            TL_SOFTMAX_WARP_LAUNCH(DT, 8, V, 16);                                                    \
+            TL_SOFTMAX_WARP_LAUNCH(DT, 16, V, 8);                                                    \
         else if (cols <= 256)                                                                        \
             TL_SOFTMAX_WARP_LAUNCH(DT, 8, V, 32);                                                    \
         else                                                                                         \
