@@ -4,6 +4,7 @@ declares, validates arguments before touching a GPU, and plans launches
 import os
 import re
 
+import numpy as np
 import pytest
 
 import tensor_core_gemm_tl_b200 as tg
@@ -320,3 +321,25 @@ def test_plan_is_total_and_consistent_for_any_shape():
         assert p.workspace_bytes >= need
 
     check()
+
+
+def test_plan_from_many_threads_matches_one_thread():
+    """The planner called from eight threads at once (ctypes releases the GIL
+    for each call) returns, for every shape, the plan one thread computes."""
+    from concurrent.futures import ThreadPoolExecutor
+    rng = np.random.default_rng(5)
+    cases = [(int(M), int(N), int(K), int(dt), int(epi))
+             for M, N, K, dt, epi in zip(rng.integers(1, 70000, 600), rng.integers(1, 70000, 600),
+                                         rng.integers(1, 70000, 600), rng.integers(0, 2, 600),
+                                         rng.integers(0, 6, 600))]
+
+    def one(case):
+        M, N, K, dt, epi = case
+        st, p = tg.tl_gemm_plan(P, P, P if epi in (1, 2, 4) else 0, P, M, N, K, dt, epi, 148, None)
+        assert st == 0
+        return tuple(sorted(p.as_dict().items()))
+
+    expected = [one(c) for c in cases]
+    with ThreadPoolExecutor(max_workers=8) as pool:
+        for _ in range(3):
+            assert list(pool.map(one, cases)) == expected
