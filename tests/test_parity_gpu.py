@@ -333,3 +333,56 @@ def test_host_side_encode_failure_is_reported_and_nothing_runs():
     C = run_library(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU)
     ref = oracle.gemm(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU)
     compare(C, ref, wl.BF16, accumulation_bound(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU, ref))
+
+
+# ------------------------------------------------------------------ concurrent callers
+def test_concurrent_calls_from_threads_on_their_own_streams():
+    """Eight threads call the library at once, each on a stream of its own
+    (ctypes releases the GIL for every call): GEMMs that take the padded-copy
+    path and the split last round (both with workspace from the stream-ordered
+    pool) and the plain path, attention and row softmax.  Every output equals,
+    bit for bit, the same call made alone beforehand on one thread."""
+    from concurrent.futures import ThreadPoolExecutor
+    t = tg()
+    assert t.plan(16384, 1024, 8192, dtype=1)["split"] > 1 and t.plan(4000, 3000, 2050, dtype=1)["pad_a"]
+    g = torch.Generator(device="cuda").manual_seed(7)
+
+    def rnd(*shape):
+        return torch.randn(*shape, device="cuda", generator=g).to(torch.bfloat16)
+
+    jobs = {
+        "split": (rnd(16384, 8192), rnd(8192, 1024), None, None),
+        "padded": (rnd(4000, 2050), rnd(2050, 3000), rnd(3000), "bias_gelu"),
+        "plain": (rnd(1024, 768), rnd(768, 2048), rnd(2048), "bias"),
+    }
+    qkv = [rnd(2, 4, 700, 128) for _ in range(3)]
+    xs = rnd(333, 50257)
+
+    def run(name, stream):
+        if name == "attention":
+            return t.attention(*qkv, causal=True, stream=stream)
+        if name == "softmax":
+            return t.softmax(xs, stream=stream)
+        A, B, bias, epi = jobs[name]
+        return t.gemm(A, B, bias, epilogue=epi, stream=stream)
+
+    names = list(jobs) + ["attention", "softmax"]
+    torch.cuda.synchronize()
+    alone = {n: run(n, torch.cuda.current_stream()).view(torch.int16).cpu() for n in names}
+    assert t.check_device() == 0
+
+    def worker(idx):
+        s = torch.cuda.Stream()
+        order = names[idx % len(names):] + names[:idx % len(names)]
+        with torch.cuda.stream(s):
+            outs = {n: run(n, s) for n in order for _ in range(2)}
+        s.synchronize()
+        return {n: o.view(torch.int16).cpu() for n, o in outs.items()}
+
+    with ThreadPoolExecutor(max_workers=8) as pool:
+        results = list(pool.map(worker, range(8)))
+    torch.cuda.synchronize()
+    assert t.check_device() == 0
+    for res in results:
+        for n in names:
+            assert torch.equal(res[n], alone[n]), n
