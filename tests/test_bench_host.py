@@ -97,3 +97,19 @@ def test_traffic_is_tied_to_the_kernel_source(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: src)
     assert bench.ncu_traffic("w1") == 123
     assert bench.ncu_traffic("w2") is None
+
+
+def test_attention_flop_count_closed_forms():
+    """The attention figures count 4 D flops per kept (query, key) pair: all
+    Sq Sk pairs without a mask; with the causal mask (key j <= query i) row i
+    keeps min(i + 1, Sk) keys, whose sum has a closed form for Sq <= Sk (a
+    triangle) and for Sq > Sk (a triangle plus full rows)."""
+    from tensor_core_gemm_tl_b200.compare import attention_flops
+    B, H, D = 3, 5, 64
+    assert attention_flops(B, H, 4096, 4096, D, False) == 4 * B * H * D * 4096 * 4096
+    assert attention_flops(B, H, 4096, 4096, D, True) == 4 * B * H * D * 4096 * 4097 // 2
+    Sq, Sk = 300, 1000  # every row sees i + 1 keys
+    assert attention_flops(B, H, Sq, Sk, D, True) == 4 * B * H * D * Sq * (Sq + 1) // 2
+    Sq, Sk = 1000, 300  # rows past Sk - 1 see all Sk keys
+    kept = Sk * (Sk + 1) // 2 + (Sq - Sk) * Sk
+    assert attention_flops(B, H, Sq, Sk, D, True) == 4 * B * H * D * kept
