@@ -28,6 +28,14 @@
  * the call; a call that must re-lay out an operand (see tl_gemm) takes a
  * stream-ordered temporary from a library-owned CUDA memory pool and returns
  * it on the same stream.
+ *
+ * Threads: every entry point may be called from several host threads at
+ * once, each on its own stream (or the same one).  The library's host state
+ * (per device: the memory pool, the kernels' shared-memory limits and their
+ * occupancy figures) is guarded by a lock held only while that state is
+ * read or first set, never across a launch; tensor maps are encoded per call.
+ * The results of concurrent calls equal those of the same calls made one at
+ * a time.
  */
 #ifndef TL_GEMM_H
 #define TL_GEMM_H
