@@ -53,6 +53,12 @@ MUTANTS = [
     ("attn_mask_wrong_direction", "const int64_t nkeys = causal ? (i + 1 < Sk ? i + 1 : Sk) : Sk;",
      "const int64_t nkeys = causal ? (i < Sk ? i : Sk) + (i == 0) : Sk;"),
     ("attn_scale_ignored", "s[j] = scale * acc;", "s[j] = acc;"),
+    ("attn_scale_squared", "s[j] = scale * acc;", "s[j] = scale * scale * acc;"),
+    ("attn_mask_bottom_right", "const int64_t nkeys = causal ? (i + 1 < Sk ? i + 1 : Sk) : Sk;",
+     "const int64_t off = Sk > Sq ? Sk - Sq : 0;\n"
+     "        const int64_t nkeys = causal ? (i + 1 + off < Sk ? i + 1 + off : Sk) : Sk;"),
+    ("attn_k_from_next_head", "const uint16_t *k = K + (bh * Sk + j) * D;",
+     "const uint16_t *k = K + (((bh + 1) % BH) * Sk + j) * D;"),
     ("attn_no_max_subtraction", "const double w = exp(s[j] - m);", "const double w = exp(s[j]);"),
     ("attn_unnormalised", "o[d] /= l;", "o[d] /= 1.0;"),
     ("attn_v_from_query_row", "const uint16_t *v = V + (bh * Sk + j) * D;",
