@@ -4,16 +4,33 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 One step is one C = epilogue(A . B) call through the C ABI on the workload's
-full size (default: 4096 x 4096 x 4096 fp16, no epilogue -- the GEMM the
-TileLang pages benchmark).  Inputs are seeded synthetic data, resident in HBM
-before the timed region; the timed region rotates over enough input/output
-sets that every step reads operands that are not in L2.  Timing uses CUDA
-events on the launching stream; with N > 1 (torchrun, one process per GPU)
-each rank runs an independent replica (weak scaling, no data-path
+full size.  The default workload is the largest configuration: a transformer
+MLP up-projection, 8192 x 16384 x 4096 in bf16 with the fused bias + exact
+GELU epilogue (the fused epilogue is what the TileLang GPU kernel design
+article, paragraph 5, is about).  Inputs are seeded synthetic data, resident
+in HBM before the timed region; the timed region rotates over enough
+input/output sets that every step reads operands that are not in L2.  Timing
+uses CUDA events on the launching stream; with N > 1 (torchrun, one process
+per GPU) each rank runs an independent replica (weak scaling, no data-path
 collective) and the slowest rank's time counts.
 
+Beside the headline the JSON line carries:
+  per_config  every GEMM configuration of the benchmark set (the pages' 4096^3
+              fp16 GEMM with and without the epilogue, the small fused case,
+              the MLP up-projection, and the ragged / tall / skinny bf16
+              shapes with and without bias + GELU), each timed the same way
+              as a short burst: TFLOP/s, the fraction of the measured dense
+              peak, GB/s of compulsory traffic and its fraction of the
+              measured HBM copy bandwidth, and the same GEMM with its operands
+              left warm in L2;
+  sustained   the headline GEMM run back to back for a few seconds, in the
+              power-capped steady state, against the sustained peak.
+A timed region shorter than a second is a burst and is compared with the
+burst peak; a longer one with the sustained peak.
+
 Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
-instead (bounded row samples of the same workload on the host cores).
+instead (the same bounded row samples of the same workload on the host cores
+that the cpu_baseline figure uses).
 """
 from __future__ import annotations
 
@@ -39,6 +56,24 @@ METRIC = ("GEMM TFLOP/s (1Ã—B200) and fraction of dense fp16/bf16 tensor peak, Â
 UNIT = "TFLOP/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# A timed region at least this long runs in the power-capped steady state.
+SUSTAINED_REGION_S = 1.0
+# Multiply-adds of one oracle call (one sample): about 2 s on 16 host cores.
+ORACLE_SAMPLE_MACS = 1 << 35
+
+# The benchmark set: every GEMM configuration the metric is quoted on.
+PER_CONFIG = (
+    "gemm256_f16_bias_gelu",
+    "gemm4096_f16",
+    "gemm4096_f16_bias_gelu",
+    "mlp_up_8192x16384x4096_bf16_bias_gelu",
+    "ragged_4000x3000x2050_bf16",
+    "ragged_4000x3000x2050_bf16_bias_gelu",
+    "tall_16384x1024x8192_bf16",
+    "tall_16384x1024x8192_bf16_bias_gelu",
+    "skinny_128x16384x4096_bf16",
+    "skinny_128x16384x4096_bf16_bias_gelu",
+)
 
 
 def log(*a):
@@ -86,6 +121,34 @@ def measured_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def tensor_peak(peaks: dict, region_s: float):
+    """(peak TFLOP/s, its name) for a timed region of `region_s` seconds: a
+    burst is compared with the burst figure, a region of a second or more
+    with the sustained (power-capped) figure.  fp16 and bf16 share the dense
+    tensor rate."""
+    burst = float(peaks["bf16_tflops"])
+    if region_s >= SUSTAINED_REGION_S:
+        return float(peaks.get("bf16_tflops_sustained", burst)), "bf16_tflops_sustained"
+    return burst, "bf16_tflops"
+
+
+# Below this time at the roofline a GEMM is bound by launch latency.
+LATENCY_BOUND_S = 5e-6
+
+
+def bound_of(w) -> str:
+    """What bounds the workload at the measured peaks: 'latency' when both its
+    tensor time and its compulsory-traffic time are a few microseconds (the
+    256^3 case), 'hbm' when the traffic takes longer than the flops (the
+    skinny 128-row shape), else 'tensor'."""
+    peaks, _ = measured_peaks()
+    t_tensor = w.flops / (float(peaks["bf16_tflops"]) * 1e12)
+    t_hbm = w.min_bytes() / (float(peaks["hbm_gbs"]) * 1e9)
+    if max(t_tensor, t_hbm) < LATENCY_BOUND_S:
+        return "latency"
+    return "hbm" if t_hbm > t_tensor else "tensor"
+
+
 # The files the GEMM kernel's code and launch are built from; a traffic figure
 # taken on other sources of these files no longer describes the kernel.
 GEMM_SOURCES = ("sm100.cuh", "gemm_kernel.cuh", "config_table.inc", "tl_gemm.cu")
@@ -123,7 +186,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.002):
+    def __init__(self, index: int, period_s: float = 0.0005):
         self.ok = False
         self.samples, self.reasons = [], 0
         self.period = period_s
@@ -139,18 +202,22 @@ class ClockSampler:
             self.max_mhz = None
         self._stop = threading.Event()
 
-    def _run(self):
+    def _sample(self):
         nv = self.nv
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
-                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self.period)
 
     def __enter__(self):
         if self.ok:
+            self._sample()  # at least one sample even for a region shorter than the period
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         return self
@@ -169,33 +236,37 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ the oracle as a CPU baseline
-def oracle_rows_rate(w, A, B, bias, rows, repeats=1):
-    """Seconds and flops for the oracle computing `rows` rows of C."""
-    import oracle  # test infrastructure: the CPU-baseline leg only
+def oracle_sample_rows(w, seed: int = 0) -> np.ndarray:
+    """The rows of C one oracle sample computes: a fixed number of multiply-adds
+    (ORACLE_SAMPLE_MACS), rows drawn without replacement, sorted."""
+    n = int(max(1, min(w.M, round(ORACLE_SAMPLE_MACS / (w.N * w.K)))))
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(w.M, size=n, replace=False))
+
+
+def oracle_sample(w, A, B, bias, rows):
+    """One oracle call on `rows` rows of C: (seconds, flops)."""
+    import oracle  # test infrastructure: the CPU-baseline leg and the reference arm only
     t0 = time.perf_counter()
-    for _ in range(repeats):
-        oracle.gemm(A, B, bias, w.dtype, w.epi, rows=rows)
-    dt = time.perf_counter() - t0
-    return dt, 2.0 * len(rows) * w.N * w.K * repeats
+    oracle.gemm(A, B, bias, w.dtype, w.epi, rows=rows)
+    return time.perf_counter() - t0, 2.0 * len(rows) * w.N * w.K
 
 
 def cpu_baseline(w, A, B, bias, budget_s=12.0):
-    """Oracle throughput on a bounded sample of rows, sized for ~budget_s."""
+    """Oracle throughput: samples of the same size as the reference arm's
+    steps, as many as fit in about budget_s (at least one)."""
     import oracle
-    rng = np.random.default_rng(0)
-    # each call has a fixed cost (decoding B) plus a cost per row: time two
-    # sizes and size the sample from the marginal cost per row
-    small = np.sort(rng.choice(w.M, size=min(4, w.M), replace=False))
-    large = np.sort(rng.choice(w.M, size=min(32, w.M), replace=False))
-    t1, _ = oracle_rows_rate(w, A, B, bias, small)
-    t2, _ = oracle_rows_rate(w, A, B, bias, large)
-    per_row = max((t2 - t1) / max(len(large) - len(small), 1), t2 / len(large) / 8, 1e-9)
-    fixed = max(t1 - per_row * len(small), 0.0)
-    n = int(max(1, min(w.M, (budget_s - fixed) / per_row)))
-    rows = np.sort(rng.choice(w.M, size=n, replace=False))
-    t, f = oracle_rows_rate(w, A, B, bias, rows)
-    return {"value": f / t / 1e12, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": f"{n} of {w.M} rows of C ({n}x{w.N}x{w.K} multiply-adds, fp64), {t:.1f} s"}
+    rows = oracle_sample_rows(w)
+    t_tot = f_tot = 0.0
+    calls = 0
+    while calls == 0 or t_tot + t_tot / calls <= budget_s:
+        t, f = oracle_sample(w, A, B, bias, rows)
+        t_tot += t
+        f_tot += f
+        calls += 1
+    return {"value": f_tot / t_tot / 1e12, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{calls} oracle calls of {len(rows)} of {w.M} rows of C each "
+                      f"({len(rows)}x{w.N}x{w.K} multiply-adds, fp64), {t_tot:.1f} s"}
 
 
 # ------------------------------------------------------------------ the GPU arm
@@ -210,6 +281,137 @@ def ensure_library():
         mod.build(force=True)
 
 
+def rotation_sets(w) -> int:
+    """Input/output sets the timed region rotates over: together at least
+    three times the L2, so every step's operands come from HBM."""
+    set_bytes = 2 * (w.M * w.K + w.K * w.N + w.M * w.N)
+    return max(2, int(np.ceil(3 * L2_BYTES / set_bytes)))
+
+
+def l2_note(w) -> str:
+    set_bytes = 2 * (w.M * w.K + w.K * w.N + w.M * w.N)
+    n = rotation_sets(w)
+    return (f"inputs larger than L2: {n} rotating input/output sets of {set_bytes / 2**20:.0f} MiB "
+            f"({n * set_bytes / 2**20:.0f} MiB > {L2_BYTES / 2**20:.0f} MiB L2)")
+
+
+def common_config(w, seed: int, ws: int) -> dict:
+    """The workload keys both arms print."""
+    return {**w.describe(), "seed": seed, "parallelism": f"replicas{ws}" if ws > 1 else "single",
+            "l2": l2_note(w)}
+
+
+class GemmBench:
+    """Device buffers of one workload and the launch of one step."""
+
+    _host_cache: dict = {}
+
+    def __init__(self, w, dev, seed, tg):
+        import torch
+        self.w, self.dev, self.tg = w, dev, tg
+        self.tdt = torch.float16 if w.dtype == wl.F16 else torch.bfloat16
+        self.A_bits, self.B_bits, self.bias_bits = self.host_inputs(w, seed)
+
+        def dev_tensor(bits):
+            return torch.from_numpy(bits.view(np.int16)).to(dev).view(self.tdt)
+
+        A0, B0 = dev_tensor(self.A_bits), dev_tensor(self.B_bits)
+        self.bias = dev_tensor(self.bias_bits) if self.bias_bits is not None else None
+        self.nsets = rotation_sets(w)
+        self.sets = []
+        for i in range(self.nsets):
+            self.sets.append((A0 if i == 0 else A0.clone(), B0 if i == 0 else B0.clone(),
+                              torch.empty((w.M, w.N), dtype=self.tdt, device=dev)))
+        self.epi = "bias_gelu" if w.epi == wl.EPI_BIAS_GELU else None
+        s0 = self.sets[0]
+        self.plan = tg.plan(w.M, w.N, w.K, w.dtype, self.epi,
+                            num_sms=torch.cuda.get_device_properties(dev).multi_processor_count,
+                            ptrs=(s0[0].data_ptr(), s0[1].data_ptr(),
+                                  self.bias.data_ptr() if self.bias is not None else 0, s0[2].data_ptr()))
+        self.launches_per_step = 1 + self.plan["pad_a"] + self.plan["pad_b"]
+
+    @classmethod
+    def host_inputs(cls, w, seed):
+        # the plain and the bias + GELU form of a shape draw the same A and B
+        key = (w.M, w.N, w.K, w.dtype, w.a, w.b, seed)
+        if key not in cls._host_cache:
+            cls._host_cache.clear()
+            A, B, _ = wl.make_inputs(wl.Workload(w.name, w.M, w.N, w.K, w.dtype, wl.EPI_NONE, w.a, w.b, None), seed)
+            cls._host_cache[key] = (A, B)
+        A, B = cls._host_cache[key]
+        return A, B, wl.make_bias(w, seed)
+
+    def step(self, i, stream, rotate=True):
+        A, B, C = self.sets[i % self.nsets if rotate else 0]
+        self.tg.gemm(A, B, self.bias, epilogue=self.epi, out=C, stream=stream)
+
+    def free(self):
+        self.sets = []
+        self.bias = None
+
+
+def timed_region(bench, stream, steps, warmup, ramp_s, rotate=True, sampler=None, dist=None):
+    """Run an untimed clock ramp and `warmup` steps, then time exactly `steps`
+    steps between two events on `stream` (barrier and synchronize on both
+    sides).  Returns the region's milliseconds on this rank."""
+    import torch
+    t_end = time.time() + ramp_s
+    i = 0
+    while time.time() < t_end:
+        for _ in range(5):
+            bench.step(i, stream, rotate)
+            i += 1
+        torch.cuda.synchronize()
+    for j in range(warmup):
+        bench.step(j, stream, rotate)
+    torch.cuda.synchronize()
+    if bench.tg.check_device() != 0:
+        raise RuntimeError(f"device error during the warm-up of {bench.w.name}")
+    # Events only at the two ends of the region: an event between launches
+    # would serialise them and hide the overlap of one kernel's set-up with the
+    # previous kernel's tail.
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ctx = sampler if sampler is not None else _NullCtx()
+    with ctx:
+        t0.record(stream)
+        for j in range(steps):
+            bench.step(j, stream, rotate)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    if bench.tg.check_device() != 0:
+        raise RuntimeError(f"device error in the timed region of {bench.w.name}")
+    return t0.elapsed_time(t1)
+
+
+class _NullCtx:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+def per_config_entry(w, bench, ms, warm_ms, peaks):
+    tflops = w.flops / (ms / 1e3) / 1e12
+    gbs = w.min_bytes() / (ms / 1e3) / 1e9
+    peak, peak_name = tensor_peak(peaks, 0.0)
+    hbm = float(peaks["hbm_gbs"])
+    bound = bound_of(w)
+    e = {"ms": round(ms, 5), "tflops": round(tflops, 2), "frac": round(tflops / peak, 4),
+         "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4), "bound": bound,
+         "warm_l2_tflops": round(w.flops / (warm_ms / 1e3) / 1e12, 2),
+         "kernel_config": bench.plan["config_name"], "split": bench.plan["split"],
+         "launches_per_step": bench.launches_per_step}
+    # the roofline fraction of the bound that applies
+    e["roofline_frac"] = e["frac_hbm"] if bound == "hbm" else e["frac"]
+    return e
+
+
 def run_gpu(args, w):
     import torch
     ws, rank, local = dist_env()
@@ -220,89 +422,51 @@ def run_gpu(args, w):
     ensure_library()
     import tensor_core_gemm_tl_b200 as tg
 
-    A_bits, B_bits, bias_bits = wl.make_inputs(w, args.seed)
-    tdt = torch.float16 if w.dtype == wl.F16 else torch.bfloat16
-
-    def dev_tensor(bits):
-        return torch.from_numpy(bits.view(np.int16)).to(dev).view(tdt)
-
-    A0, B0 = dev_tensor(A_bits), dev_tensor(B_bits)
-    bias0 = dev_tensor(bias_bits) if bias_bits is not None else None
-    set_bytes = 2 * (w.M * w.K + w.K * w.N + w.M * w.N)
-    nsets = max(2, int(np.ceil(3 * L2_BYTES / set_bytes)))
-    sets = []
-    for i in range(nsets):
-        A = A0 if i == 0 else A0.clone()
-        B = B0 if i == 0 else B0.clone()
-        C = torch.empty((w.M, w.N), dtype=tdt, device=dev)
-        sets.append((A, B, C))
     stream = torch.cuda.current_stream(dev)
-    epi = "bias_gelu" if w.epi == wl.EPI_BIAS_GELU else None
-
-    plan = tg.plan(w.M, w.N, w.K, w.dtype, epi, num_sms=torch.cuda.get_device_properties(dev).multi_processor_count,
-                   ptrs=(sets[0][0].data_ptr(), sets[0][1].data_ptr(),
-                         bias0.data_ptr() if bias0 is not None else 0, sets[0][2].data_ptr()))
-    launches_per_step = 1 + plan["pad_a"] + plan["pad_b"]
-
-    def step(i):
-        A, B, C = sets[i % nsets]
-        tg.gemm(A, B, bias0, epilogue=epi, out=C, stream=stream)
-
-    # bring clocks up, then the W untimed warm-up steps
-    t_end = time.time() + args.ramp_s
-    i = 0
-    while time.time() < t_end:
-        for _ in range(20):
-            step(i)
-            i += 1
-        torch.cuda.synchronize()
-    for j in range(args.warmup):
-        step(j)
-    torch.cuda.synchronize()
-    if tg.check_device() != 0:
-        raise RuntimeError("device error during warm-up")
-
+    peaks, peak_src = measured_peaks()
     K = args.steps
-    # Events only at the two ends of the region: an event between launches
-    # would serialise them and hide the overlap of one kernel's set-up with the
-    # previous kernel's tail.  The kernel's average launch duration is then the
-    # region time over the launches in it (gaps included, so it errs low).
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    # ---------------------------------------------------------------- headline: a burst
+    head = GemmBench(w, dev, args.seed, tg)
     sampler = ClockSampler(local)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with sampler:
-        t_start.record(stream)
-        for j in range(K):
-            step(j)
-        t_end.record(stream)
-        torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    region_ms = t_start.elapsed_time(t_end)
-    if tg.check_device() != 0:
-        raise RuntimeError("device error in the timed region")
+    region_ms = timed_region(head, stream, K, args.warmup, args.ramp_s, sampler=sampler, dist=dist)
     region_ms_max = max_over_ranks(region_ms, dist, dev)
-    gemm_launches = K  # the GEMM kernel runs once per step
-    kernel_ms = region_ms / gemm_launches
-
+    clocks = sampler.summary()
+    kernel_ms = region_ms / K  # one GEMM launch per step (plus the pad copies when an operand needs them)
     value = aggregate(w.flops * K, region_ms_max / 1e3, ws) / 1e12
+    peak, peak_name = tensor_peak(peaks, region_ms_max / 1e3)
+    achieved = w.flops / (kernel_ms / 1e3) / 1e12
+    bound = bound_of(w)
+    roof = {"bound": bound, "unit": UNIT, "traffic": ncu_traffic(w.name),
+            "kernel_ms": round(kernel_ms, 5), "kernel_ms_is": "timed region / GEMM launches",
+            "algorithmic_flops_per_launch": w.flops, "min_hbm_bytes_per_launch": w.min_bytes(),
+            "region_s": round(region_ms_max / 1e3, 4)}
+    if bound == "hbm":
+        gbs = w.min_bytes() / (kernel_ms / 1e3) / 1e9
+        roof.update({"achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                     "frac": round(gbs / float(peaks["hbm_gbs"]), 4),
+                     "peak_source": f"{peak_src} hbm_gbs (copy)", "tflops": round(achieved, 2)})
+    else:
+        roof.update({"achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_src} {peak_name} (cuBLAS; a region under "
+                                    f"{SUSTAINED_REGION_S:g} s is a burst); fp16 dense rate equals bf16"})
 
-    # End to end through the public API, the way a caller streams work through
-    # it: every step copies its inputs from pinned host memory, runs the GEMM and
+    # ---------------------------------------------------------------- end to end through the public API
+    # Every step copies its inputs from pinned host memory, runs the GEMM and
     # copies C back; consecutive steps alternate between two CUDA streams, so
     # one step's copies overlap another step's GEMM.
     e2e_steps = max(3, min(K, args.e2e_steps))
     nstreams = 2
-    A_h = torch.from_numpy(A_bits.view(np.int16)).view(tdt).pin_memory()
-    B_h = torch.from_numpy(B_bits.view(np.int16)).view(tdt).pin_memory()
-    b_h = torch.from_numpy(bias_bits.view(np.int16)).view(tdt).pin_memory() if bias_bits is not None else None
+    tdt = head.tdt
+    A_h = torch.from_numpy(head.A_bits.view(np.int16)).view(tdt).pin_memory()
+    B_h = torch.from_numpy(head.B_bits.view(np.int16)).view(tdt).pin_memory()
+    b_h = (torch.from_numpy(head.bias_bits.view(np.int16)).view(tdt).pin_memory()
+           if head.bias_bits is not None else None)
     streams = [torch.cuda.Stream(dev) for _ in range(nstreams)]
     lanes = []
     for i in range(nstreams):
-        Ad, Bd, Cd = sets[i % nsets]
-        bd = torch.empty_like(bias0) if bias0 is not None else None
+        Ad, Bd, Cd = head.sets[i % head.nsets]
+        bd = torch.empty_like(head.bias) if head.bias is not None else None
         lanes.append((streams[i], Ad, Bd, bd, Cd, torch.empty((w.M, w.N), dtype=tdt).pin_memory()))
 
     def e2e_step(j):
@@ -312,7 +476,7 @@ def run_gpu(args, w):
             Bd.copy_(B_h, non_blocking=True)
             if bd is not None:
                 bd.copy_(b_h, non_blocking=True)
-            tg.gemm(Ad, Bd, bd, epilogue=epi, out=Cd, stream=s)
+            tg.gemm(Ad, Bd, bd, epilogue=head.epi, out=Cd, stream=s)
             C_h.copy_(Cd, non_blocking=True)
 
     for j in range(2 * nstreams):
@@ -332,43 +496,57 @@ def run_gpu(args, w):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     e2e_value = aggregate(w.flops * e2e_steps, e2e_ms / 1e3, ws) / 1e12
-    h2d = 2 * (w.M * w.K + w.K * w.N) + (2 * w.N if bias_bits is not None else 0)
+    h2d = 2 * (w.M * w.K + w.K * w.N) + (2 * w.N if head.bias_bits is not None else 0)
     d2h = 2 * w.M * w.N
+    del lanes, A_h, B_h, b_h
 
-    peaks, peak_src = measured_peaks()
-    # fp16 and bf16 share the dense tensor rate.  A timed region that runs under
-    # sustained load (the clock ramp plus the region last a second or more) is
-    # compared with the sustained figure, a short burst with the burst figure.
-    burst = float(peaks["bf16_tflops"])
-    sustained = float(peaks.get("bf16_tflops_sustained", burst))
-    long_run = args.ramp_s + region_ms_max / 1e3 >= 1.0
-    peak = sustained if long_run else burst
-    peak_name = "bf16_tflops_sustained (back-to-back cuBLAS loop)" if long_run else "bf16_tflops (burst, cuBLAS)"
-    achieved = w.flops / (kernel_ms / 1e3) / 1e12
+    # ---------------------------------------------------------------- every configuration, as a burst
+    per_config = {}
+    if not args.no_per_config:
+        for name in PER_CONFIG:
+            wc = wl.WORKLOADS[name]
+            b = head if name == w.name else GemmBench(wc, dev, args.seed, tg)
+            time.sleep(args.rest_s)  # let the power controller settle between bursts
+            ms = max_over_ranks(timed_region(b, stream, K, args.warmup, args.ramp_s, dist=dist), dist, dev) / K
+            warm_ms = max_over_ranks(timed_region(b, stream, K, args.warmup, 0.0, rotate=False, dist=dist),
+                                     dist, dev) / K
+            per_config[name] = per_config_entry(wc, b, ms, warm_ms, peaks)
+            if b is not head:
+                b.free()
+                del b
+            torch.cuda.empty_cache()
+
+    # ---------------------------------------------------------------- the headline, sustained
+    sustained = None
+    if args.sustained_s > 0:
+        n = max(K, int(np.ceil(args.sustained_s / (kernel_ms / 1e3))))
+        s_sampler = ClockSampler(local, period_s=0.01)
+        s_ms = max_over_ranks(timed_region(head, stream, n, args.warmup, 0.0, sampler=s_sampler, dist=dist),
+                              dist, dev)
+        s_tflops = w.flops * n / (s_ms / 1e3) / 1e12
+        s_peak, s_name = tensor_peak(peaks, s_ms / 1e3)
+        sustained = {"steps": n, "region_s": round(s_ms / 1e3, 3), "tflops": round(s_tflops, 2),
+                     "peak": s_peak, "frac": round(s_tflops / s_peak, 4), "peak_source": f"{peak_src} {s_name}",
+                     "clocks": s_sampler.summary()}
+
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": ws, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(region_ms_max / K, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.DTYPE_NAMES[w.dtype], "data": "synthetic",
         "impl": "tl_gemm",
-        "config": {**w.describe(), "kernel_config": plan["config_name"], "grid": plan["grid"],
-                   "parallelism": f"replicas{ws}" if ws > 1 else "single",
-                   "l2": f"rotating {nsets} input/output sets of {set_bytes / 2**20:.0f} MiB "
-                         f"({nsets * set_bytes / 2**20:.0f} MiB > {L2_BYTES / 2**20:.0f} MiB L2)",
-                   "accumulate": "f32", "seed": args.seed},
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": UNIT,
-                     "frac": round(achieved / peak, 4), "traffic": ncu_traffic(w.name),
-                     "peak_source": f"{peak_src} {peak_name}; fp16 dense rate equals bf16",
-                     "frac_of_burst_peak": round(achieved / burst, 4),
-                     "kernel_ms": round(kernel_ms, 5), "kernel_ms_is": "timed region / launches",
-                     "algorithmic_flops_per_launch": w.flops,
-                     "min_hbm_bytes_per_launch": w.min_bytes()},
+        "config": common_config(w, args.seed, ws),
+        "kernel": {"config": head.plan["config_name"], "grid": head.plan["grid"], "split": head.plan["split"],
+                   "accumulate": "f32"},
+        "roofline": roof,
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps, "streams": nstreams},
-        "gpu_launches": K * launches_per_step,
-        "clocks": sampler.summary(),
+        "gpu_launches": K * head.launches_per_step,
+        "clocks": clocks,
+        "per_config": per_config,
+        "sustained": sustained,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(w, A_bits, B_bits, bias_bits, args.cpu_budget_s)
+        out["cpu_baseline"] = cpu_baseline(w, head.A_bits, head.B_bits, head.bias_bits, args.cpu_budget_s)
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -383,37 +561,25 @@ def run_reference(args, w):
         return  # the oracle runs once, on rank 0's host cores
     import oracle
     A, B, bias = wl.make_inputs(w, args.seed)
-    rng = np.random.default_rng(1)
-
-    def points(n):
-        return rng.integers(0, w.M, n), rng.integers(0, w.N, n)
-
-    def timed(n):
-        ii, jj = points(n)
-        t0 = time.perf_counter()
-        oracle.gemm_points(A, B, bias, w.dtype, w.epi, ii, jj)
-        return time.perf_counter() - t0
-
-    # one step = `n` single elements of C (2K flops each) through the oracle's
-    # element entry point, sized so that all steps fit in about ref_budget_s
-    timed(256)
-    per_point = max(timed(2048) / 2048, 1e-9)
-    total_steps = args.steps + args.warmup
-    n = int(max(64, min(w.M * w.N, args.ref_budget_s / total_steps / per_point)))
+    rows = oracle_sample_rows(w)
+    # one step = one oracle call on the same row sample the cpu_baseline leg
+    # times, so that the two CPU figures measure the same thing
     for _ in range(args.warmup):
-        timed(n)
-    t_tot = 0.0
+        oracle_sample(w, A, B, bias, rows)
+    t_tot = f_tot = 0.0
     for _ in range(args.steps):
-        t_tot += timed(n)
-    f_tot = 2.0 * w.K * n * args.steps
+        t, f = oracle_sample(w, A, B, bias, rows)
+        t_tot += t
+        f_tot += f
     value = f_tot / t_tot / 1e12
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * t_tot / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {**w.describe(), "seed": args.seed},
+        "config": common_config(w, args.seed, ws),
         "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": oracle.max_threads(),
-                         "sample": f"{n} random elements of C per step (2K flops each), fp64"},
+                         "sample": f"one oracle call per step on {len(rows)} of {w.M} rows of C "
+                                   f"({len(rows)}x{w.N}x{w.K} multiply-adds, fp64)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
@@ -422,16 +588,20 @@ def run_reference(args, w):
 def parse(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=wl.HEADLINE, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--impl", default="tl_gemm", choices=["tl_gemm", "reference"])
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--ramp-s", type=float, default=1.0, help="untimed clock ramp before the warm-up steps")
+    ap.add_argument("--ramp-s", type=float, default=0.05,
+                    help="untimed back-to-back launches before the warm-up steps (brings the SM clock up)")
+    ap.add_argument("--rest-s", type=float, default=0.5, help="idle time before each per-configuration burst")
+    ap.add_argument("--sustained-s", type=float, default=3.0,
+                    help="length of the sustained (power-capped) run of the headline; 0 skips it")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
-    ap.add_argument("--ref-budget-s", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -78,7 +78,7 @@ typedef enum {
     TL_ERR_MISALIGNED = 3,      /* a pointer not aligned to its 2-byte element */
     TL_ERR_CUDA = 4,            /* a CUDA runtime or driver call failed */
     TL_ERR_DEVICE_TIMEOUT = 5,  /* a bounded wait inside a kernel ran out (see tl_check_device) */
-    TL_ERR_SCRATCH_LIMIT = 6    /* tl_gemm_noalloc: the call needs more than TL_NOALLOC_SCRATCH_BYTES */
+    TL_ERR_SCRATCH_LIMIT = 6    /* tl_gemm_noalloc: the call needs more workspace than TL_NOALLOC_SCRATCH_BYTES */
 } tl_status;
 
 /* A cudaStream_t, passed as an opaque pointer; NULL is the legacy default stream. */
@@ -132,17 +132,26 @@ TL_API tl_status tl_gemm(const void *A, const void *B, const void *bias, void *C
  * TL_NOALLOC_SCRATCH_BYTES that the library declares statically: each GPU the
  * library is used on holds that much device memory until the process exits.
  *
+ * What goes into the scratch area is everything tl_gemm would put in its
+ * temporary: the zero-padded copies of A and/or B, and, for a shape whose
+ * last round of tiles is split along K, the fp32 partial sums of the split
+ * tiles and their arrival words.  tl_gemm_plan reports the bytes a call needs
+ * as workspace_bytes; every call with workspace_bytes > 0 uses the scratch
+ * area, aligned shapes that split included, and a call with workspace_bytes
+ * == 0 does not touch it.
+ *
  * Arguments, layout rules, results and errors are those of tl_gemm, plus
- * TL_ERR_SCRATCH_LIMIT when the padded copies the call needs are larger than
- * TL_NOALLOC_SCRATCH_BYTES (tl_gemm_plan reports the need as
- * workspace_bytes).  Nothing is enqueued in that case.  A call whose operands
- * need no padding uses no scratch at all.
+ * TL_ERR_SCRATCH_LIMIT when the call needs more workspace than
+ * TL_NOALLOC_SCRATCH_BYTES.  Nothing is enqueued in that case.
  *
  * The scratch area is shared by all calls on a device and keeps what the last
- * call wrote; each call rewrites every byte of it that it later reads.  Calls
- * whose work can overlap on the GPU (different streams with no ordering
- * between them) race on the scratch area and can give wrong results: order
- * them on one stream, or with events.
+ * call wrote; each call writes every byte of it that it later reads (partial
+ * sums and arrival words are tagged with the launch's own stamp, so nothing a
+ * previous call left behind is ever taken for this call's data).  Calls that
+ * use the scratch area and whose work can overlap on the GPU (different
+ * streams with no ordering between them) race on it and can give wrong
+ * results -- padded copies and split partial sums alike: order them on one
+ * stream, or with events.
  *
  * The first call on each device does a one-time set-up with that device
  * current: it looks up the device address of the scratch area, raises the

@@ -43,6 +43,20 @@ _EPILOGUES = {None: TL_EPI_NONE, "none": TL_EPI_NONE, "bias_gelu": TL_EPI_BIAS_G
               "bias_gelu_tanh": TL_EPI_BIAS_GELU_TANH, "gelu_tanh": TL_EPI_GELU_TANH}
 
 
+def _require_device_tensor(name, t, device, dtype=None, shape=None):
+    """Raise ValueError unless `t` is a contiguous CUDA tensor on `device` (and
+    of `dtype` / `shape` when given): a host or foreign-device pointer must
+    never reach a kernel's loads or stores."""
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
 def _epi_code(epilogue):
     if isinstance(epilogue, int) and TL_EPI_NONE <= epilogue <= TL_EPI_GELU_TANH:
         return epilogue
@@ -74,14 +88,17 @@ def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0,
     for name, t in (("A", A), ("B", B)):
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if B.device != A.device:
+        raise ValueError(f"B is on {B.device}, A on {A.device}")
     dt = _dtype_code(A)
     if B.dtype != A.dtype:
         raise TypeError("A and B must have the same dtype")
     M, K = A.shape
     N = B.shape[0] if b_transposed else B.shape[1]
     if epi in TL_EPI_WITH_BIAS:
-        if bias is None or bias.shape != (N,) or bias.dtype != A.dtype or not bias.is_cuda or not bias.is_contiguous():
+        if bias is None:
             raise ValueError("this epilogue needs a contiguous CUDA bias of length N in the input dtype")
+        _require_device_tensor("bias", bias, A.device, A.dtype, (N,))
     if out_dtype is None:
         out_dtype = out.dtype if out is not None else A.dtype
     if out_dtype not in (A.dtype, torch.float32):
@@ -89,8 +106,8 @@ def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0,
     c_f32 = out_dtype == torch.float32
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=A.device)
-    elif out.shape != (M, N) or out.dtype != out_dtype or not out.is_contiguous() or not out.is_cuda:
-        raise ValueError("out must be a contiguous CUDA tensor of shape (M, N) and C's dtype")
+    else:
+        _require_device_tensor("out", out, A.device, out_dtype, (M, N))
     s = stream if stream is not None else torch.cuda.current_stream(A.device)
     bias_ptr = bias.data_ptr() if bias is not None and epi in TL_EPI_WITH_BIAS else 0
     with torch.cuda.device(A.device):
@@ -113,18 +130,20 @@ def attention(q, k, v, causal: bool = False, scale: float = 0.0, out=None, lse=N
     import torch
     if q.dim() != 4 or k.shape != v.shape or k.dim() != 4 or q.shape[:2] != k.shape[:2] or q.shape[3] != k.shape[3]:
         raise ValueError(f"shapes q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)} do not match")
+    if not q.is_cuda:
+        raise ValueError("q must be a CUDA tensor")
     for name, t in (("q", q), ("k", k), ("v", v)):
-        if not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype:
-            raise ValueError(f"{name} must be a contiguous CUDA tensor of q's dtype")
+        _require_device_tensor(name, t, q.device, q.dtype)
     dt = _dtype_code(q)
     B, H, Sq, D = q.shape
     Sk = k.shape[2]
+    # every given tensor is checked before anything is allocated
+    if lse is not None:
+        _require_device_tensor("lse", lse, q.device, torch.float32, (B, H, Sq))
     if out is None:
         out = torch.empty_like(q)
-    elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
-        raise ValueError("out must be contiguous, of q's shape and dtype")
-    if lse is not None and (lse.shape != (B, H, Sq) or lse.dtype != torch.float32 or not lse.is_contiguous()):
-        raise ValueError("lse must be a contiguous float32 tensor of shape (B, H, Sq)")
+    else:
+        _require_device_tensor("out", out, q.device, q.dtype, q.shape)
     s = stream if stream is not None else torch.cuda.current_stream(q.device)
     with torch.cuda.device(q.device):
         st = tl_attention_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
@@ -141,9 +160,10 @@ def softmax(x, out=None, stream=None):
     if x.dim() != 2 or not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous 2-D CUDA tensor")
     dt = _dtype_code(x)
-    out = torch.empty_like(x) if out is None else out
-    if out.shape != x.shape or out.dtype != x.dtype or not out.is_contiguous():
-        raise ValueError("out must match x")
+    if out is None:
+        out = torch.empty_like(x)
+    else:
+        _require_device_tensor("out", out, x.device, x.dtype, x.shape)
     s = stream if stream is not None else torch.cuda.current_stream(x.device)
     with torch.cuda.device(x.device):
         st = tl_softmax_rows(x.data_ptr(), out.data_ptr(), x.shape[0], x.shape[1], dt, s.cuda_stream)
@@ -155,9 +175,14 @@ def softmax(x, out=None, stream=None):
 def vector_add(a, b, out=None, stream=None):
     """a + b for contiguous float32 CUDA tensors of one shape."""
     import torch
-    if a.shape != b.shape or a.dtype != torch.float32 or b.dtype != torch.float32 or not a.is_cuda:
-        raise ValueError("a and b must be float32 CUDA tensors of one shape")
-    out = torch.empty_like(a) if out is None else out
+    if not a.is_cuda:
+        raise ValueError("a must be a CUDA tensor")
+    _require_device_tensor("a", a, a.device, torch.float32)
+    _require_device_tensor("b", b, a.device, torch.float32, a.shape)
+    if out is None:
+        out = torch.empty_like(a)
+    else:
+        _require_device_tensor("out", out, a.device, torch.float32, a.shape)
     s = stream if stream is not None else torch.cuda.current_stream(a.device)
     with torch.cuda.device(a.device):
         st = tl_vector_add(a.data_ptr(), b.data_ptr(), out.data_ptr(), a.numel(), s.cuda_stream)

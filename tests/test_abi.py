@@ -169,6 +169,87 @@ def test_torch_wrapper_rejects_bad_tensors():
         tg._epi_code("relu")
 
 
+class _FakeCuda:
+    """Stands in for a CUDA tensor on a machine without one: it carries what
+    the binding's checks read, and fails the test if a pointer is taken."""
+
+    def __init__(self, shape, dtype, device="cuda:0", contiguous=True):
+        import torch
+        self.shape = torch.Size(shape)
+        self.dtype = dtype
+        self.device = torch.device(device)
+        self.is_cuda = self.device.type == "cuda"
+        self._contiguous = contiguous
+
+    def is_contiguous(self):
+        return self._contiguous
+
+    def dim(self):
+        return len(self.shape)
+
+    def numel(self):
+        return int(np.prod(self.shape))
+
+    def data_ptr(self):
+        raise AssertionError("a pointer was taken from a tensor that should have been rejected")
+
+
+def _bad_tensor_cases():
+    import torch
+    bf, f32 = torch.bfloat16, torch.float32
+    F = _FakeCuda
+    cpu = lambda shape, dt: torch.zeros(shape, dtype=dt)  # noqa: E731
+    q = lambda: F((1, 2, 128, 64), bf)  # noqa: E731
+    x = lambda: F((8, 256), bf)  # noqa: E731
+    v = lambda: F((1000,), f32)  # noqa: E731
+    A, B = (lambda: F((64, 32), bf)), (lambda: F((32, 48), bf))  # noqa: E731
+    return [
+        # attention: out / lse on the host, on another device, of the wrong shape, dtype or layout
+        ("attention", lambda: tg.attention(q(), q(), q(), out=cpu((1, 2, 128, 64), bf))),
+        ("attention", lambda: tg.attention(q(), q(), q(), out=F((1, 2, 128, 64), bf, "cuda:1"))),
+        ("attention", lambda: tg.attention(q(), q(), q(), out=F((1, 2, 128, 64), bf, contiguous=False))),
+        ("attention", lambda: tg.attention(q(), q(), q(), lse=cpu((1, 2, 128), f32))),
+        ("attention", lambda: tg.attention(q(), q(), q(), lse=F((1, 2, 128), bf))),
+        ("attention", lambda: tg.attention(q(), q(), q(), lse=F((1, 2, 127), f32))),
+        ("attention", lambda: tg.attention(q(), q(), q(), lse=F((1, 2, 128), f32, contiguous=False))),
+        ("attention", lambda: tg.attention(q(), F((1, 2, 128, 64), bf, "cuda:1"), q())),
+        # softmax: out on the host or elsewhere
+        ("softmax", lambda: tg.softmax(x(), out=cpu((8, 256), bf))),
+        ("softmax", lambda: tg.softmax(x(), out=F((8, 256), bf, "cuda:1"))),
+        ("softmax", lambda: tg.softmax(x(), out=F((8, 256), bf, contiguous=False))),
+        ("softmax", lambda: tg.softmax(x(), out=F((8, 255), bf))),
+        # vector add: b and out on the host, elsewhere, strided, or of another shape
+        ("vector_add", lambda: tg.vector_add(v(), cpu((1000,), f32))),
+        ("vector_add", lambda: tg.vector_add(v(), F((1000,), f32, "cuda:1"))),
+        ("vector_add", lambda: tg.vector_add(v(), F((1000,), f32, contiguous=False))),
+        ("vector_add", lambda: tg.vector_add(F((1000,), f32, contiguous=False), v())),
+        ("vector_add", lambda: tg.vector_add(v(), v(), out=cpu((1000,), f32))),
+        ("vector_add", lambda: tg.vector_add(v(), v(), out=F((999,), f32))),
+        ("vector_add", lambda: tg.vector_add(v(), v(), out=F((1000,), f32, contiguous=False))),
+        # GEMM: B, bias and out on the host or another device
+        ("gemm", lambda: tg.gemm(A(), F((32, 48), bf, "cuda:1"))),
+        ("gemm", lambda: tg.gemm(A(), B(), cpu((48,), bf))),
+        ("gemm", lambda: tg.gemm(A(), B(), F((48,), bf, "cuda:1"))),
+        ("gemm", lambda: tg.gemm(A(), B(), out=cpu((64, 48), bf))),
+        ("gemm", lambda: tg.gemm(A(), B(), out=F((64, 48), bf, "cuda:1"))),
+    ]
+
+
+@pytest.mark.parametrize("case", range(24))
+def test_binding_rejects_host_and_foreign_tensors_before_any_launch(case, monkeypatch):
+    cases = _bad_tensor_cases()
+    assert len(cases) == 24
+    _, call = cases[case]
+
+    def no_launch(*a, **k):
+        raise AssertionError("the C ABI was called with a tensor the binding should have rejected")
+
+    for name in ("tl_gemm", "tl_gemm_ex", "tl_attention_fwd", "tl_softmax_rows", "tl_vector_add"):
+        monkeypatch.setattr(tg, name, no_launch)
+    with pytest.raises(ValueError):
+        call()
+
+
 @pytest.mark.parametrize("M,N,K,config,split,full", [
     (4096, 4096, 4096, 4, 2, 222),   # 256 pair tiles on 74 pairs: 3 rounds + 34 tiles split in two
     (4096, 4096, 4096, 1, 2, 444),   # 512 single-CTA tiles on 148: 68 left over, split in two

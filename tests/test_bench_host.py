@@ -58,7 +58,8 @@ def test_single_process_needs_no_process_group():
 
 def test_argument_contract():
     a = bench.parse([])
-    assert a.gpus == 1 and a.warmup >= 3 and a.steps >= 1 and a.workload == "gemm4096_f16"
+    assert a.gpus == 1 and a.warmup >= 3 and a.steps >= 1
+    assert a.workload == "mlp_up_8192x16384x4096_bf16_bias_gelu"  # the largest configuration
     with pytest.raises(SystemExit):
         bench.parse(["--warmup", "2"])
 
@@ -67,8 +68,8 @@ def test_reference_arm_json_line():
     env = dict(os.environ, PYTHONPATH=ROOT)
     env.pop("WORLD_SIZE", None)
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--workload", "gemm256_f16_bias_gelu", "--steps", "3", "--warmup", "3",
-                        "--ref-budget-s", "2"], capture_output=True, text=True, timeout=300, env=env)
+                        "--workload", "gemm256_f16_bias_gelu", "--steps", "3", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300, env=env)
     assert r.returncode == 0, r.stderr
     lines = [x for x in r.stdout.splitlines() if x.strip()]
     assert len(lines) == 1
@@ -77,6 +78,8 @@ def test_reference_arm_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"] == "gemm256_f16_bias_gelu"
+    # the same workload keys the GPU arm prints
+    assert d["config"] == bench.common_config(bench.wl.WORKLOADS["gemm256_f16_bias_gelu"], 0, 1)
 
 
 def test_reference_arm_other_ranks_print_nothing():
