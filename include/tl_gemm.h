@@ -25,9 +25,9 @@
  * configuration give bit-identical results.
  *
  * All calls are host functions.  None of them allocates memory that outlives
- * the call; a call that must re-lay out an operand (see tl_gemm) takes a
- * stream-ordered temporary from a library-owned CUDA memory pool and returns
- * it on the same stream.
+ * the call; a call that must re-lay out an operand, or whose last round of
+ * tiles is cut along K (see tl_gemm), takes a stream-ordered temporary from a
+ * library-owned CUDA memory pool and returns it on the same stream.
  *
  * Threads: every entry point may be called from several host threads at
  * once, each on its own stream (or the same one).  The library's host state
@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define TL_VERSION 1001 /* major * 1000 + minor */
+#define TL_VERSION 1002 /* major * 1000 + minor */
 
 #if defined(__GNUC__)
 #define TL_API __attribute__((visibility("default")))
@@ -106,6 +106,16 @@ typedef void *tl_stream;
  * through the tensor-memory-access unit.  Both are slower than the aligned
  * path but give the same numbers.
  *
+ * Work split: output tiles are dealt to persistent units (one SM, or a pair
+ * of SMs); when the last round of tiles would leave units idle for much of a
+ * tile's time, its k-blocks are spread evenly over all units instead, and
+ * each partly computed tile is finished by the unit that completes its last
+ * part, which adds the parts' float32 partial sums in k order (a fixed order:
+ * results stay bit-reproducible).  The partial sums live in the same
+ * stream-ordered temporary (tl_gemm_plan's workspace_bytes).  No part of the
+ * kernel waits for another unit, so concurrent calls on several streams
+ * cannot stall one another.
+ *
  * Ownership: the caller owns every buffer and must keep them alive until the
  * work on `stream` completes.  The call does not synchronize.
  *
@@ -159,7 +169,7 @@ TL_API tl_status tl_gemm(const void *A, const void *B, const void *bias, void *C
  * Make that first call before any stream capture begins.  After it, a call
  * allocates nothing, on the device or on the host.
  */
-#define TL_NOALLOC_SCRATCH_BYTES (32ull << 20)
+#define TL_NOALLOC_SCRATCH_BYTES (64ull << 20)
 
 TL_API tl_status tl_gemm_noalloc(const void *A, const void *B, const void *bias, void *C,
                          int64_t M, int64_t N, int64_t K,
@@ -224,16 +234,18 @@ typedef struct {
     int32_t config;       /* 0: the library's choice for the shape; k > 0: kernel
                              configuration k - 1 (see tl_num_configs)            */
     int32_t inject_fault; /* test hook, 0 in production: 1 makes the copy warp
-                             skip its first stage without issuing the copy, so
-                             the consumer's bounded wait runs out and the kernel
-                             returns with TL_ERR_DEVICE_TIMEOUT recorded; 2 makes
+                             (of both CTAs, with a CTA pair) skip its first
+                             stage without issuing the copy, so the MMA warp's
+                             bounded wait runs out and the kernel drains what
+                             it issued and returns with TL_ERR_DEVICE_TIMEOUT
+                             recorded (bit 1 of the detail word); 2 makes
                              the host treat the encoding of A's tensor map as
                              failed: the call returns TL_ERR_CUDA and the GEMM
                              kernel is not launched (padding copies the shape
                              needs may already be enqueued; their temporary is
                              released on the stream)                             */
     uint64_t timeout_ns;  /* bound on every wait inside the kernel; 0 = 10 s     */
-    int32_t no_split;     /* 1: never split the tiles of a short last round      */
+    int32_t no_split;     /* 1: never cut the tiles of a short last round along K */
     int32_t b_layout;     /* 0: B is K x N row-major (leading dimension N);
                              1: B is given transposed, N x K row-major (leading
                              dimension K) -- the layout of a weight W in A.W^T */
@@ -257,8 +269,8 @@ TL_API tl_status tl_gemm_ex(const void *A, const void *B, const void *bias, void
  * early, C is incomplete), TL_ERR_CUDA if the synchronization failed, TL_OK
  * otherwise.  `detail`, if not NULL, receives the raw error word (which waits
  * gave up: bit 0 copy warp, bit 1 MMA warp on data, bit 2 MMA warp on the
- * accumulator, bit 3 epilogue warps, bit 4 final drain, bit 5 the last K part
- * of a split tile waiting for an earlier part, bit 6 the row softmax waiting
+ * accumulator, bit 3 epilogue warps, bit 4 final drain, bit 5 a part of a
+ * split tile that could not record its arrival, bit 6 the row softmax waiting
  * for a row's copy into shared memory, bit 7 -- in the checked build
  * libtlgemm_checked.so only -- an index invariant of the GEMM kernel failed).
  */
@@ -275,13 +287,24 @@ typedef struct {
     int32_t tiles_m, tiles_n;
     int32_t grid;            /* persistent CTAs launched                       */
     int32_t cluster_ctas;    /* 1, or 2 when pairs of CTAs share each tile     */
-    int32_t split;           /* K parts of each tile of the last, partial round
-                                of tiles (1: none are split)                   */
-    int32_t full_tiles;      /* tiles computed whole; the rest are split       */
+    int32_t split;           /* the last, partial round of tiles has its k-blocks
+                                spread evenly over all units, so one tile can be
+                                shared by several units: the most units sharing
+                                one tile (1: nothing is split)                  */
+    int32_t full_tiles;      /* tiles computed whole by one unit; the rest form
+                                the split last round                           */
     int32_t pad_a, pad_b;    /* 1 when the operand is first copied to a padded temporary */
     int32_t direct_store;    /* 1 when C is stored element by element          */
     int32_t smem_bytes;      /* dynamic shared memory per CTA                  */
     int64_t workspace_bytes; /* stream-ordered temporary the call takes        */
+    int32_t tail_units;      /* units the split last round is spread over (0: no
+                                split); unit u < tail_units takes the last
+                                round's k-blocks [u T / tail_units, (u + 1) T /
+                                tail_units), T = (tiles - full_tiles) * k-blocks
+                                per tile, tiles in order, each tile's k-blocks in
+                                order                                           */
+    int32_t num_slots;       /* partial-sum slots in the workspace (slot u + r:
+                                unit u's part of last-round tile r)             */
 } tl_plan;
 
 TL_API tl_status tl_gemm_plan(const void *A, const void *B, const void *bias, void *C,

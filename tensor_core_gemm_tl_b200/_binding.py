@@ -52,7 +52,8 @@ class Plan(ctypes.Structure):
                 ("tiles_n", ctypes.c_int32), ("grid", ctypes.c_int32), ("cluster_ctas", ctypes.c_int32),
                 ("split", ctypes.c_int32), ("full_tiles", ctypes.c_int32), ("pad_a", ctypes.c_int32),
                 ("pad_b", ctypes.c_int32), ("direct_store", ctypes.c_int32),
-                ("smem_bytes", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64)]
+                ("smem_bytes", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64),
+                ("tail_units", ctypes.c_int32), ("num_slots", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}

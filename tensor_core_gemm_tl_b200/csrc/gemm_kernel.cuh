@@ -27,8 +27,11 @@
 // Two TMEM accumulators (2 x BN fp32 columns) let the epilogue of tile i run
 // while the MMAs of tile i+1 accumulate.  Every wait is bounded by a
 // %globaltimer limit: on expiry the kernel records which wait gave up in a
-// device error word, lets its issued copies and MMAs land, frees TMEM and
-// returns (no trap, no hang).
+// device error word, lets its issued copies and MMAs land (with a CTA pair,
+// the even CTA drains the copies of both), frees TMEM and returns (no trap,
+// no hang).  The last round of tiles can be cut along K across units; the
+// parts of a tile are combined by whichever unit finishes last, so no unit
+// ever waits for another.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -49,7 +52,7 @@ enum : unsigned {
     ERR_MMA_ACC = 4u,
     ERR_EPILOGUE = 8u,
     ERR_DRAIN = 16u,
-    ERR_SPLIT = 32u,   // the last part of a split tile gave up waiting for an earlier part
+    ERR_SPLIT = 32u,   // a part of a split tile could not record its arrival (C incomplete)
     ERR_CHECK = 128u,  // checked build only: an index invariant failed (the access was skipped)
 };
 
@@ -80,56 +83,125 @@ struct GemmParams {
     int32_t epi_bias;        // fused epilogue: add bias[col]
     int32_t epi_gelu;        // fused epilogue: 0 no GELU, 1 exact (erf) GELU, 2 tanh-form GELU
     int32_t bias_vec16;      // bias is 16-byte aligned: load 8 values per access
-    int32_t inject_fault;    // test hook: skip the first stage's copy
+    int32_t inject_fault;    // test hook: every producer skips its first stage
     uint16_t *C;             // 16-bit element-store path only
     float *C32;              // float32 output only
     int32_t c32_vec16;       // float32 output: base 16-byte aligned and ldc % 4 == 0
     int64_t ldc;             // element-store and float32 paths (elements)
     uint64_t timeout_ns;
-    // Work items: tiles [0, full_tiles) whole, then each remaining tile split
-    // along K into `split` parts, item = full_tiles + r * split + part.  Parts
-    // 0 .. split-2 leave fp32 partial sums in `partials` and stamp their flag
-    // with `epoch`; the last part adds them, in part order, to its own sum and
-    // runs the epilogue.
-    int32_t full_tiles, split, num_items;
-    int32_t num_slabs;       // 128-row fp32 partial slabs the workspace holds
-    float *partials;
-    unsigned long long *flags;
-    unsigned long long epoch;  // unique per launch
+    // Work: tiles [0, full_tiles) whole, dealt round-robin to the units (CTAs,
+    // or CTA pairs); then the `tail_tiles` tiles of the last round, whose
+    // tail_tiles * num_kb k-blocks are cut into `tail_units` consecutive
+    // ranges, one per unit.  A tile whose k-blocks fall to several units is
+    // finished by whichever of them arrives last: each writes its fp32 partial
+    // sums to its own slot of `partials` and then counts itself on the tile's
+    // arrival word (tagged with this launch's `epoch`); the unit that completes
+    // the count adds the parts in k order and runs the epilogue.  No unit ever
+    // waits for another.
+    int32_t full_tiles, tail_tiles, tail_units;
+    int32_t num_slots;       // partial-sum slots in the workspace (tail_units + tail_tiles - 1)
+    float *partials;         // [slot][cta of the pair][128 rows][BN columns] fp32
+    unsigned long long *arrivals;  // [tail tile][cta][lane quarter][64-column chunk]
+    unsigned long long epoch;  // unique per launch, below 2^56
 };
 
+// One unit of work: k-blocks [kb0, kb1) of output tile `tile`.  `tail` is the
+// tile's index in the last round when its k-blocks are cut across units (else
+// -1).
 struct WorkItem {
-    int tile, part, kb0, kb1;  // output tile, part index, k-block range [kb0, kb1)
+    int tile, kb0, kb1, tail;
 };
 
-__device__ __forceinline__ WorkItem work_item(int item, const GemmParams &p)
+// What one unit computes: n_full whole tiles (unit, unit + num_units, ...),
+// then up to two pieces of the last round (its k-block range can end in the
+// next tile).
+struct UnitWork {
+    int n_full, n_seg;
+    int seg_r0, seg_kb00, seg_kb10;
+    int seg_r1, seg_kb01, seg_kb11;
+};
+
+__device__ __forceinline__ UnitWork unit_work(int unit, int num_units, const GemmParams &p)
+{
+    UnitWork u{};
+    u.n_full = unit < p.full_tiles ? (p.full_tiles - 1 - unit) / num_units + 1 : 0;
+    u.n_seg = 0;
+    if (unit < p.tail_units) {
+        const int64_t T = static_cast<int64_t>(p.tail_tiles) * p.num_kb;
+        int64_t g = static_cast<int64_t>(unit) * T / p.tail_units;
+        const int64_t g1 = static_cast<int64_t>(unit + 1) * T / p.tail_units;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            if (g >= g1)
+                break;
+            const int r = static_cast<int>(g / p.num_kb);
+            const int64_t base = static_cast<int64_t>(r) * p.num_kb;
+            const int64_t end = g1 < base + p.num_kb ? g1 : base + p.num_kb;
+            if (i == 0) {
+                u.seg_r0 = r;
+                u.seg_kb00 = static_cast<int>(g - base);
+                u.seg_kb10 = static_cast<int>(end - base);
+            } else {
+                u.seg_r1 = r;
+                u.seg_kb01 = static_cast<int>(g - base);
+                u.seg_kb11 = static_cast<int>(end - base);
+            }
+            u.n_seg = i + 1;
+            g = end;
+        }
+    }
+    return u;
+}
+
+__device__ __forceinline__ WorkItem work_item(const UnitWork &u, int i, int unit, int num_units,
+                                              const GemmParams &p)
 {
     WorkItem w;
-    if (item < p.full_tiles) {
-        w.tile = item;
-        w.part = 0;
+    if (i < u.n_full) {
+        w.tile = unit + i * num_units;
         w.kb0 = 0;
         w.kb1 = p.num_kb;
+        w.tail = -1;
     } else {
-        const int r = (item - p.full_tiles) / p.split;
-        w.part = item - p.full_tiles - r * p.split;
-        w.tile = p.full_tiles + r;
-        w.kb0 = (w.part * p.num_kb) / p.split;
-        w.kb1 = ((w.part + 1) * p.num_kb) / p.split;
+        const bool second = i > u.n_full;
+        w.tail = second ? u.seg_r1 : u.seg_r0;
+        w.tile = p.full_tiles + w.tail;
+        w.kb0 = second ? u.seg_kb01 : u.seg_kb00;
+        w.kb1 = second ? u.seg_kb11 : u.seg_kb10;
     }
     return w;
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *addr)
+// The units whose k-block ranges meet tail tile r: first .. last.  Unit u's
+// range starts at floor(u T / U), so the unit holding global k-block x is
+// ceil((x + 1) U / T) - 1 (T tail k-blocks, U tail units).
+__device__ __forceinline__ void tail_contributors(int r, const GemmParams &p, int &first, int &last)
 {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(addr) : "memory");
-    return v;
+    const int64_t T = static_cast<int64_t>(p.tail_tiles) * p.num_kb;
+    const int64_t U = p.tail_units;
+    const int64_t x0 = static_cast<int64_t>(r) * p.num_kb;
+    const int64_t x1 = x0 + p.num_kb - 1;
+    first = static_cast<int>(((x0 + 1) * U + T - 1) / T) - 1;
+    last = static_cast<int>(((x1 + 1) * U + T - 1) / T) - 1;
 }
 
-__device__ __forceinline__ void st_release_u64(unsigned long long *addr, unsigned long long v)
+// Count one more part of a split tile on its arrival word and return the
+// count (0 if the word could not be updated, which is recorded).  The word's
+// upper 56 bits hold the launch's epoch: a word that carries another epoch
+// (left by an earlier launch, or never written) counts as zero.
+__device__ __forceinline__ unsigned arrive_tagged(unsigned long long *word, unsigned long long epoch)
 {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(addr), "l"(v) : "memory");
+    const unsigned long long tag = epoch << 8;
+    unsigned long long old = ld_relaxed_u64(word);
+    for (int i = 0; i < 4096; ++i) {
+        const unsigned long long next = (old & ~0xFFull) == tag ? old + 1ull : (tag | 1ull);
+        const unsigned long long seen = atom_cas_acq_rel_u64(word, old, next);
+        if (seen == old)
+            return static_cast<unsigned>(next & 0xFFull);
+        old = seen;
+    }
+    atomicOr(&g_device_error, ERR_SPLIT);
+    return 0u;
 }
 
 // Compile-time tile configuration.  Each CTA owns BM = 128 output rows (one
@@ -162,7 +234,10 @@ struct TileConfig {
     static constexpr int OFF_C = OFF_B + STAGES * B_STAGE_BYTES;
     static constexpr int OFF_BAR = OFF_C + C_STAGING_BYTES;
     static constexpr int NUM_BARS = 2 * STAGES + 5;
-    static constexpr int SMEM_USED = OFF_BAR + NUM_BARS * 8 + 16;
+    // after the barriers: TMEM address, abort flag, 8 spare bytes, then the
+    // copies issued per stage by this CTA and (pair) by the odd CTA
+    static constexpr int OFF_COUNTS = OFF_BAR + NUM_BARS * 8 + 16;
+    static constexpr int SMEM_USED = OFF_COUNTS + 2 * STAGES * 4;
     static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024
     static constexpr int THREADS = 64 + 32 * EPI_WARPS;  // producer, MMA, epilogue warps
     static_assert(BN_LOCAL % 64 == 0 && BN >= 64 && BN <= 256, "BN");
@@ -222,30 +297,6 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
         }
     }
     return true;
-}
-
-// Bounded wait, by every lane, until an earlier part of a split tile has
-// stamped its flag with this launch's epoch.
-__device__ __forceinline__ bool wait_part(const unsigned long long *flag, unsigned long long epoch,
-                                          volatile int *abort_flag, uint64_t timeout_ns, uint32_t peer_abort)
-{
-    if (ld_acquire_u64(flag) == epoch)
-        return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
-        __nanosleep(100);
-        if (ld_acquire_u64(flag) == epoch)
-            return true;
-        if (*abort_flag)
-            return false;
-        if (global_timer_ns() - t0 > timeout_ns) {
-            *abort_flag = 1;
-            if (peer_abort)
-                st_shared_cluster_u32(peer_abort, 1u);
-            atomicOr(&g_device_error, ERR_SPLIT);
-            return false;
-        }
-    }
 }
 
 template <int DT>
@@ -369,6 +420,9 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + CF::OFF_BAR + CF::NUM_BARS * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const uint32_t peer_abort = PAIR ? mapa_shared(smem_addr(tmem_slot + 1), rank ^ 1u) : 0u;
+    // copies issued per stage: by this CTA, and (on the even CTA of a pair) by the odd one
+    volatile uint32_t *issue_count = reinterpret_cast<volatile uint32_t *>(smem + CF::OFF_COUNTS);
+    volatile uint32_t *peer_issue_count = issue_count + CF::STAGES;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < CF::STAGES; ++s) {
@@ -381,6 +435,8 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
+        for (int s = 0; s < 2 * CF::STAGES; ++s)
+            issue_count[s] = 0u;
         fence_mbar_init();
         fence_proxy_async_smem();
     }
@@ -413,21 +469,21 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
     grid_dependency_wait();
     grid_launch_dependents();
 
-    // Last fill issued per stage (bit s set) and its phase parity: on an abort,
-    // every copy issued is waited for before the CTA exits.
-    uint32_t issued = 0, issued_parity = 0;
+    // Every role walks the same list of work items.
+    const UnitWork uw = unit_work(unit, num_units, p);
+    const int n_items = uw.n_full + uw.n_seg;
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            bool skip = p.inject_fault != 0 && leader;
+            bool skip = p.inject_fault != 0;  // both CTAs of a pair skip the same stage
             bool ok = true;
-            for (int item = unit; ok && item < p.num_items; item += num_units) {
-                const WorkItem w = work_item(item, p);
+            for (int i = 0; ok && i < n_items; ++i) {
+                const WorkItem w = work_item(uw, i, unit, num_units, p);
                 int tm, tn;
                 tile_coords(w.tile, p, tm, tn);
-                check_ok(w.tile < p.num_tiles && w.part < p.split && w.kb0 <= w.kb1 && w.kb1 <= p.num_kb &&
+                check_ok(w.tile < p.num_tiles && w.tail < p.tail_tiles && w.kb0 < w.kb1 && w.kb1 <= p.num_kb &&
                          tm < p.tiles_m && tn < p.tiles_n);  // TMA clips anything outside: record only
                 const int a_row = tm * CF::TILE_M + static_cast<int>(rank) * CF::BM;
                 const int b_col = tn * CF::BN + static_cast<int>(rank) * CF::BN_LOCAL;
@@ -469,8 +525,7 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                                                 kb * CF::BK);
                             }
                         }
-                        issued |= 1u << stage;
-                        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                        issue_count[stage] = issue_count[stage] + 1u;
                     }
                     if (++stage == CF::STAGES) {
                         stage = 0;
@@ -494,8 +549,8 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int item = unit; ok && item < p.num_items; item += num_units) {
-                const WorkItem w = work_item(item, p);
+            for (int i = 0; ok && i < n_items; ++i) {
+                const WorkItem w = work_item(uw, i, unit, num_units, p);
                 if (!wait_bounded<PAIR>(tempty_bar(acc), acc_phase ^ 1u, abort_flag, timeout, ERR_MMA_ACC,
                                         peer_abort)) {
                     ok = false;
@@ -561,14 +616,17 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
         uint8_t *buf = cstage + (warp - 2) * CF::C_BOX_BYTES;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int item = unit; item < p.num_items; item += num_units) {
-            const WorkItem w = work_item(item, p);
+        for (int i = 0; i < n_items; ++i) {
+            const WorkItem w = work_item(uw, i, unit, num_units, p);
             int tm, tn;
             tile_coords(w.tile, p, tm, tn);
-            check_ok(w.tile < p.num_tiles && w.part < p.split && tm < p.tiles_m && tn < p.tiles_n);
+            check_ok(w.tile < p.num_tiles && w.tail < p.tail_tiles && tm < p.tiles_m && tn < p.tiles_n);
             const int n0 = tn * CF::BN;
-            const bool split_tile = w.tile >= p.full_tiles;
-            const int r_tail = w.tile - p.full_tiles;
+            // a tile of the last round whose k-blocks several units share
+            int t_first = unit, t_last = unit;
+            if (w.tail >= 0)
+                tail_contributors(w.tail, p, t_first, t_last);
+            const bool shared_tile = t_last > t_first;
             const int row0 = tm * CF::TILE_M + static_cast<int>(rank) * CF::BM + q * 32;  // this warp's rows
             if (!wait_bounded<PAIR>(tfull_bar(acc), acc_phase, abort_flag, timeout, ERR_EPILOGUE, peer_abort))
                 break;
@@ -601,50 +659,54 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                 if (col0 >= p.N || row0 >= p.M)
                     continue;  // nothing of this chunk lies inside C
 
-                if (split_tile) {
-                    // partial sums of one split tile: [part < split-1][cta][128 rows][BN cols] fp32,
-                    // one flag per (part, cta, lane quarter, chunk)
-                    const size_t slab0 = static_cast<size_t>(r_tail) * (p.split - 1) * CF::CTAS + rank;
-                    const size_t slab_step = CF::CTAS;  // from part to part + 1
+                if (shared_tile) {
+                    // This chunk's fp32 partial sums go to this unit's slot; the
+                    // part that arrives last on the chunk's word adds all the
+                    // parts in k order (first .. last unit) and stores C.
+                    const size_t slab_elems = static_cast<size_t>(CF::BM) * CF::BN;
                     const size_t row_off = (static_cast<size_t>(q) * 32 + lane) * CF::BN + c * 64;
-                    const size_t flag_off = static_cast<size_t>(q) * CHUNKS + c;
-                    if (!check_ok(slab0 + (p.split - 2) * slab_step < static_cast<size_t>(p.num_slabs)))
+                    auto slab_of = [&](int u) {
+                        return static_cast<size_t>(u + w.tail) * CF::CTAS + rank;  // slot u + r is unique per (unit, tail tile)
+                    };
+                    if (!check_ok(slab_of(t_last) < static_cast<size_t>(p.num_slots) * CF::CTAS))
                         continue;  // outside the workspace
-                    if (w.part < p.split - 1) {
-                        const size_t slab = slab0 + w.part * slab_step;
-                        float4 *dst = reinterpret_cast<float4 *>(p.partials + slab * CF::BM * CF::BN + row_off);
+                    float4 *mine = reinterpret_cast<float4 *>(p.partials + slab_of(unit) * slab_elems + row_off);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            __stcg(dst + i, make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                                        __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
-                        __threadfence();
-                        __syncwarp();
-                        if (lane == 0)
-                            st_release_u64(p.flags + slab * 4 * CHUNKS + flag_off, p.epoch);
-                        continue;  // the last part stores this chunk of C
+                    for (int i = 0; i < 16; ++i)
+                        __stcg(mine + i, make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                     __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
+                    __threadfence();
+                    __syncwarp();
+                    unsigned count = 0;
+                    if (lane == 0) {
+                        const size_t word = ((static_cast<size_t>(w.tail) * CF::CTAS + rank) * 4 + q) * CHUNKS + c;
+                        count = arrive_tagged(p.arrivals + word, p.epoch);
                     }
-                    // last part: sum = part 0 + part 1 + ... + this part, in that order
-                    bool have = true;
-                    for (int part = 0; have && part < p.split - 1; ++part)
-                        have = wait_part(p.flags + (slab0 + part * slab_step) * 4 * CHUNKS + flag_off, p.epoch,
-                                         abort_flag, timeout, peer_abort);
-                    if (!__all_sync(0xffffffffu, have))
-                        continue;  // recorded in the error word; C stays incomplete
-                    const float4 *src0 = reinterpret_cast<const float4 *>(p.partials + slab0 * CF::BM * CF::BN + row_off);
+                    count = __shfl_sync(0xffffffffu, count, 0);
+                    if (count != static_cast<unsigned>(t_last - t_first + 1))
+                        continue;  // an earlier arrival: the last part stores this chunk
+                    __threadfence();
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        float4 a = __ldcg(src0 + i);
-                        for (int part = 1; part < p.split - 1; ++part) {
-                            const float4 b = __ldcg(src0 + part * slab_step * CF::BM * CF::BN / 4 + i);
-                            a.x += b.x;
-                            a.y += b.y;
-                            a.z += b.z;
-                            a.w += b.w;
+                        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int u = t_first; u <= t_last; ++u) {
+                            const float4 b = u == unit ? make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                                     __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]))
+                                                       : __ldcg(reinterpret_cast<const float4 *>(
+                                                                    p.partials + slab_of(u) * slab_elems + row_off) + i);
+                            if (u == t_first) {
+                                a = b;
+                            } else {
+                                a.x += b.x;
+                                a.y += b.y;
+                                a.z += b.z;
+                                a.w += b.w;
+                            }
                         }
-                        r[4 * i] = __float_as_uint(a.x + __uint_as_float(r[4 * i]));
-                        r[4 * i + 1] = __float_as_uint(a.y + __uint_as_float(r[4 * i + 1]));
-                        r[4 * i + 2] = __float_as_uint(a.z + __uint_as_float(r[4 * i + 2]));
-                        r[4 * i + 3] = __float_as_uint(a.w + __uint_as_float(r[4 * i + 3]));
+                        r[4 * i] = __float_as_uint(a.x);
+                        r[4 * i + 1] = __float_as_uint(a.y);
+                        r[4 * i + 2] = __float_as_uint(a.z);
+                        r[4 * i + 3] = __float_as_uint(a.w);
                     }
                 }
 
@@ -719,8 +781,7 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                                         crow[j] = v[j];
                             }
                         }
-                        continue;
-                    }
+                    } else {
                     uint32_t packed[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
@@ -748,6 +809,7 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                             }
                         }
                     }
+                    }  // 16-bit C
                 }
                 if constexpr (STORE == STORE_TMA) {
                     fence_proxy_async_smem();
@@ -772,19 +834,43 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
 
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 0 && lane == 0 && *abort_flag) {
-        if constexpr (PAIR) {
-            // The pair's copies complete on the even CTA's barriers, which an
-            // abort can leave short of their arrival: give whatever is still in
-            // flight a fixed grace period (loads finish in microseconds).
-            const uint64_t t0 = global_timer_ns();
-            while (global_timer_ns() - t0 < 200000ull) {
-            }
-        } else {
-            // Some role gave up: copies it never consumed may still be landing.
+    if constexpr (PAIR) {
+        // The odd CTA's copies complete on the even CTA's barriers: hand the
+        // even CTA this CTA's per-stage copy counts, so that it can drain for
+        // both.
+        if (!leader && warp == 0 && lane == 0) {
             for (int s = 0; s < CF::STAGES; ++s)
-                if (issued & (1u << s))
-                    wait_drain(full_bar(s), (issued_parity >> s) & 1u, timeout);
+                st_shared_cluster_u32(mapa_shared(smem_addr(const_cast<uint32_t *>(peer_issue_count + s)), 0),
+                                      issue_count[s]);
+        }
+        cluster_sync();
+    }
+    if (leader && warp == 0 && lane == 0 && *abort_flag) {
+        // Some role gave up: copies no one consumed may still be landing.
+        // Stage s's copies before the last phase anyone issued were all
+        // consumed (a copy is issued only after its slot's previous contents
+        // were), so only that last phase can be pending.  With a pair, that
+        // phase may have been issued by one CTA only; the even CTA then
+        // completes the half that will never come (the odd CTA's bytes, or its
+        // own arrival with the odd CTA's byte count) and waits for the half
+        // that is in flight.
+        for (int s = 0; s < CF::STAGES; ++s) {
+            const uint32_t mine = issue_count[s];
+            const uint32_t peer = PAIR ? peer_issue_count[s] : mine;
+            const uint32_t n = mine > peer ? mine : peer;
+            if (n == 0)
+                continue;
+            if (mine + 1 < n || peer + 1 < n) {
+                atomicOr(&g_device_error, ERR_DRAIN);  // cannot happen: the counts differ by one at most
+                continue;
+            }
+            if constexpr (PAIR) {
+                if (mine == n && peer + 1 == n)
+                    mbar_complete_tx(full_bar(s), CF::STAGE_BYTES);
+                else if (peer == n && mine + 1 == n)
+                    mbar_arrive_expect_tx(full_bar(s), CF::STAGE_BYTES);
+            }
+            wait_drain(full_bar(s), (n - 1) & 1u, timeout);
         }
     }
     if constexpr (PAIR)

@@ -57,6 +57,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return done != 0;
 }
 
+// Count `bytes` of the current phase's transaction as done without a copy
+// (used only to let a phase complete whose other half was never issued).
+__device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// ---------------------------------------------------------------- global-memory atomics
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *addr)
+{
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(addr) : "memory");
+    return v;
+}
+
+// Compare-and-swap with acquire-release semantics at GPU scope; returns the
+// value found at `addr`.
+__device__ __forceinline__ unsigned long long atom_cas_acq_rel_u64(unsigned long long *addr, unsigned long long cmp,
+                                                                  unsigned long long val)
+{
+    unsigned long long old;
+    asm volatile("atom.acq_rel.gpu.global.cas.b64 %0, [%1], %2, %3;" : "=l"(old) : "l"(addr), "l"(cmp), "l"(val)
+                 : "memory");
+    return old;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map)
 {

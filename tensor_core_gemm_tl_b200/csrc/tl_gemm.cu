@@ -132,27 +132,9 @@ int model_config(int64_t M, int64_t N, int num_sms)
     return best;
 }
 
-// Best single-CTA configuration by the same model (the fault hook needs one).
-int model_config_single(int64_t M, int64_t N, int num_sms)
-{
-    int best = 0;
-    double best_cost = 1e300;
-    static const double eff[] = {0.62, 0.5, 0.33};
-    for (int i = 0; i < 3; ++i) {
-        const ConfigEntry &c = kConfigs[i];
-        const int64_t tiles = ceil_div(M, c.bm) * ceil_div(N, c.bn);
-        const double cost = static_cast<double>(ceil_div(tiles, num_sms)) * c.bm * c.bn / eff[i];
-        if (cost < best_cost - 1e-9) {
-            best_cost = cost;
-            best = i;
-        }
-    }
-    return best;
-}
-
-// The measured choice for this shape, else the wave model without splitting
-// (on a power-capped B200 the sweep found splitting the last round a loss for
-// most shapes).
+// The measured choice for this shape (configuration, and whether its last
+// round may be cut along K), else the wave model with the split rule of
+// tail_split.
 int choose_config(int64_t M, int64_t N, int64_t K, int dtype, int epi, int num_sms, bool *split)
 {
     for (const TableRow &r : kTable) {
@@ -164,7 +146,7 @@ int choose_config(int64_t M, int64_t N, int64_t K, int dtype, int epi, int num_s
             }
         }
     }
-    *split = false;
+    *split = true;
     return model_config(M, N, num_sms);
 }
 
@@ -174,8 +156,9 @@ struct Plan {
     tl_plan pub;
     int64_t lda, ldb;        // row lengths (elements) of the operands the kernel reads
     int64_t a_ws_off, b_ws_off;
-    int64_t partial_off, flag_off;  // split-tile partial sums and their flags
+    int64_t partial_off, arrival_off;  // split-tile partial sums and their arrival words
     int32_t num_kb;
+    int32_t tail_tiles, tail_units, num_slots;
 };
 
 bool epi_has_bias(int epi)
@@ -222,8 +205,6 @@ tl_status validate(const void *A, const void *B, const void *bias, void *C, int6
     if (opt && ((opt->no_split != 0 && opt->no_split != 1) || (opt->b_layout != 0 && opt->b_layout != 1) ||
                 (opt->c_float32 != 0 && opt->c_float32 != 1)))
         return TL_ERR_INVALID_ARG;
-    if (opt && opt->inject_fault == 1 && opt->config > 0 && kConfigs[opt->config - 1].ctas != 1)
-        return TL_ERR_UNSUPPORTED;  // the fault hook exists for single-CTA configurations only
     const int64_t lim = 0x7FFFFFFFll;
     if (M > lim || N > lim || K > lim)
         return TL_ERR_UNSUPPORTED;
@@ -234,29 +215,45 @@ tl_status validate(const void *A, const void *B, const void *bias, void *C, int6
 }
 
 // How the tiles of one launch are cut into work items.  Tiles fill whole
-// rounds of `units` (CTAs, or CTA pairs) first; when the last round would be
-// at most half full, each of its tiles is split along K into `split` parts so
-// that the round takes 1/split of a tile's time.  (With fewer tiles than
-// units, the same rule is plain split-K.)  Every unit then holds at most one
-// part of the last round, and all units are resident together, so the last
-// part of a tile can wait for the earlier parts without any risk of waiting
-// on work that is queued behind it.
-void split_tail(int64_t tiles, int64_t units, int64_t num_kb, int32_t *split, int64_t *full_tiles)
+// rounds of `units` (CTAs, or CTA pairs) first.  The tiles of a last, partial
+// round would leave units idle for a whole tile's time; instead their
+// k-blocks can be spread evenly over the units, each unit taking one
+// consecutive range (which may end inside the next tile).  A tile whose
+// k-blocks fall to several units is summed by the last of them to finish (see
+// the kernel): nobody waits, so nothing depends on all units being resident.
+// The split is taken when it saves at least max(4, num_kb / 8) k-blocks of
+// the last round's time -- below that the partial sums' traffic and the extra
+// epilogue pass eat the gain -- and every unit then gets at least 4 k-blocks.
+struct TailSplit {
+    int64_t full_tiles, tail_tiles, tail_units;
+    int32_t max_parts;  // most units sharing one tile (1: none shared)
+};
+
+TailSplit tail_split(int64_t tiles, int64_t units, int64_t num_kb, bool allow)
 {
-    *split = 1;
-    *full_tiles = tiles;
+    TailSplit t{tiles, 0, 0, 1};
     const int64_t rem = tiles % units;
-    if (rem == 0 || num_kb < 8)
-        return;
-    int64_t s = units / rem;
-    if (s > 4)
-        s = 4;
-    if (s > num_kb / 4)
-        s = num_kb / 4;
-    if (s >= 2) {
-        *split = static_cast<int32_t>(s);
-        *full_tiles = tiles - rem;
+    if (!allow || rem == 0 || num_kb < 8)
+        return t;
+    const int64_t T = rem * num_kb;
+    const int64_t tail_units = units < T / 4 ? units : T / 4;
+    if (tail_units <= rem)
+        return t;
+    const int64_t saved = num_kb - (T + tail_units - 1) / tail_units;
+    const int64_t need = num_kb / 8 > 4 ? num_kb / 8 : 4;
+    if (saved < need)
+        return t;
+    t.full_tiles = tiles - rem;
+    t.tail_tiles = rem;
+    t.tail_units = tail_units;
+    // units meeting tail tile r: ceil((x + 1) U / T) - 1 for its first and last k-block x
+    for (int64_t r = 0; r < rem; ++r) {
+        const int64_t first = ((r * num_kb + 1) * tail_units + T - 1) / T - 1;
+        const int64_t last = (((r + 1) * num_kb) * tail_units + T - 1) / T - 1;
+        if (last - first + 1 > t.max_parts)
+            t.max_parts = static_cast<int32_t>(last - first + 1);
     }
+    return t;
 }
 
 tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N,
@@ -270,8 +267,6 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
         return TL_ERR_INVALID_ARG;
     bool table_split = true;  // a forced configuration splits unless told not to
     int ci = (opt && opt->config > 0) ? opt->config - 1 : choose_config(M, N, K, dtype, epi, num_sms, &table_split);
-    if (opt && opt->inject_fault == 1 && kConfigs[ci].ctas != 1)
-        ci = model_config_single(M, N, num_sms);
     const ConfigEntry &c = kConfigs[ci];
     Plan p{};
     tl_plan &q = p.pub;
@@ -289,14 +284,22 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
     if (max_units > 0 && max_units < units)
         units = max_units;
     p.num_kb = static_cast<int32_t>(ceil_div(K, c.bk));
-    int64_t full_tiles = tiles;
-    int32_t split = 1;
-    if (table_split && !(opt && (opt->inject_fault == 1 || opt->no_split)))
-        split_tail(tiles, units, p.num_kb, &split, &full_tiles);
-    const int64_t items = full_tiles + (tiles - full_tiles) * split;
-    q.split = split;
-    q.full_tiles = static_cast<int32_t>(full_tiles);
-    q.grid = static_cast<int32_t>((items < units ? items : units) * c.ctas);
+    const TailSplit ts = tail_split(tiles, units, p.num_kb, table_split && !(opt && opt->no_split));
+    q.split = ts.max_parts;
+    q.full_tiles = static_cast<int32_t>(ts.full_tiles);
+    p.tail_tiles = static_cast<int32_t>(ts.tail_tiles);
+    p.tail_units = static_cast<int32_t>(ts.tail_units);
+    p.num_slots = ts.tail_tiles > 0 ? static_cast<int32_t>(ts.tail_units + ts.tail_tiles - 1) : 0;
+    q.tail_units = p.tail_units;
+    q.num_slots = p.num_slots;
+    // units that get work: those with whole tiles, and those with a piece of
+    // the split last round
+    int64_t busy = ts.full_tiles < units ? ts.full_tiles : units;
+    if (ts.tail_tiles > 0 && ts.tail_units > busy)
+        busy = ts.tail_units;
+    if (ts.tail_tiles == 0)
+        busy = tiles < units ? tiles : units;
+    q.grid = static_cast<int32_t>(busy * c.ctas);
     q.cluster_ctas = c.ctas;
     q.smem_bytes = c.smem_bytes;
     // TMA needs a 16-byte-aligned base and row strides that are multiples of 16 bytes.
@@ -318,13 +321,15 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
         p.b_ws_off = ws;
         ws += ceil_div(b_rows * p.ldb * 2, 256) * 256;
     }
-    p.partial_off = p.flag_off = -1;
-    if (split > 1) {
-        const int64_t slabs = (tiles - full_tiles) * (split - 1) * c.ctas;  // 128-row partial slabs
+    p.partial_off = p.arrival_off = -1;
+    if (ts.tail_tiles > 0) {
+        // one 128 x BN fp32 slab per (slot, CTA of the pair); one arrival word
+        // per (tail tile, CTA, TMEM lane quarter, 64-column chunk)
+        const int64_t slabs = static_cast<int64_t>(p.num_slots) * c.ctas;
         p.partial_off = ws;
         ws += ceil_div(slabs * 128 * c.bn * 4, 256) * 256;
-        p.flag_off = ws;
-        ws += ceil_div(slabs * 4 * (c.bn / 64) * 8, 256) * 256;
+        p.arrival_off = ws;
+        ws += ceil_div(ts.tail_tiles * c.ctas * 4 * (c.bn / 64) * 8, 256) * 256;
     }
     q.workspace_bytes = ws;
     *out = p;
@@ -467,19 +472,22 @@ tl_status launch_pad(const void *src, int64_t rows, int64_t cols, void *dst, int
 // Launch the GEMM itself with operands the kernel can read through TMA.
 std::atomic<unsigned long long> g_epoch{0};
 
-// A launch stamp no earlier launch of this process has used, starting from a
+// A launch stamp below 2^56 (it shares a 64-bit arrival word with an 8-bit
+// count) that no earlier launch of this process has used, starting from a
 // random point so that memory left by another process never matches it.
 unsigned long long next_epoch()
 {
+    constexpr unsigned long long kMask = (1ull << 56) - 1;
     unsigned long long e = g_epoch.fetch_add(1) + 1;
     if (e == 1) {
         std::random_device rd;
-        const unsigned long long base = ((static_cast<unsigned long long>(rd()) << 32) ^ rd()) | 1ull;
+        const unsigned long long base = (((static_cast<unsigned long long>(rd()) << 32) ^ rd()) & kMask) | 1ull;
         unsigned long long expected = 1;
         g_epoch.compare_exchange_strong(expected, base);
         e = g_epoch.fetch_add(1) + 1;
     }
-    return e;
+    e &= kMask;
+    return e ? e : 1ull;
 }
 
 tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *bias, void *C, int64_t M,
@@ -528,18 +536,18 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
     gp.c32_vec16 = store == STORE_F32 && aligned(C, 16) && N % 4 == 0;
     gp.ldc = N;
     gp.timeout_ns = (opt && opt->timeout_ns) ? opt->timeout_ns : kDefaultTimeoutNs;
-    gp.split = p.pub.split;
     gp.full_tiles = p.pub.full_tiles;
-    gp.num_items = p.pub.full_tiles + (gp.num_tiles - p.pub.full_tiles) * p.pub.split;
-    gp.num_slabs = (gp.num_tiles - p.pub.full_tiles) * (p.pub.split - 1) * c.ctas;
+    gp.tail_tiles = p.tail_tiles;
+    gp.tail_units = p.tail_units;
+    gp.num_slots = p.num_slots;
     gp.partials = nullptr;
-    gp.flags = nullptr;
+    gp.arrivals = nullptr;
     gp.epoch = 0;
-    if (p.pub.split > 1) {
+    if (p.tail_tiles > 0) {
         if (!workspace)
             return TL_ERR_INVALID_ARG;
         gp.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + p.partial_off);
-        gp.flags = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + p.flag_off);
+        gp.arrivals = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + p.arrival_off);
         gp.epoch = next_epoch();
     }
 
@@ -568,7 +576,8 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
 }
 
 // The plan for this device: for CTA-pair configurations, no more pairs than
-// can be resident at once (the split-tile rule relies on it).
+// can be resident at once (a persistent unit that is not resident would only
+// start when another has finished all its work).
 tl_status device_plan(DeviceState *d, const void *A, const void *B, const void *bias, void *C, int64_t M,
                       int64_t N, int64_t K, int dtype, int epi, const tl_gemm_options *opt, Plan *p)
 {

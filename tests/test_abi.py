@@ -138,16 +138,13 @@ def test_plan_forced_config():
         assert p["grid"] % p["cluster_ctas"] == 0 and p["grid"] <= 148
 
 
-def test_fault_hook_only_on_single_cta_configs():
+def test_fault_hook_is_accepted_on_every_config():
+    # single CTAs and CTA pairs alike: with a pair, both CTAs skip the same stage
     for k in range(1, tg.tl_num_configs() + 1):
         opt = tg.Options(config=k, inject_fault=1)
         st, p = tg.tl_gemm_plan(P, P, 0, P, 512, 512, 512, 0, 0, 148, opt)
-        if tg.tl_config_name(k - 1).endswith("_pair"):
-            assert st == tg.Status.UNSUPPORTED
-        else:
-            assert st == 0 and p.cluster_ctas == 1
-    st, p = tg.tl_gemm_plan(P, P, 0, P, 4096, 4096, 4096, 0, 0, 148, tg.Options(inject_fault=1))
-    assert st == 0 and p.cluster_ctas == 1
+        assert st == 0 and p.config == k - 1
+        assert p.cluster_ctas == (2 if tg.tl_config_name(k - 1).endswith("_pair") else 1)
 
 
 def test_plan_skinny_prefers_narrow_tiles():
@@ -250,28 +247,28 @@ def test_binding_rejects_host_and_foreign_tensors_before_any_launch(case, monkey
         call()
 
 
-@pytest.mark.parametrize("M,N,K,config,split,full", [
-    (4096, 4096, 4096, 4, 2, 222),   # 256 pair tiles on 74 pairs: 3 rounds + 34 tiles split in two
-    (4096, 4096, 4096, 1, 2, 444),   # 512 single-CTA tiles on 148: 68 left over, split in two
-    (1024, 1024, 2048, 1, 4, 0),     # 32 tiles on 148 SMs: plain split-K, 4 parts
-    (1024, 1024, 1024, 4, 4, 0),     # 16 pair tiles on 74 pairs: 4 parts
-    (1280, 1536, 1024, 4, 2, 0),     # 30 tiles: 2 parts
-    (1024, 1280, 1536, 4, 3, 0),     # 20 tiles: 3 parts
-    (2560, 640, 1024, 3, 2, 148),    # 200 tiles of 128 x 64: one full round, 52 tiles split
-    (8192, 16384, 4096, 4, 1, 2048), # last round 50 of 74: not worth splitting
-    (700, 900, 333, 4, 1, 12),       # too few k blocks to split
+@pytest.mark.parametrize("M,N,K,config,dtype,split,full", [
+    (4096, 4096, 4096, 4, 1, True, 222),    # 256 pair tiles on 74 pairs: 3 rounds + 34 tiles spread over 74
+    (4096, 4096, 4096, 1, 1, True, 444),    # 512 single-CTA tiles on 148: 68 left over
+    (1024, 1024, 2048, 1, 1, True, 0),      # 32 tiles on 148 SMs: split-K over every SM
+    (1024, 1024, 1024, 4, 1, True, 0),      # 16 pair tiles on 74 pairs
+    (2560, 640, 1024, 3, 1, True, 148),     # 200 tiles of 128 x 64: one full round, then 52 tiles
+    (128, 16384, 4096, 2, 1, True, 0),      # the skinny shape: 128 tiles on 148 SMs
+    (4000, 3000, 2050, 4, 1, True, 148),    # the ragged shape: 192 pair tiles, 44 in the last round
+    (8192, 16384, 4096, 4, 1, True, 1998),  # 2048 pair tiles = 27 rounds of 74 + 50
+    (700, 900, 333, 4, 1, False, 12),       # too few k-blocks to split
+    (16384, 1024, 8192, 4, 1, True, 222),   # the tall shape
 ])
-def test_plan_splits_only_a_short_last_round(M, N, K, config, split, full):
-    p = tg.plan(M, N, K, tg.TL_BF16, None, num_sms=148, config=config)
+def test_plan_splits_only_a_short_last_round(M, N, K, config, dtype, split, full):
+    from schedule_model import check_schedule
+    p = tg.plan(M, N, K, dtype, None, num_sms=148, config=config)
     tiles = p["tiles_m"] * p["tiles_n"]
-    assert p["split"] == split and p["full_tiles"] == full
-    units = 148 // p["cluster_ctas"]
-    items = p["full_tiles"] + (tiles - p["full_tiles"]) * p["split"]
-    assert p["grid"] == min(items, units) * p["cluster_ctas"]
-    if split > 1:
-        # every unit holds at most one part of the last round
-        assert (tiles - full) * split <= units and full % units == 0
-        assert p["workspace_bytes"] >= (tiles - full) * (split - 1) * p["cluster_ctas"] * 128 * p["block_n"] * 4
+    assert (p["split"] > 1) == split and p["full_tiles"] == (full if split else tiles)
+    parts = check_schedule(p, 148, K)
+    if split:
+        slabs = p["num_slots"] * p["cluster_ctas"]
+        assert p["workspace_bytes"] >= slabs * 128 * p["block_n"] * 4
+        assert parts <= 254  # the arrival count is 8 bits
     else:
         assert p["workspace_bytes"] == 0 or p["pad_a"] or p["pad_b"]
 
@@ -284,9 +281,13 @@ def test_host_fault_hook_is_valid_and_changes_no_plan():
     assert tg.tl_gemm_ex(P, P, 0, P, 8, 8, 8, 0, 0, 0, tg.Options(inject_fault=-1)) == tg.Status.INVALID_ARG
 
 
-def test_fault_hook_disables_the_split():
-    st, p = tg.tl_gemm_plan(P, P, 0, P, 1024, 1024, 2048, 0, 0, 148, tg.Options(config=1, inject_fault=1))
-    assert st == 0 and p.split == 1
+def test_fault_hook_plans_like_a_normal_call():
+    # the copy-skipping hook runs on the configuration the shape would use
+    # (CTA pairs included) with the same work split
+    for cfg in (0, 1, 4):
+        st, p = tg.tl_gemm_plan(P, P, 0, P, 1024, 1024, 2048, 0, 0, 148, tg.Options(config=cfg, inject_fault=1))
+        st0, p0 = tg.tl_gemm_plan(P, P, 0, P, 1024, 1024, 2048, 0, 0, 148, tg.Options(config=cfg))
+        assert st == 0 and st0 == 0 and p.as_dict() == p0.as_dict()
 
 
 def test_gelu_only_needs_no_bias_and_b_layout_is_validated():
@@ -367,11 +368,13 @@ def test_softmax_and_vector_add_validation():
 
 def test_plan_is_total_and_consistent_for_any_shape():
     """Every shape gets a configuration, and the plan is self-consistent: the
-    tiles cover C, the grid is at most one unit per SM (or pair) and at most
-    the work items, a split only cuts the last round, the shared memory fits
-    and the workspace holds the padded copies (property test over random
-    shapes, dtypes, epilogues and layouts)."""
+    tiles cover C, the grid is at most one unit per SM (or pair), a split
+    only cuts the last round and the kernel's schedule then computes every
+    k-block of every tile exactly once, the shared memory fits and the
+    workspace holds the padded copies (property test over random shapes,
+    dtypes, epilogues and layouts)."""
     from hypothesis import given, settings, strategies as st
+    from schedule_model import check_schedule
 
     @settings(max_examples=400, deadline=None)
     @given(M=st.integers(1, 70000), N=st.integers(1, 70000), K=st.integers(1, 70000),
@@ -387,10 +390,12 @@ def test_plan_is_total_and_consistent_for_any_shape():
         assert p.tiles_n * p.block_n >= N and (p.tiles_n - 1) * p.block_n < N
         tiles = p.tiles_m * p.tiles_n
         units = sms // p.cluster_ctas
-        items = p.full_tiles + (tiles - p.full_tiles) * p.split
-        assert 1 <= p.grid // p.cluster_ctas <= min(units, items) and p.grid % p.cluster_ctas == 0
+        assert 1 <= p.grid // p.cluster_ctas <= min(units, max(tiles, p.tail_units))
+        assert p.grid % p.cluster_ctas == 0
         assert p.split >= 1 and (p.split == 1) == (p.full_tiles == tiles)
         assert p.split == 1 or tiles - p.full_tiles < units  # only the short last round is split
+        if tiles <= 20000:
+            check_schedule(p.as_dict(), sms, K)  # every k-block of every tile exactly once
         assert p.smem_bytes <= 232448
         assert bool(p.direct_store) == (f32 or N % 8 != 0)  # base pointers here are 256-byte aligned
         need = 0
@@ -402,6 +407,31 @@ def test_plan_is_total_and_consistent_for_any_shape():
         assert p.workspace_bytes >= need
 
     check()
+
+
+def test_split_schedule_covers_every_k_block_once():
+    """For shapes of up to a few thousand tiles, with every configuration and
+    several unit counts, the schedule the kernel derives from the plan (the
+    index arithmetic of its unit_work / tail_contributors, restated in
+    tests/schedule_model.py) computes every k-block of every tile exactly
+    once, sums each shared tile over the units the kernel adds up, and keeps
+    partial-sum slots inside the workspace."""
+    from hypothesis import given, settings, strategies as st
+    from schedule_model import check_schedule
+    seen = {"split": 0}
+
+    @settings(max_examples=600, deadline=None)
+    @given(M=st.integers(1, 9000), N=st.integers(1, 9000), K=st.integers(1, 20000),
+           config=st.integers(0, tg.tl_num_configs()), sms=st.sampled_from([148, 132, 20, 8, 2]))
+    def check(M, N, K, config, sms):
+        s, p = tg.tl_gemm_plan(P, P, 0, P, M, N, K, 1, 0, sms, tg.Options(config=config))
+        assert s == 0
+        if p.tiles_m * p.tiles_n <= 20000:
+            if check_schedule(p.as_dict(), sms, K) > 1:
+                seen["split"] += 1
+
+    check()
+    assert seen["split"] > 50  # the split path was exercised
 
 
 def test_plan_from_many_threads_matches_one_thread():

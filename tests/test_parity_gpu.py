@@ -110,15 +110,18 @@ def test_every_config_vs_oracle(config, epi):
 
 
 SPLIT_CASES = [
-    # (M, N, K, config, dtype, epilogue): the tiles of a short last round are
-    # split along K and their partial sums added by the last part
-    (1024, 1024, 2048, 1, wl.BF16, wl.EPI_BIAS_GELU),   # 4 parts, single CTA
-    (1024, 1024, 1024, 4, wl.F16, wl.EPI_NONE),         # 4 parts, CTA pairs
-    (1280, 1536, 1024, 4, wl.BF16, wl.EPI_BIAS_GELU),   # 2 parts, CTA pairs
-    (1024, 1280, 1536, 4, wl.F16, wl.EPI_BIAS_GELU),    # 3 parts, CTA pairs
-    (2560, 640, 1024, 3, wl.BF16, wl.EPI_NONE),         # a full round, then 2 parts
-    (1000, 1000, 2000, 1, wl.F16, wl.EPI_BIAS_GELU),    # ragged M, N tails, 4 parts
-    (1001, 999, 2051, 4, wl.BF16, wl.EPI_BIAS_GELU),    # padded A and B, element stores, 4 parts
+    # (M, N, K, config, dtype, epilogue): the k-blocks of a short last round
+    # are spread over every unit; a tile shared by several units is summed by
+    # the last of them to finish
+    (1024, 1024, 2048, 1, wl.BF16, wl.EPI_BIAS_GELU),   # 32 tiles on 148 SMs, single CTA
+    (1024, 1024, 1024, 4, wl.F16, wl.EPI_NONE),         # 16 pair tiles on 74 pairs
+    (1280, 1536, 1024, 4, wl.BF16, wl.EPI_BIAS_GELU),   # 30 pair tiles
+    (1024, 1280, 1536, 4, wl.F16, wl.EPI_BIAS_GELU),    # 20 pair tiles
+    (2560, 640, 1024, 3, wl.BF16, wl.EPI_NONE),         # a full round, then 52 tiles
+    (1000, 1000, 2000, 1, wl.F16, wl.EPI_BIAS_GELU),    # ragged M, N tails
+    (1001, 999, 2051, 4, wl.BF16, wl.EPI_BIAS_GELU),    # padded A and B, element stores
+    (128, 4096, 4096, 2, wl.BF16, wl.EPI_BIAS_GELU),    # skinny: 32 tiles over 148 SMs, 4 or 5 parts each
+    (4000, 3000, 2050, 4, wl.BF16, wl.EPI_NONE),        # the ragged workload's shape: 44 tiles in the last round
 ]
 
 
@@ -314,6 +317,35 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     compare(C, ref, wl.F16, accumulation_bound(A, B, None, wl.F16, 0, ref))
 
 
+@pytest.mark.parametrize("config", ALL_CONFIGS)
+def test_fault_hook_on_every_config_drains_and_context_survives(config):
+    """Every producer (with a CTA pair, both CTAs' producers) skips the same
+    stage without issuing its copies: the MMA warp's wait on that stage runs
+    out, the kernel records it, drains the copies it did issue -- the even
+    CTA of a pair waits on its barriers for both CTAs' copies -- frees Tensor
+    Memory and returns.  Bit 1 is set and the drain bit is clear; the next
+    calls on the same context, with and without a split last round, are
+    right."""
+    import tensor_core_gemm_tl_b200 as m
+    stream = torch.cuda.current_stream().cuda_stream
+    for M, N, K in ((512, 512, 1024), (1024, 1024, 2048)):
+        A, B, bias = inputs(M, N, K, wl.BF16, wl.EPI_BIAS_GELU, seed=config)
+        dA, dB, db = to_device(A, wl.BF16), to_device(B, wl.BF16), to_device(bias, wl.BF16)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        opt = m.Options(config=config, inject_fault=1, timeout_ns=100_000_000)
+        st = m.tl_gemm_ex(dA.data_ptr(), dB.data_ptr(), db.data_ptr(), out.data_ptr(), M, N, K, wl.BF16,
+                          wl.EPI_BIAS_GELU, stream, opt)
+        assert st == 0
+        st, word = m.tl_check_device(stream)
+        assert st == int(m.Status.DEVICE_TIMEOUT)
+        assert word & 2, word          # the MMA warp's wait on data gave up
+        assert not (word & 16), word   # every issued copy and MMA drained in time
+        assert not (word & 128), word
+        ref = oracle.gemm(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU)
+        C = run_library(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU, config=config)
+        compare(C, ref, wl.BF16, accumulation_bound(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU, ref))
+
+
 def test_host_side_encode_failure_is_reported_and_nothing_runs():
     """The host treats A's tensor-map encode as failed (test hook 2): the call
     returns TL_ERR_CUDA before any kernel is launched, C is untouched, no device
@@ -336,6 +368,73 @@ def test_host_side_encode_failure_is_reported_and_nothing_runs():
 
 
 # ------------------------------------------------------------------ concurrent callers
+def test_split_gemms_on_concurrent_streams_never_wait_on_each_other():
+    """No part of a split tile waits for another unit, so GEMMs whose last
+    round is split can share the GPU with anything: two split GEMMs launched
+    together on two streams, a split GEMM launched while a long plain GEMM
+    holds every SM, and a split GEMM through tl_gemm_noalloc beside one
+    through tl_gemm.  Each returns TL_OK with no device error, matches the
+    oracle, and equals bit for bit the same call made alone."""
+    import tensor_core_gemm_tl_b200 as m
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cases = [(1024, 1024, 2048, 1, wl.BF16, wl.EPI_BIAS_GELU), (1280, 1536, 1024, 4, wl.F16, wl.EPI_NONE)]
+    bufs = []
+    for M, N, K, config, dt, epi in cases:
+        assert m.plan(M, N, K, dt, "bias_gelu" if epi else None, num_sms=sms, config=config)["split"] > 1
+        A, B, bias = inputs(M, N, K, dt, epi, seed=M + K)
+        dA, dB = to_device(A, dt), to_device(B, dt)
+        db = to_device(bias, dt) if bias is not None else None
+        ref = oracle.gemm(A, B, bias, dt, epi)
+        alone = run_library(A, B, bias, dt, epi, config=config)
+        compare(alone, ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
+        bufs.append((M, N, K, config, dt, epi, dA, dB, db, alone))
+    big = torch.randn(8192, 8192, device="cuda").to(torch.bfloat16)
+    big_out = torch.empty_like(big)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def launch(case, stream, entry="ex"):
+        M, N, K, config, dt, epi, dA, dB, db, _ = case
+        out = torch.empty((M, N), dtype=torch.float16 if dt == wl.F16 else torch.bfloat16, device="cuda")
+        bp = db.data_ptr() if db is not None else 0
+        if entry == "noalloc":
+            st = m.tl_gemm_noalloc(dA.data_ptr(), dB.data_ptr(), bp, out.data_ptr(), M, N, K, dt, epi,
+                                   stream.cuda_stream)
+        else:
+            st = m.tl_gemm_ex(dA.data_ptr(), dB.data_ptr(), bp, out.data_ptr(), M, N, K, dt, epi, stream.cuda_stream,
+                              m.Options(config=config))
+        assert st == 0, m.tl_status_string(st)
+        return out
+
+    def bits(t):
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+    for rep in range(3):
+        torch.cuda.synchronize()
+        # two split GEMMs at once
+        o1, o2 = launch(bufs[0], s1), launch(bufs[1], s2)
+        # a split GEMM behind a long GEMM that fills every SM
+        with torch.cuda.stream(s1):
+            t = tg()
+            t.gemm(big, big, out=big_out, stream=s1)
+        o3 = launch(bufs[0], s2)
+        # the allocation-free entry point beside tl_gemm (separate workspaces)
+        M, N, K, config, dt, epi = cases[0][:6]
+        if m.plan(M, N, K, dt, "bias_gelu", num_sms=sms)["split"] > 1:
+            o4 = launch(bufs[0], s1, "noalloc")
+            o5 = launch(bufs[0], s2, "ex")
+        else:
+            o4 = o5 = None
+        torch.cuda.synchronize()
+        assert t.check_device() == 0
+        assert np.array_equal(bits(o1), bufs[0][-1]) and np.array_equal(bits(o3), bufs[0][-1])
+        assert np.array_equal(bits(o2), bufs[1][-1])
+        if o4 is not None:
+            assert np.array_equal(bits(o5), bufs[0][-1])
+            ref = oracle.gemm(*inputs(M, N, K, dt, epi, seed=M + K), dt, epi)
+            compare(bits(o4), ref, dt)
+
+
+
 def test_concurrent_calls_from_threads_on_their_own_streams():
     """Eight threads call the library at once, each on a stream of its own
     (ctypes releases the GIL for every call): GEMMs that take the padded-copy
