@@ -396,7 +396,7 @@ class _NullCtx:
         return False
 
 
-def per_config_entry(w, bench, ms, warm_ms, peaks):
+def per_config_entry(w, bench, ms, warm_ms, peaks, clocks):
     tflops = w.flops / (ms / 1e3) / 1e12
     gbs = w.min_bytes() / (ms / 1e3) / 1e9
     peak, peak_name = tensor_peak(peaks, 0.0)
@@ -406,7 +406,8 @@ def per_config_entry(w, bench, ms, warm_ms, peaks):
          "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4), "bound": bound,
          "warm_l2_tflops": round(w.flops / (warm_ms / 1e3) / 1e12, 2),
          "kernel_config": bench.plan["config_name"], "split": bench.plan["split"],
-         "launches_per_step": bench.launches_per_step}
+         "launches_per_step": bench.launches_per_step, "sm_mhz": clocks["sm_mhz"],
+         "reasons": clocks["reasons"]}
     # the roofline fraction of the bound that applies
     e["roofline_frac"] = e["frac_hbm"] if bound == "hbm" else e["frac"]
     return e
@@ -450,6 +451,27 @@ def run_gpu(args, w):
         roof.update({"achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
                      "peak_source": f"{peak_src} {peak_name} (cuBLAS; a region under "
                                     f"{SUSTAINED_REGION_S:g} s is a burst); fp16 dense rate equals bf16"})
+
+    # ---------------------------------------------------------------- every configuration, as a burst
+    per_config = {}
+    if not args.no_per_config:
+        for name in PER_CONFIG:
+            wc = wl.WORKLOADS[name]
+            b = head if name == w.name else GemmBench(wc, dev, args.seed, tg)
+            # each region starts after an idle pause, so that it runs at the
+            # unthrottled clock like the headline burst
+            time.sleep(args.rest_s)
+            cs = ClockSampler(local)
+            ms = max_over_ranks(timed_region(b, stream, K, args.warmup, args.ramp_s, sampler=cs, dist=dist),
+                                dist, dev) / K
+            time.sleep(args.rest_s)
+            warm_ms = max_over_ranks(timed_region(b, stream, K, args.warmup, args.ramp_s, rotate=False, dist=dist),
+                                     dist, dev) / K
+            per_config[name] = per_config_entry(wc, b, ms, warm_ms, peaks, cs.summary())
+            if b is not head:
+                b.free()
+                del b
+            torch.cuda.empty_cache()
 
     # ---------------------------------------------------------------- end to end through the public API
     # Every step copies its inputs from pinned host memory, runs the GEMM and
@@ -499,22 +521,6 @@ def run_gpu(args, w):
     h2d = 2 * (w.M * w.K + w.K * w.N) + (2 * w.N if head.bias_bits is not None else 0)
     d2h = 2 * w.M * w.N
     del lanes, A_h, B_h, b_h
-
-    # ---------------------------------------------------------------- every configuration, as a burst
-    per_config = {}
-    if not args.no_per_config:
-        for name in PER_CONFIG:
-            wc = wl.WORKLOADS[name]
-            b = head if name == w.name else GemmBench(wc, dev, args.seed, tg)
-            time.sleep(args.rest_s)  # let the power controller settle between bursts
-            ms = max_over_ranks(timed_region(b, stream, K, args.warmup, args.ramp_s, dist=dist), dist, dev) / K
-            warm_ms = max_over_ranks(timed_region(b, stream, K, args.warmup, 0.0, rotate=False, dist=dist),
-                                     dist, dev) / K
-            per_config[name] = per_config_entry(wc, b, ms, warm_ms, peaks)
-            if b is not head:
-                b.free()
-                del b
-            torch.cuda.empty_cache()
 
     # ---------------------------------------------------------------- the headline, sustained
     sustained = None
@@ -593,9 +599,9 @@ def parse(argv=None):
     ap.add_argument("--workload", default=wl.HEADLINE, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--impl", default="tl_gemm", choices=["tl_gemm", "reference"])
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--ramp-s", type=float, default=0.05,
+    ap.add_argument("--ramp-s", type=float, default=0.01,
                     help="untimed back-to-back launches before the warm-up steps (brings the SM clock up)")
-    ap.add_argument("--rest-s", type=float, default=0.5, help="idle time before each per-configuration burst")
+    ap.add_argument("--rest-s", type=float, default=1.5, help="idle time before each per-configuration burst")
     ap.add_argument("--sustained-s", type=float, default=3.0,
                     help="length of the sustained (power-capped) run of the headline; 0 skips it")
     ap.add_argument("--e2e-steps", type=int, default=20)

@@ -253,6 +253,10 @@ typedef struct {
                              1: C is float32, the epilogue's fp32 result itself
                              (4-byte aligned; 16-byte aligned rows take vector
                              stores).  C is then stored without the TMA unit.  */
+    int32_t raster_group; /* output-tile rows per rasterisation group (tiles are
+                             visited column by column inside a group of this
+                             many tile rows, so that the tiles running together
+                             share operands in L2); 0: the library's choice     */
 } tl_gemm_options;
 
 /* tl_gemm with options (NULL options == tl_gemm).  Same arguments and errors;
@@ -305,6 +309,8 @@ typedef struct {
                                 order                                           */
     int32_t num_slots;       /* partial-sum slots in the workspace (slot u + r:
                                 unit u's part of last-round tile r)             */
+    int32_t raster_group;    /* output-tile rows per rasterisation group       */
+    int32_t reserved;        /* 0                                              */
 } tl_plan;
 
 TL_API tl_status tl_gemm_plan(const void *A, const void *B, const void *bias, void *C,

@@ -66,7 +66,7 @@ def _epi_code(epilogue):
 
 
 def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0, timeout_ns: int = 0,
-         no_split: bool = False, b_transposed: bool = False, out_dtype=None):
+         no_split: bool = False, b_transposed: bool = False, out_dtype=None, raster_group: int = 0):
     """C = epilogue(A @ B) for row-major CUDA tensors A (M x K) and B (K x N),
     or B given as N x K (``b_transposed=True``: C = epilogue(A @ B.T), the
     layout of a linear layer's weight).
@@ -78,7 +78,8 @@ def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0,
     epilogue's fp32 result without rounding to 16 bits.  ``out`` (M x N) is
     written if given, else allocated.  Runs asynchronously on ``stream``
     (default: torch's current stream).  ``config`` = k > 0 forces kernel
-    configuration k - 1.
+    configuration k - 1; ``raster_group`` > 0 sets the output-tile rows per
+    rasterisation group.
     """
     import torch
     epi = _epi_code(epilogue if epilogue is not None else ("bias_gelu" if bias is not None else None))
@@ -111,9 +112,9 @@ def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0,
     s = stream if stream is not None else torch.cuda.current_stream(A.device)
     bias_ptr = bias.data_ptr() if bias is not None and epi in TL_EPI_WITH_BIAS else 0
     with torch.cuda.device(A.device):
-        if config or timeout_ns or no_split or b_transposed or c_f32:
+        if config or timeout_ns or no_split or b_transposed or c_f32 or raster_group:
             opt = Options(config=config, inject_fault=0, timeout_ns=timeout_ns, no_split=int(no_split),
-                          b_layout=int(bool(b_transposed)), c_float32=int(c_f32))
+                          b_layout=int(bool(b_transposed)), c_float32=int(c_f32), raster_group=raster_group)
             st = tl_gemm_ex(A.data_ptr(), B.data_ptr(), bias_ptr, out.data_ptr(), M, N, K, dt, epi,
                             s.cuda_stream, opt)
         else:

@@ -39,10 +39,11 @@ class Options(ctypes.Structure):
     """tl_gemm_options: config (0 = library's choice, k = configuration k-1),
     inject_fault (test hook: 1 device-side stall, 2 host-side encode failure), timeout_ns (0 = 10 s), no_split (1 = never split
     the tiles of a short last round), b_layout (1 = B given as N x K),
-    c_float32 (1 = C is float32)."""
+    c_float32 (1 = C is float32), raster_group (tile rows per rasterisation
+    group, 0 = library's choice)."""
     _fields_ = [("config", ctypes.c_int32), ("inject_fault", ctypes.c_int32),
                 ("timeout_ns", ctypes.c_uint64), ("no_split", ctypes.c_int32), ("b_layout", ctypes.c_int32),
-                ("c_float32", ctypes.c_int32)]
+                ("c_float32", ctypes.c_int32), ("raster_group", ctypes.c_int32)]
 
 
 class Plan(ctypes.Structure):
@@ -53,7 +54,8 @@ class Plan(ctypes.Structure):
                 ("split", ctypes.c_int32), ("full_tiles", ctypes.c_int32), ("pad_a", ctypes.c_int32),
                 ("pad_b", ctypes.c_int32), ("direct_store", ctypes.c_int32),
                 ("smem_bytes", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64),
-                ("tail_units", ctypes.c_int32), ("num_slots", ctypes.c_int32)]
+                ("tail_units", ctypes.c_int32), ("num_slots", ctypes.c_int32),
+                ("raster_group", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}

@@ -142,13 +142,14 @@ def compare_attention(B, H, Sq, Sk, D, causal, launches=20, warmup=5):
 ROWWISE_SHAPES = [(16384, 8192), (65536, 1024), (4096, 50257), (262144, 128)]
 
 
-def compare_rowwise(launches=20, warmup=5):
+def compare_rowwise(launches=20, warmup=5, shapes=ROWWISE_SHAPES, vector_n=1 << 28):
     """Achieved HBM bandwidth (compulsory bytes / time) of the row softmax and
-    the vector add against torch.softmax and torch.add."""
+    the vector add against torch.softmax and torch.add (vector_n = 0 skips
+    the vector add)."""
     import torch
     import tensor_core_gemm_tl_b200 as tg
     out = []
-    for rows, cols in ROWWISE_SHAPES:
+    for rows, cols in shapes:
         x = torch.randn(rows, cols, device="cuda", dtype=torch.bfloat16)
         y = torch.empty_like(x)
         nbytes = 2 * 2 * rows * cols
@@ -162,7 +163,11 @@ def compare_rowwise(launches=20, warmup=5):
         out.append({"softmax": f"{rows}x{cols} bf16",
                     "tl_gbs": round(nbytes / _median_ms(ours, 1, launches, warmup) / 1e6, 1),
                     "torch_gbs": round(nbytes / _median_ms(ref, 1, launches, warmup) / 1e6, 1)})
-    n = 1 << 28
+    n = vector_n
+    if n <= 0:
+        if tg.check_device() != 0:
+            raise RuntimeError("device error")
+        return out
     a = torch.randn(n, device="cuda")
     b = torch.randn(n, device="cuda")
     c = torch.empty_like(a)
@@ -188,6 +193,9 @@ def main(argv=None):
     ap.add_argument("--launches", type=int, default=40)
     ap.add_argument("--attention", action="store_true", help="time attention forward instead of the GEMMs")
     ap.add_argument("--rowwise", action="store_true", help="time the row softmax and the vector add")
+    ap.add_argument("--rowwise-shapes", default=None,
+                    help="comma-separated ROWSxCOLS softmax shapes (default: the four standard ones)")
+    ap.add_argument("--vector-n", type=int, default=1 << 28, help="vector add length (0: skip it)")
     a = ap.parse_args(argv)
     import torch
     torch.cuda.set_device(0)
@@ -196,7 +204,10 @@ def main(argv=None):
             print(json.dumps(compare_attention(*shape)), flush=True)
         return 0
     if a.rowwise:
-        for rec in compare_rowwise():
+        shapes = ROWWISE_SHAPES
+        if a.rowwise_shapes is not None:
+            shapes = [tuple(int(v) for v in x.split("x")) for x in a.rowwise_shapes.split(",") if x]
+        for rec in compare_rowwise(launches=min(a.launches, 20), shapes=shapes, vector_n=a.vector_n):
             print(json.dumps(rec), flush=True)
         return 0
     todo = list(wl.WORKLOADS.values())

@@ -100,7 +100,7 @@ struct GemmParams {
     // waits for another.
     int32_t full_tiles, tail_tiles, tail_units;
     int32_t num_slots;       // partial-sum slots in the workspace (tail_units + tail_tiles - 1)
-    float *partials;         // [slot][cta of the pair][128 rows][BN columns] fp32
+    float *partials;         // [slot][cta of the pair][lane quarter][64-column chunk][16 float4][32 lanes]
     unsigned long long *arrivals;  // [tail tile][cta][lane quarter][64-column chunk]
     unsigned long long epoch;  // unique per launch, below 2^56
 };
@@ -662,19 +662,23 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                 if (shared_tile) {
                     // This chunk's fp32 partial sums go to this unit's slot; the
                     // part that arrives last on the chunk's word adds all the
-                    // parts in k order (first .. last unit) and stores C.
-                    const size_t slab_elems = static_cast<size_t>(CF::BM) * CF::BN;
-                    const size_t row_off = (static_cast<size_t>(q) * 32 + lane) * CF::BN + c * 64;
-                    auto slab_of = [&](int u) {
-                        return static_cast<size_t>(u + w.tail) * CF::CTAS + rank;  // slot u + r is unique per (unit, tail tile)
+                    // parts in k order (first .. last unit) and stores C.  A
+                    // slot holds each warp's chunk as 16 float4 columns of 32
+                    // lanes, so every access below is 512 contiguous bytes.
+                    const size_t slab_f4 = static_cast<size_t>(CF::BM) * CF::BN / 4;
+                    const size_t chunk_off = ((static_cast<size_t>(q) * CHUNKS + c) * 16) * 32 + lane;
+                    auto slot_f4 = [&](int u) {
+                        // slot u + r is unique per (unit, tail tile)
+                        return reinterpret_cast<float4 *>(p.partials) +
+                               (static_cast<size_t>(u + w.tail) * CF::CTAS + rank) * slab_f4 + chunk_off;
                     };
-                    if (!check_ok(slab_of(t_last) < static_cast<size_t>(p.num_slots) * CF::CTAS))
+                    if (!check_ok(static_cast<size_t>(t_last + w.tail) < static_cast<size_t>(p.num_slots)))
                         continue;  // outside the workspace
-                    float4 *mine = reinterpret_cast<float4 *>(p.partials + slab_of(unit) * slab_elems + row_off);
+                    float4 *mine = slot_f4(unit);
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        __stcg(mine + i, make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                                     __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
+                        __stcg(mine + 32 * i, make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                          __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
                     __threadfence();
                     __syncwarp();
                     unsigned count = 0;
@@ -686,27 +690,37 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                     if (count != static_cast<unsigned>(t_last - t_first + 1))
                         continue;  // an earlier arrival: the last part stores this chunk
                     __threadfence();
+                    // sum = part(first) + part(first + 1) + ... + part(last), this
+                    // unit's own part read back like the others; 8 loads in
+                    // flight per batch
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-                        for (int u = t_first; u <= t_last; ++u) {
-                            const float4 b = u == unit ? make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                                                     __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]))
-                                                       : __ldcg(reinterpret_cast<const float4 *>(
-                                                                    p.partials + slab_of(u) * slab_elems + row_off) + i);
-                            if (u == t_first) {
-                                a = b;
-                            } else {
-                                a.x += b.x;
-                                a.y += b.y;
-                                a.z += b.z;
-                                a.w += b.w;
+                    for (int h = 0; h < 2; ++h) {
+                        float4 acc[8];
+                        const float4 *src = slot_f4(t_first) + 32 * 8 * h;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            acc[i] = __ldcg(src + 32 * i);
+                        for (int u = t_first + 1; u <= t_last; ++u) {
+                            const float4 *su = slot_f4(u) + 32 * 8 * h;
+                            float4 b[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                b[i] = __ldcg(su + 32 * i);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                acc[i].x += b[i].x;
+                                acc[i].y += b[i].y;
+                                acc[i].z += b[i].z;
+                                acc[i].w += b[i].w;
                             }
                         }
-                        r[4 * i] = __float_as_uint(a.x);
-                        r[4 * i + 1] = __float_as_uint(a.y);
-                        r[4 * i + 2] = __float_as_uint(a.z);
-                        r[4 * i + 3] = __float_as_uint(a.w);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            r[32 * h + 4 * i] = __float_as_uint(acc[i].x);
+                            r[32 * h + 4 * i + 1] = __float_as_uint(acc[i].y);
+                            r[32 * h + 4 * i + 2] = __float_as_uint(acc[i].z);
+                            r[32 * h + 4 * i + 3] = __float_as_uint(acc[i].w);
+                        }
                     }
                 }
 
@@ -886,30 +900,76 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
     }
 }
 
-// Zero-padded copy of a rows x cols matrix of 16-bit values (any alignment of
-// `src`) into dst with a row length of dst_cols (a multiple of 8) and a
-// 16-byte-aligned base: each thread writes 8 values (16 bytes) at a time.
+// Zero-padded copy of a rows x cols matrix of 16-bit values (any 2-byte
+// aligned `src`) into dst with a row length of dst_cols (a multiple of 8) and
+// a 16-byte-aligned base.  One warp per row: lane l reads the l-th 16-byte
+// word of the row's aligned span (512 contiguous bytes per warp step), takes
+// the next word from lane l + 1 and shifts the pair into place, so every
+// global access is a whole aligned 16-byte word.  A word is read only when it
+// holds at least one byte of the row (it then lies in memory the row's
+// allocation covers); bytes past `cols` are written as zero.
+__device__ __forceinline__ uint32_t shift_pair(uint32_t lo, uint32_t hi, uint32_t byte_shift)
+{
+    return __funnelshift_r(lo, hi, 8u * byte_shift);
+}
+
 __global__ void __launch_bounds__(256) pad_copy_kernel(const uint16_t *__restrict__ src, int64_t rows,
                                                        int64_t cols, uint16_t *__restrict__ dst,
                                                        int64_t dst_cols)
 {
-    const int64_t chunks_per_row = dst_cols >> 3;
-    const int64_t total = rows * chunks_per_row;
-    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
-         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t r = idx / chunks_per_row;
-        const int64_t c0 = (idx - r * chunks_per_row) << 3;
-        const uint16_t *s = src + r * cols;
-        uint16_t e[8];
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    const int64_t chunks = dst_cols >> 3;  // 16-byte words of a destination row
+    for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+        const uintptr_t row_begin = reinterpret_cast<uintptr_t>(src + r * cols);
+        const uintptr_t row_end = row_begin + static_cast<uintptr_t>(cols) * 2;
+        const uintptr_t base = row_begin & ~static_cast<uintptr_t>(15);
+        const uint32_t mis = static_cast<uint32_t>(row_begin - base);  // 0, 2, ..., 14
+        uint4 *drow = reinterpret_cast<uint4 *>(dst + r * dst_cols);
+        for (int64_t c0 = 0; c0 < chunks; c0 += 32) {
+            const int64_t c = c0 + lane;
+            // the aligned word at base + 16 c, if any byte of it is in the row
+            // (also for c == chunks: its first bytes can end chunk c - 1)
+            const uintptr_t wa = base + 16 * static_cast<uintptr_t>(c);
+            uint4 lo = make_uint4(0u, 0u, 0u, 0u);
+            if (wa < row_end)
+                lo = __ldg(reinterpret_cast<const uint4 *>(wa));
+            uint4 hi;
+            hi.x = __shfl_down_sync(0xffffffffu, lo.x, 1);
+            hi.y = __shfl_down_sync(0xffffffffu, lo.y, 1);
+            hi.z = __shfl_down_sync(0xffffffffu, lo.z, 1);
+            hi.w = __shfl_down_sync(0xffffffffu, lo.w, 1);
+            if (lane == 31) {
+                hi = make_uint4(0u, 0u, 0u, 0u);
+                if (mis != 0 && wa + 16 < row_end)
+                    hi = __ldg(reinterpret_cast<const uint4 *>(wa + 16));
+            }
+            if (c >= chunks)
+                continue;
+            // bytes [mis, mis + 16) of lo:hi
+            const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+            const uint32_t q = mis >> 2, b = mis & 3u;
+            uint32_t o[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            e[i] = (c0 + i < cols) ? s[c0 + i] : static_cast<uint16_t>(0);
-        uint4 w;
-        w.x = e[0] | (static_cast<uint32_t>(e[1]) << 16);
-        w.y = e[2] | (static_cast<uint32_t>(e[3]) << 16);
-        w.z = e[4] | (static_cast<uint32_t>(e[5]) << 16);
-        w.w = e[6] | (static_cast<uint32_t>(e[7]) << 16);
-        *reinterpret_cast<uint4 *>(dst + r * dst_cols + c0) = w;
+            for (int k = 0; k < 4; ++k) {
+                // words q + k and q + k + 1 of w, selected without dynamic indexing
+                uint32_t a0 = w[k], a1 = w[k + 1];
+                if (q == 1) { a0 = w[k + 1]; a1 = w[k + 2]; }
+                if (q == 2) { a0 = w[k + 2]; a1 = w[k + 3]; }
+                if (q == 3) { a0 = w[k + 3]; a1 = w[k + 4]; }
+                o[k] = b ? shift_pair(a0, a1, b) : a0;
+            }
+            // zero the values at or past `cols`
+            const int64_t e0 = 8 * c;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (e0 + 2 * k >= cols)
+                    o[k] = 0u;
+                else if (e0 + 2 * k + 1 >= cols)
+                    o[k] &= 0xFFFFu;
+            }
+            drow[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
     }
 }
 

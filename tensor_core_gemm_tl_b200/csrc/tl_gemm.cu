@@ -25,6 +25,7 @@ namespace tl {
 namespace {
 
 constexpr uint64_t kDefaultTimeoutNs = 10ull * 1000 * 1000 * 1000;
+constexpr int kDefaultRasterGroup = 8;  // output-tile rows per rasterisation group
 
 using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
 
@@ -93,6 +94,7 @@ struct TableRow {
     int dtype, epi;
     const char *config;
     int split;  // 1: split the tiles of a short last round; 0: never
+    int group;  // output-tile rows per rasterisation group (0: the default)
 };
 const TableRow kTable[] = {
 #include "config_table.inc"
@@ -135,18 +137,20 @@ int model_config(int64_t M, int64_t N, int num_sms)
 // The measured choice for this shape (configuration, and whether its last
 // round may be cut along K), else the wave model with the split rule of
 // tail_split.
-int choose_config(int64_t M, int64_t N, int64_t K, int dtype, int epi, int num_sms, bool *split)
+int choose_config(int64_t M, int64_t N, int64_t K, int dtype, int epi, int num_sms, bool *split, int *group)
 {
     for (const TableRow &r : kTable) {
         if (r.m == M && r.n == N && r.k == K && r.dtype == dtype && r.epi == (epi != 0 ? 1 : 0)) {
             const int i = config_index(r.config);
             if (i >= 0) {
                 *split = r.split != 0;
+                *group = r.group;
                 return i;
             }
         }
     }
     *split = true;
+    *group = 0;
     return model_config(M, N, num_sms);
 }
 
@@ -203,7 +207,7 @@ tl_status validate(const void *A, const void *B, const void *bias, void *C, int6
     if (opt && (opt->inject_fault < 0 || opt->inject_fault > 2))
         return TL_ERR_INVALID_ARG;
     if (opt && ((opt->no_split != 0 && opt->no_split != 1) || (opt->b_layout != 0 && opt->b_layout != 1) ||
-                (opt->c_float32 != 0 && opt->c_float32 != 1)))
+                (opt->c_float32 != 0 && opt->c_float32 != 1) || opt->raster_group < 0))
         return TL_ERR_INVALID_ARG;
     const int64_t lim = 0x7FFFFFFFll;
     if (M > lim || N > lim || K > lim)
@@ -266,7 +270,9 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
     if (num_sms <= 0)
         return TL_ERR_INVALID_ARG;
     bool table_split = true;  // a forced configuration splits unless told not to
-    int ci = (opt && opt->config > 0) ? opt->config - 1 : choose_config(M, N, K, dtype, epi, num_sms, &table_split);
+    int table_group = 0;
+    int ci = (opt && opt->config > 0) ? opt->config - 1
+                                      : choose_config(M, N, K, dtype, epi, num_sms, &table_split, &table_group);
     const ConfigEntry &c = kConfigs[ci];
     Plan p{};
     tl_plan &q = p.pub;
@@ -332,6 +338,10 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
         ws += ceil_div(ts.tail_tiles * c.ctas * 4 * (c.bn / 64) * 8, 256) * 256;
     }
     q.workspace_bytes = ws;
+    int group = (opt && opt->raster_group > 0) ? opt->raster_group : (table_group > 0 ? table_group : kDefaultRasterGroup);
+    if (group > q.tiles_m)
+        group = q.tiles_m;
+    q.raster_group = group;
     *out = p;
     return TL_OK;
 }
@@ -457,8 +467,8 @@ tl_status max_active_clusters(DeviceState *d, KernelFn fn, const cudaLaunchConfi
 tl_status launch_pad(const void *src, int64_t rows, int64_t cols, void *dst, int64_t dst_cols, int num_sms,
                      cudaStream_t stream)
 {
-    const int64_t work = rows * (dst_cols / 8);
-    int64_t blocks = ceil_div(work, 256);
+    // one warp per row, eight rows per block
+    int64_t blocks = ceil_div(rows, 8);
     const int64_t cap = static_cast<int64_t>(num_sms) * 8;
     if (blocks > cap)
         blocks = cap;
@@ -523,7 +533,7 @@ tl_status launch_gemm(const Plan &p, const void *A, const void *B, const void *b
     gp.tiles_n = p.pub.tiles_n;
     gp.num_tiles = p.pub.tiles_m * p.pub.tiles_n;
     gp.num_kb = static_cast<int32_t>(ceil_div(K, c.bk));
-    gp.group_m = 8;
+    gp.group_m = p.pub.raster_group;
     gp.bias = static_cast<const uint16_t *>(bias);
     gp.bias_vec16 = bias && aligned(bias, 16);
     gp.epi_bias = epi_has_bias(epi);
