@@ -679,17 +679,19 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                     for (int i = 0; i < 16; ++i)
                         __stcg(mine + 32 * i, make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
                                                           __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
-                    __threadfence();
+                    // the warp's writes, then one release by lane 0 (the warp
+                    // barrier orders the other lanes' writes before it)
                     __syncwarp();
                     unsigned count = 0;
                     if (lane == 0) {
                         const size_t word = ((static_cast<size_t>(w.tail) * CF::CTAS + rank) * 4 + q) * CHUNKS + c;
+                        fence_acq_rel_gpu();
                         count = arrive_tagged(p.arrivals + word, p.epoch);
                     }
                     count = __shfl_sync(0xffffffffu, count, 0);
                     if (count != static_cast<unsigned>(t_last - t_first + 1))
                         continue;  // an earlier arrival: the last part stores this chunk
-                    __threadfence();
+                    __syncwarp();  // lane 0's acquire orders the reads below
                     // sum = part(first) + part(first + 1) + ... + part(last), this
                     // unit's own part read back like the others; 8 loads in
                     // flight per batch

@@ -72,6 +72,11 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
     return v;
 }
 
+__device__ __forceinline__ void fence_acq_rel_gpu()
+{
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 // Compare-and-swap with acquire-release semantics at GPU scope; returns the
 // value found at `addr`.
 __device__ __forceinline__ unsigned long long atom_cas_acq_rel_u64(unsigned long long *addr, unsigned long long cmp,

@@ -110,22 +110,72 @@ int config_index(const char *name)
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Model for shapes the sweep has not measured: time ~ waves x tile width,
-// with narrower tiles running the tensor pipe less efficiently (they read
-// more shared memory per MMA flop).
-int model_config(int64_t M, int64_t N, int num_sms)
+// How the tiles of one launch are cut into work items.  Tiles fill whole
+// rounds of `units` (CTAs, or CTA pairs) first.  The tiles of a last, partial
+// round would leave units idle for a whole tile's time; instead their
+// k-blocks can be spread evenly over the units, each unit taking one
+// consecutive range (which may end inside the next tile).  A tile whose
+// k-blocks fall to several units is summed by the last of them to finish (see
+// the kernel): nobody waits, so nothing depends on all units being resident.
+// The split is taken when it saves at least max(4, num_kb / 8) k-blocks of
+// the last round's time -- below that the partial sums' traffic and the extra
+// epilogue pass eat the gain -- and every unit then gets at least 4 k-blocks.
+struct TailSplit {
+    int64_t full_tiles, tail_tiles, tail_units;
+    int32_t max_parts;  // most units sharing one tile (1: none shared)
+};
+
+TailSplit tail_split(int64_t tiles, int64_t units, int64_t num_kb, bool allow)
 {
-    // relative tensor-pipe efficiency of each configuration when it has enough
-    // tiles (operand bytes each SM must pull per MMA flop)
-    static const double eff[] = {0.62, 0.5, 0.33, 0.95, 0.7};
+    TailSplit t{tiles, 0, 0, 1};
+    const int64_t rem = tiles % units;
+    if (!allow || rem == 0 || num_kb < 8)
+        return t;
+    const int64_t T = rem * num_kb;
+    const int64_t tail_units = units < T / 4 ? units : T / 4;
+    if (tail_units <= rem)
+        return t;
+    const int64_t saved = num_kb - (T + tail_units - 1) / tail_units;
+    const int64_t need = num_kb / 8 > 4 ? num_kb / 8 : 4;
+    if (saved < need)
+        return t;
+    t.full_tiles = tiles - rem;
+    t.tail_tiles = rem;
+    t.tail_units = tail_units;
+    // units meeting tail tile r: ceil((x + 1) U / T) - 1 for its first and last k-block x
+    for (int64_t r = 0; r < rem; ++r) {
+        const int64_t first = ((r * num_kb + 1) * tail_units + T - 1) / T - 1;
+        const int64_t last = (((r + 1) * num_kb) * tail_units + T - 1) / T - 1;
+        if (last - first + 1 > t.max_parts)
+            t.max_parts = static_cast<int32_t>(last - first + 1);
+    }
+    return t;
+}
+
+// Model for shapes the sweep has not measured: the busiest unit's time, in
+// tiles of each configuration weighted by its measured relative tensor-pipe
+// efficiency (narrower tiles pull more operand bytes per MMA flop into each
+// SM).  Whole rounds of tiles count fully; a split last round counts as the
+// k-blocks each unit then takes plus two k-blocks for the partial sums; a
+// partial round that is not split counts as a whole one.
+int model_config(int64_t M, int64_t N, int64_t K, int num_sms)
+{
+    // bm128_bn256, bm128_bn128, bm128_bn64, pair 256 x 256, pair 256 x 128
+    static const double eff[] = {0.86, 0.67, 0.36, 0.95, 0.68};
     int best = 0;
     double best_cost = 1e300;
     for (int i = 0; i < num_configs(); ++i) {
         const ConfigEntry &c = kConfigs[i];
         const int64_t tiles = ceil_div(M, c.bm) * ceil_div(N, c.bn);
         const int64_t units = num_sms / c.ctas;
-        const double waves = static_cast<double>(ceil_div(tiles, units));
-        const double cost = waves * (static_cast<double>(c.bm) * c.bn / c.ctas) / eff[i];
+        const int64_t num_kb = ceil_div(K, c.bk);
+        const TailSplit ts = tail_split(tiles, units, num_kb, true);
+        double rounds = static_cast<double>(ts.full_tiles / units);
+        if (ts.tail_tiles > 0)
+            rounds += (static_cast<double>(ceil_div(ts.tail_tiles * num_kb, ts.tail_units)) + 2.0) / num_kb;
+        else if (tiles % units)
+            rounds += 1.0;
+        const double cost = rounds * (static_cast<double>(c.bm) * c.bn / c.ctas) / eff[i];
         if (cost < best_cost - 1e-9) {
             best_cost = cost;
             best = i;
@@ -151,7 +201,7 @@ int choose_config(int64_t M, int64_t N, int64_t K, int dtype, int epi, int num_s
     }
     *split = true;
     *group = 0;
-    return model_config(M, N, num_sms);
+    return model_config(M, N, K, num_sms);
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -216,48 +266,6 @@ tl_status validate(const void *A, const void *B, const void *bias, void *C, int6
     if (!aligned(A, 2) || !aligned(B, 2) || !aligned(C, c_f32 ? 4 : 2) || (needs_bias && !aligned(bias, 2)))
         return TL_ERR_MISALIGNED;
     return TL_OK;
-}
-
-// How the tiles of one launch are cut into work items.  Tiles fill whole
-// rounds of `units` (CTAs, or CTA pairs) first.  The tiles of a last, partial
-// round would leave units idle for a whole tile's time; instead their
-// k-blocks can be spread evenly over the units, each unit taking one
-// consecutive range (which may end inside the next tile).  A tile whose
-// k-blocks fall to several units is summed by the last of them to finish (see
-// the kernel): nobody waits, so nothing depends on all units being resident.
-// The split is taken when it saves at least max(4, num_kb / 8) k-blocks of
-// the last round's time -- below that the partial sums' traffic and the extra
-// epilogue pass eat the gain -- and every unit then gets at least 4 k-blocks.
-struct TailSplit {
-    int64_t full_tiles, tail_tiles, tail_units;
-    int32_t max_parts;  // most units sharing one tile (1: none shared)
-};
-
-TailSplit tail_split(int64_t tiles, int64_t units, int64_t num_kb, bool allow)
-{
-    TailSplit t{tiles, 0, 0, 1};
-    const int64_t rem = tiles % units;
-    if (!allow || rem == 0 || num_kb < 8)
-        return t;
-    const int64_t T = rem * num_kb;
-    const int64_t tail_units = units < T / 4 ? units : T / 4;
-    if (tail_units <= rem)
-        return t;
-    const int64_t saved = num_kb - (T + tail_units - 1) / tail_units;
-    const int64_t need = num_kb / 8 > 4 ? num_kb / 8 : 4;
-    if (saved < need)
-        return t;
-    t.full_tiles = tiles - rem;
-    t.tail_tiles = rem;
-    t.tail_units = tail_units;
-    // units meeting tail tile r: ceil((x + 1) U / T) - 1 for its first and last k-block x
-    for (int64_t r = 0; r < rem; ++r) {
-        const int64_t first = ((r * num_kb + 1) * tail_units + T - 1) / T - 1;
-        const int64_t last = (((r + 1) * num_kb) * tail_units + T - 1) / T - 1;
-        if (last - first + 1 > t.max_parts)
-            t.max_parts = static_cast<int32_t>(last - first + 1);
-    }
-    return t;
 }
 
 tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int64_t M, int64_t N,
