@@ -257,6 +257,10 @@ typedef struct {
                              visited column by column inside a group of this
                              many tile rows, so that the tiles running together
                              share operands in L2); 0: the library's choice     */
+    int32_t force_split;  /* 1: cut a partial last round along K whenever it is
+                             possible (every unit gets at least 4 k-blocks),
+                             even where the library's cost rule says it does
+                             not pay -- for tests and sweeps; not with no_split */
 } tl_gemm_options;
 
 /* tl_gemm with options (NULL options == tl_gemm).  Same arguments and errors;

@@ -66,7 +66,8 @@ def _epi_code(epilogue):
 
 
 def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0, timeout_ns: int = 0,
-         no_split: bool = False, b_transposed: bool = False, out_dtype=None, raster_group: int = 0):
+         no_split: bool = False, b_transposed: bool = False, out_dtype=None, raster_group: int = 0,
+         force_split: bool = False):
     """C = epilogue(A @ B) for row-major CUDA tensors A (M x K) and B (K x N),
     or B given as N x K (``b_transposed=True``: C = epilogue(A @ B.T), the
     layout of a linear layer's weight).
@@ -112,9 +113,10 @@ def gemm(A, B, bias=None, epilogue=None, out=None, stream=None, config: int = 0,
     s = stream if stream is not None else torch.cuda.current_stream(A.device)
     bias_ptr = bias.data_ptr() if bias is not None and epi in TL_EPI_WITH_BIAS else 0
     with torch.cuda.device(A.device):
-        if config or timeout_ns or no_split or b_transposed or c_f32 or raster_group:
+        if config or timeout_ns or no_split or b_transposed or c_f32 or raster_group or force_split:
             opt = Options(config=config, inject_fault=0, timeout_ns=timeout_ns, no_split=int(no_split),
-                          b_layout=int(bool(b_transposed)), c_float32=int(c_f32), raster_group=raster_group)
+                          b_layout=int(bool(b_transposed)), c_float32=int(c_f32), raster_group=raster_group,
+                          force_split=int(bool(force_split)))
             st = tl_gemm_ex(A.data_ptr(), B.data_ptr(), bias_ptr, out.data_ptr(), M, N, K, dt, epi,
                             s.cuda_stream, opt)
         else:
@@ -203,12 +205,13 @@ def check_device(stream=None) -> int:
 
 
 def plan(M, N, K, dtype=TL_F16, epilogue=None, num_sms=148, config=0, ptrs=(256, 256, 256, 256),
-         b_transposed=False, no_split=False, c_float32=False) -> dict:
+         b_transposed=False, no_split=False, c_float32=False, force_split=False, raster_group=0) -> dict:
     """The host plan for a call (no GPU needed): config, grid, padding, store path."""
     a, b, bias, c = ptrs
     epi = _epi_code(epilogue)
-    opt = Options(config=config, b_layout=int(b_transposed), no_split=int(no_split), c_float32=int(c_float32)) \
-        if (config or b_transposed or no_split or c_float32) else None
+    opt = Options(config=config, b_layout=int(b_transposed), no_split=int(no_split), c_float32=int(c_float32),
+                  force_split=int(force_split), raster_group=raster_group) \
+        if (config or b_transposed or no_split or c_float32 or force_split or raster_group) else None
     st, p = tl_gemm_plan(a, b, bias if epi in TL_EPI_WITH_BIAS else 0, c, M, N, K, dtype, epi, num_sms, opt)
     if st != 0:
         raise TLError(st, "tl_gemm_plan")

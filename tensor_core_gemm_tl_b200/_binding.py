@@ -40,10 +40,11 @@ class Options(ctypes.Structure):
     inject_fault (test hook: 1 device-side stall, 2 host-side encode failure), timeout_ns (0 = 10 s), no_split (1 = never split
     the tiles of a short last round), b_layout (1 = B given as N x K),
     c_float32 (1 = C is float32), raster_group (tile rows per rasterisation
-    group, 0 = library's choice)."""
+    group, 0 = library's choice), force_split (1 = cut a partial last round
+    along K whenever possible)."""
     _fields_ = [("config", ctypes.c_int32), ("inject_fault", ctypes.c_int32),
                 ("timeout_ns", ctypes.c_uint64), ("no_split", ctypes.c_int32), ("b_layout", ctypes.c_int32),
-                ("c_float32", ctypes.c_int32), ("raster_group", ctypes.c_int32)]
+                ("c_float32", ctypes.c_int32), ("raster_group", ctypes.c_int32), ("force_split", ctypes.c_int32)]
 
 
 class Plan(ctypes.Structure):

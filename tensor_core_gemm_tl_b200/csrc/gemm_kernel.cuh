@@ -101,7 +101,7 @@ struct GemmParams {
     int32_t full_tiles, tail_tiles, tail_units;
     int32_t num_slots;       // partial-sum slots in the workspace (tail_units + tail_tiles - 1)
     float *partials;         // [slot][cta of the pair][lane quarter][64-column chunk][16 float4][32 lanes]
-    unsigned long long *arrivals;  // [tail tile][cta][lane quarter][64-column chunk]
+    unsigned long long *arrivals;  // [tail tile][cta][lane quarter][warp of the quarter]
     unsigned long long epoch;  // unique per launch, below 2^56
 };
 
@@ -642,90 +642,11 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                         mbar_arrive(tempty_bar(acc));
                 }
             };
-            if (my_last < 0)
-                release_accumulator();
-#pragma unroll 1
-            for (int c = half; c < CHUNKS; c += 2) {
-                uint32_t r[64];
-                if (!check_ok(acc * CF::ACC_COLS + c * 64 + 64 <= CF::TMEM_COLS))
-                    continue;  // outside this CTA's Tensor Memory
-                const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(acc * CF::ACC_COLS + c * 64);
-                tmem_load_32cols(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-                tmem_load_32cols(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-                tmem_load_wait();
-                if (c == my_last)
-                    release_accumulator();
+            // Epilogue of one 32-row x 64-column chunk of C from its fp32 sums
+            // (this warp's rows, columns col0 ..): + bias, GELU, one rounding,
+            // store.
+            auto store_chunk = [&](int c, uint32_t (&r)[64]) {
                 const int col0 = n0 + c * 64;
-                if (col0 >= p.N || row0 >= p.M)
-                    continue;  // nothing of this chunk lies inside C
-
-                if (shared_tile) {
-                    // This chunk's fp32 partial sums go to this unit's slot; the
-                    // part that arrives last on the chunk's word adds all the
-                    // parts in k order (first .. last unit) and stores C.  A
-                    // slot holds each warp's chunk as 16 float4 columns of 32
-                    // lanes, so every access below is 512 contiguous bytes.
-                    const size_t slab_f4 = static_cast<size_t>(CF::BM) * CF::BN / 4;
-                    const size_t chunk_off = ((static_cast<size_t>(q) * CHUNKS + c) * 16) * 32 + lane;
-                    auto slot_f4 = [&](int u) {
-                        // slot u + r is unique per (unit, tail tile)
-                        return reinterpret_cast<float4 *>(p.partials) +
-                               (static_cast<size_t>(u + w.tail) * CF::CTAS + rank) * slab_f4 + chunk_off;
-                    };
-                    if (!check_ok(static_cast<size_t>(t_last + w.tail) < static_cast<size_t>(p.num_slots)))
-                        continue;  // outside the workspace
-                    float4 *mine = slot_f4(unit);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        __stcg(mine + 32 * i, make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                                          __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
-                    // the warp's writes, then one release by lane 0 (the warp
-                    // barrier orders the other lanes' writes before it)
-                    __syncwarp();
-                    unsigned count = 0;
-                    if (lane == 0) {
-                        const size_t word = ((static_cast<size_t>(w.tail) * CF::CTAS + rank) * 4 + q) * CHUNKS + c;
-                        fence_acq_rel_gpu();
-                        count = arrive_tagged(p.arrivals + word, p.epoch);
-                    }
-                    count = __shfl_sync(0xffffffffu, count, 0);
-                    if (count != static_cast<unsigned>(t_last - t_first + 1))
-                        continue;  // an earlier arrival: the last part stores this chunk
-                    __syncwarp();  // lane 0's acquire orders the reads below
-                    // sum = part(first) + part(first + 1) + ... + part(last), this
-                    // unit's own part read back like the others; 8 loads in
-                    // flight per batch
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        float4 acc[8];
-                        const float4 *src = slot_f4(t_first) + 32 * 8 * h;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            acc[i] = __ldcg(src + 32 * i);
-                        for (int u = t_first + 1; u <= t_last; ++u) {
-                            const float4 *su = slot_f4(u) + 32 * 8 * h;
-                            float4 b[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                b[i] = __ldcg(su + 32 * i);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                acc[i].x += b[i].x;
-                                acc[i].y += b[i].y;
-                                acc[i].z += b[i].z;
-                                acc[i].w += b[i].w;
-                            }
-                        }
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            r[32 * h + 4 * i] = __float_as_uint(acc[i].x);
-                            r[32 * h + 4 * i + 1] = __float_as_uint(acc[i].y);
-                            r[32 * h + 4 * i + 2] = __float_as_uint(acc[i].z);
-                            r[32 * h + 4 * i + 3] = __float_as_uint(acc[i].w);
-                        }
-                    }
-                }
-
                 if constexpr (STORE == STORE_TMA) {
                     // this warp's staging box: its previous store must have read it
                     if (lane == 0)
@@ -802,7 +723,7 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         packed[j] = pack2<DT>(v[2 * j], v[2 * j + 1]);
-
+    
                     if constexpr (STORE == STORE_TMA) {
                         // row `lane` of the 32 x 64 box; 16-byte chunk i lands at i ^ (lane & 7)
 #pragma unroll
@@ -833,6 +754,113 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                     if (lane == 0) {
                         tma_store_2d(&tmap_c, smem_addr(buf), col0, row0);
                         bulk_commit_group();
+                    }
+                }
+            };
+            // Chunks this warp stores: c = half, half + 2, ... inside C.
+            auto chunk_in_c = [&](int c) { return n0 + c * 64 < p.N && row0 < p.M; };
+            if (my_last < 0)
+                release_accumulator();
+            if (!shared_tile) {
+#pragma unroll 1
+                for (int c = half; c < CHUNKS; c += 2) {
+                    uint32_t r[64];
+                    if (!check_ok(acc * CF::ACC_COLS + c * 64 + 64 <= CF::TMEM_COLS))
+                        continue;  // outside this CTA's Tensor Memory
+                    const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(acc * CF::ACC_COLS + c * 64);
+                    tmem_load_32cols(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+                    tmem_load_32cols(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+                    tmem_load_wait();
+                    if (c == my_last)
+                        release_accumulator();
+                    if (chunk_in_c(c))
+                        store_chunk(c, r);
+                }
+            } else {
+                // A tile of the split last round.  Every part writes its fp32
+                // partial sums to its own slot, then counts itself on this
+                // warp's arrival word (one per tail tile, CTA, lane quarter and
+                // warp of the quarter); the part that completes the count adds
+                // the parts in k order (first .. last unit, its own read back
+                // like the others) and stores C.  A slot holds each warp's chunk
+                // as 16 float4 columns of 32 lanes: every access is 512
+                // contiguous bytes, and a part's chunk is read with all 16
+                // loads in flight.
+                const size_t slab_f4 = static_cast<size_t>(CF::BM) * CF::BN / 4;
+                auto slot_f4 = [&](int u, int c) {
+                    // slot u + r is unique per (unit, tail tile)
+                    return reinterpret_cast<float4 *>(p.partials) +
+                           (static_cast<size_t>(u + w.tail) * CF::CTAS + rank) * slab_f4 +
+                           ((static_cast<size_t>(q) * CHUNKS + c) * 16) * 32 + lane;
+                };
+                const bool slots_ok = check_ok(static_cast<size_t>(t_last + w.tail) < static_cast<size_t>(p.num_slots));
+                bool any = false;
+#pragma unroll 1
+                for (int c = half; c < CHUNKS; c += 2) {
+                    uint32_t r[64];
+                    if (!check_ok(acc * CF::ACC_COLS + c * 64 + 64 <= CF::TMEM_COLS))
+                        continue;  // outside this CTA's Tensor Memory
+                    const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(acc * CF::ACC_COLS + c * 64);
+                    tmem_load_32cols(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+                    tmem_load_32cols(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+                    tmem_load_wait();
+                    if (c == my_last)
+                        release_accumulator();
+                    if (!chunk_in_c(c) || !slots_ok)
+                        continue;
+                    any = true;
+                    float4 *mine = slot_f4(unit, c);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        __stcg(mine + 32 * i, make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                          __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
+                }
+                if (any) {
+                    // the warp's writes, then one release by lane 0 (the warp
+                    // barrier orders the other lanes' writes before it)
+                    __syncwarp();
+                    unsigned count = 0;
+                    if (lane == 0) {
+                        const size_t word = ((static_cast<size_t>(w.tail) * CF::CTAS + rank) * 4 + q) * 2 + half;
+                        fence_acq_rel_gpu();
+                        count = arrive_tagged(p.arrivals + word, p.epoch);
+                    }
+                    count = __shfl_sync(0xffffffffu, count, 0);
+                    if (count == static_cast<unsigned>(t_last - t_first + 1)) {
+                        __syncwarp();  // lane 0's acquire orders the reads below
+#pragma unroll 1
+                        for (int c = half; c < CHUNKS; c += 2) {
+                            if (!chunk_in_c(c))
+                                continue;
+                            uint32_t r[64];
+                            {
+                                const float4 *src = slot_f4(t_first, c);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) {
+                                    const float4 a = __ldcg(src + 32 * i);
+                                    r[4 * i] = __float_as_uint(a.x);
+                                    r[4 * i + 1] = __float_as_uint(a.y);
+                                    r[4 * i + 2] = __float_as_uint(a.z);
+                                    r[4 * i + 3] = __float_as_uint(a.w);
+                                }
+                            }
+#pragma unroll 1
+                            for (int u = t_first + 1; u <= t_last; ++u) {
+                                const float4 *src = slot_f4(u, c);
+                                float4 b[16];
+#pragma unroll
+                                for (int i = 0; i < 16; ++i)
+                                    b[i] = __ldcg(src + 32 * i);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) {
+                                    r[4 * i] = __float_as_uint(__uint_as_float(r[4 * i]) + b[i].x);
+                                    r[4 * i + 1] = __float_as_uint(__uint_as_float(r[4 * i + 1]) + b[i].y);
+                                    r[4 * i + 2] = __float_as_uint(__uint_as_float(r[4 * i + 2]) + b[i].z);
+                                    r[4 * i + 3] = __float_as_uint(__uint_as_float(r[4 * i + 3]) + b[i].w);
+                                }
+                            }
+                            store_chunk(c, r);
+                        }
                     }
                 }
             }

@@ -113,42 +113,57 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // How the tiles of one launch are cut into work items.  Tiles fill whole
 // rounds of `units` (CTAs, or CTA pairs) first.  The tiles of a last, partial
 // round would leave units idle for a whole tile's time; instead their
-// k-blocks can be spread evenly over the units, each unit taking one
-// consecutive range (which may end inside the next tile).  A tile whose
-// k-blocks fall to several units is summed by the last of them to finish (see
-// the kernel): nobody waits, so nothing depends on all units being resident.
-// The split is taken when it saves at least max(4, num_kb / 8) k-blocks of
-// the last round's time -- below that the partial sums' traffic and the extra
-// epilogue pass eat the gain -- and every unit then gets at least 4 k-blocks.
+// k-blocks can be spread evenly over up to two units per tile, each unit
+// taking one consecutive range (which may end inside the next tile).  A tile
+// whose k-blocks fall to several units is summed by the last of them to
+// finish (see the kernel): nobody waits, so nothing depends on all units
+// being resident.
+//
+// The split costs the last arrival of each tile a chain of round trips to L2
+// (its partial sums out, its arrival count, then every part's sums back in,
+// 16 loads in flight each) -- about two k-blocks of a 256-column tile's time
+// each, four of a narrower tile's.  Under SPLIT_POLICY the split is taken only
+// when the k-blocks it saves exceed that; SPLIT_FORCE takes it whenever the
+// last round is partial and every unit gets at least 4 k-blocks.
+enum SplitMode { SPLIT_NEVER = 0, SPLIT_POLICY = 1, SPLIT_FORCE = 2 };
+
 struct TailSplit {
     int64_t full_tiles, tail_tiles, tail_units;
     int32_t max_parts;  // most units sharing one tile (1: none shared)
 };
 
-TailSplit tail_split(int64_t tiles, int64_t units, int64_t num_kb, bool allow)
+TailSplit tail_split(int64_t tiles, int64_t units, int64_t num_kb, int block_n, int mode)
 {
     TailSplit t{tiles, 0, 0, 1};
     const int64_t rem = tiles % units;
-    if (!allow || rem == 0 || num_kb < 8)
+    if (mode == SPLIT_NEVER || rem == 0 || num_kb < 8)
         return t;
     const int64_t T = rem * num_kb;
-    const int64_t tail_units = units < T / 4 ? units : T / 4;
+    int64_t tail_units = units < 2 * rem ? units : 2 * rem;
+    if (tail_units > T / 4)
+        tail_units = T / 4;
     if (tail_units <= rem)
         return t;
-    const int64_t saved = num_kb - (T + tail_units - 1) / tail_units;
-    const int64_t need = num_kb / 8 > 4 ? num_kb / 8 : 4;
-    if (saved < need)
-        return t;
-    t.full_tiles = tiles - rem;
-    t.tail_tiles = rem;
-    t.tail_units = tail_units;
     // units meeting tail tile r: ceil((x + 1) U / T) - 1 for its first and last k-block x
+    int32_t max_parts = 1;
     for (int64_t r = 0; r < rem; ++r) {
         const int64_t first = ((r * num_kb + 1) * tail_units + T - 1) / T - 1;
         const int64_t last = (((r + 1) * num_kb) * tail_units + T - 1) / T - 1;
-        if (last - first + 1 > t.max_parts)
-            t.max_parts = static_cast<int32_t>(last - first + 1);
+        if (last - first + 1 > max_parts)
+            max_parts = static_cast<int32_t>(last - first + 1);
     }
+    if (mode == SPLIT_POLICY) {
+        const int64_t saved = num_kb - (T + tail_units - 1) / tail_units;
+        const int64_t chunks_per_warp = block_n >= 256 ? 2 : 1;
+        const int64_t round_trips = 2 + chunks_per_warp * max_parts;
+        const int64_t need = round_trips * (block_n >= 256 ? 2 : 4);
+        if (saved < need)
+            return t;
+    }
+    t.full_tiles = tiles - rem;
+    t.tail_tiles = rem;
+    t.tail_units = tail_units;
+    t.max_parts = max_parts;
     return t;
 }
 
@@ -169,7 +184,7 @@ int model_config(int64_t M, int64_t N, int64_t K, int num_sms)
         const int64_t tiles = ceil_div(M, c.bm) * ceil_div(N, c.bn);
         const int64_t units = num_sms / c.ctas;
         const int64_t num_kb = ceil_div(K, c.bk);
-        const TailSplit ts = tail_split(tiles, units, num_kb, true);
+        const TailSplit ts = tail_split(tiles, units, num_kb, c.bn, SPLIT_POLICY);
         double rounds = static_cast<double>(ts.full_tiles / units);
         if (ts.tail_tiles > 0)
             rounds += (static_cast<double>(ceil_div(ts.tail_tiles * num_kb, ts.tail_units)) + 2.0) / num_kb;
@@ -187,19 +202,19 @@ int model_config(int64_t M, int64_t N, int64_t K, int num_sms)
 // The measured choice for this shape (configuration, and whether its last
 // round may be cut along K), else the wave model with the split rule of
 // tail_split.
-int choose_config(int64_t M, int64_t N, int64_t K, int dtype, int epi, int num_sms, bool *split, int *group)
+int choose_config(int64_t M, int64_t N, int64_t K, int dtype, int epi, int num_sms, int *split_mode, int *group)
 {
     for (const TableRow &r : kTable) {
         if (r.m == M && r.n == N && r.k == K && r.dtype == dtype && r.epi == (epi != 0 ? 1 : 0)) {
             const int i = config_index(r.config);
             if (i >= 0) {
-                *split = r.split != 0;
+                *split_mode = r.split != 0 ? SPLIT_FORCE : SPLIT_NEVER;  // measured: split or not
                 *group = r.group;
                 return i;
             }
         }
     }
-    *split = true;
+    *split_mode = SPLIT_POLICY;
     *group = 0;
     return model_config(M, N, K, num_sms);
 }
@@ -257,7 +272,8 @@ tl_status validate(const void *A, const void *B, const void *bias, void *C, int6
     if (opt && (opt->inject_fault < 0 || opt->inject_fault > 2))
         return TL_ERR_INVALID_ARG;
     if (opt && ((opt->no_split != 0 && opt->no_split != 1) || (opt->b_layout != 0 && opt->b_layout != 1) ||
-                (opt->c_float32 != 0 && opt->c_float32 != 1) || opt->raster_group < 0))
+                (opt->c_float32 != 0 && opt->c_float32 != 1) || opt->raster_group < 0 ||
+                (opt->force_split != 0 && opt->force_split != 1) || (opt->force_split && opt->no_split)))
         return TL_ERR_INVALID_ARG;
     const int64_t lim = 0x7FFFFFFFll;
     if (M > lim || N > lim || K > lim)
@@ -277,10 +293,14 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
         return st;
     if (num_sms <= 0)
         return TL_ERR_INVALID_ARG;
-    bool table_split = true;  // a forced configuration splits unless told not to
+    int split_mode = SPLIT_POLICY;  // a forced configuration follows the cost rule
     int table_group = 0;
     int ci = (opt && opt->config > 0) ? opt->config - 1
-                                      : choose_config(M, N, K, dtype, epi, num_sms, &table_split, &table_group);
+                                      : choose_config(M, N, K, dtype, epi, num_sms, &split_mode, &table_group);
+    if (opt && opt->no_split)
+        split_mode = SPLIT_NEVER;
+    else if (opt && opt->force_split)
+        split_mode = SPLIT_FORCE;
     const ConfigEntry &c = kConfigs[ci];
     Plan p{};
     tl_plan &q = p.pub;
@@ -298,7 +318,7 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
     if (max_units > 0 && max_units < units)
         units = max_units;
     p.num_kb = static_cast<int32_t>(ceil_div(K, c.bk));
-    const TailSplit ts = tail_split(tiles, units, p.num_kb, table_split && !(opt && opt->no_split));
+    const TailSplit ts = tail_split(tiles, units, p.num_kb, c.bn, split_mode);
     q.split = ts.max_parts;
     q.full_tiles = static_cast<int32_t>(ts.full_tiles);
     p.tail_tiles = static_cast<int32_t>(ts.tail_tiles);
@@ -338,12 +358,12 @@ tl_status make_plan(const void *A, const void *B, const void *bias, void *C, int
     p.partial_off = p.arrival_off = -1;
     if (ts.tail_tiles > 0) {
         // one 128 x BN fp32 slab per (slot, CTA of the pair); one arrival word
-        // per (tail tile, CTA, TMEM lane quarter, 64-column chunk)
+        // per (tail tile, CTA, TMEM lane quarter, epilogue warp of the quarter)
         const int64_t slabs = static_cast<int64_t>(p.num_slots) * c.ctas;
         p.partial_off = ws;
         ws += ceil_div(slabs * 128 * c.bn * 4, 256) * 256;
         p.arrival_off = ws;
-        ws += ceil_div(ts.tail_tiles * c.ctas * 4 * (c.bn / 64) * 8, 256) * 256;
+        ws += ceil_div(ts.tail_tiles * c.ctas * 4 * 2 * 8, 256) * 256;
     }
     q.workspace_bytes = ws;
     int group = (opt && opt->raster_group > 0) ? opt->raster_group : (table_group > 0 ? table_group : kDefaultRasterGroup);

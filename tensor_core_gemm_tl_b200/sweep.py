@@ -50,7 +50,7 @@ class Operands:
         self.epi = "bias_gelu" if w.epi == wl.EPI_BIAS_GELU else None
 
 
-def time_config(ops, config, launches, warmup, no_split=False, raster_group=0, rest_s=0.5):
+def time_config(ops, config, launches, warmup, no_split=False, raster_group=0, rest_s=0.5, force_split=False):
     """Average milliseconds per launch of `launches` back-to-back launches
     (two events around the whole region), after `rest_s` of idle time and
     `warmup` launches, so that the region runs at the unthrottled clock."""
@@ -62,7 +62,7 @@ def time_config(ops, config, launches, warmup, no_split=False, raster_group=0, r
     def launch(i):
         A, B, C = ops.sets[i % ops.nsets]
         tg.gemm(A, B, ops.bias, epilogue=ops.epi, out=C, config=config, stream=stream, no_split=no_split,
-                raster_group=raster_group)
+                raster_group=raster_group, force_split=force_split)
 
     torch.cuda.synchronize()
     time.sleep(rest_s)
@@ -149,11 +149,11 @@ def main(argv=None):
         ops = Operands(w)
         best = None
         for k in range(1, tg.tl_num_configs() + 1):
-            p = tg.plan(w.M, w.N, w.K, w.dtype, ops.epi, num_sms=sms, config=k)
+            p = tg.plan(w.M, w.N, w.K, w.dtype, ops.epi, num_sms=sms, config=k, force_split=True)
             for split in ((1, 0) if p["split"] > 1 else (0,)):
                 for group in a.groups:
                     ms = time_config(ops, k, a.launches, a.warmup, no_split=not split, raster_group=group,
-                                     rest_s=a.rest_s)
+                                     rest_s=a.rest_s, force_split=bool(split))
                     tflops = w.flops / (ms / 1e3) / 1e12
                     rec = {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "dtype": wl.DTYPE_NAMES[w.dtype],
                            "epi": w.epi, "config": tg.tl_config_name(k - 1), "config_index": k - 1, "split": split,

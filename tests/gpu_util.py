@@ -38,7 +38,7 @@ def from_device(t) -> np.ndarray:
 
 
 def run_library(A_bits, B_bits, bias_bits, dt, epi, config=0, offsets=(0, 0, 0, 0), sync=True,
-                b_transposed=False, out_f32=False):
+                b_transposed=False, out_f32=False, force_split=False):
     """C bits from tl_gemm (through the C ABI) for host bit arrays.  B_bits is
     K x N; with b_transposed the library is given its transpose (N x K).  With
     out_f32 the library writes float32 C and that float32 array is returned."""
@@ -54,7 +54,8 @@ def run_library(A_bits, B_bits, bias_bits, dt, epi, config=0, offsets=(0, 0, 0, 
         out = buf[offsets[3]:].view(M, N)
     else:
         out = torch.empty((M, N), dtype=cdt, device="cuda")
-    tg.gemm(A, B, bias, epilogue=int(epi), out=out, config=config, b_transposed=b_transposed)
+    tg.gemm(A, B, bias, epilogue=int(epi), out=out, config=config, b_transposed=b_transposed,
+            force_split=force_split)
     if sync:
         torch.cuda.synchronize()
         assert tg.check_device() == 0

@@ -248,13 +248,14 @@ def test_binding_rejects_host_and_foreign_tensors_before_any_launch(case, monkey
 
 
 @pytest.mark.parametrize("M,N,K,config,dtype,split,full", [
-    (4096, 4096, 4096, 4, 1, True, 222),    # 256 pair tiles on 74 pairs: 3 rounds + 34 tiles spread over 74
+    # the cost rule: split only when the k-blocks saved exceed the reduction's round trips
+    (4096, 4096, 4096, 4, 1, True, 222),    # 256 pair tiles on 74 pairs: 3 rounds + 34 tiles over 68 pairs
     (4096, 4096, 4096, 1, 1, True, 444),    # 512 single-CTA tiles on 148: 68 left over
-    (1024, 1024, 2048, 1, 1, True, 0),      # 32 tiles on 148 SMs: split-K over every SM
-    (1024, 1024, 1024, 4, 1, True, 0),      # 16 pair tiles on 74 pairs
-    (2560, 640, 1024, 3, 1, True, 148),     # 200 tiles of 128 x 64: one full round, then 52 tiles
-    (128, 16384, 4096, 2, 1, True, 0),      # the skinny shape: 128 tiles on 148 SMs
-    (4000, 3000, 2050, 4, 1, True, 148),    # the ragged shape: 192 pair tiles, 44 in the last round
+    (1024, 1024, 2048, 1, 1, True, 0),      # 32 tiles, 2 units each
+    (1024, 1024, 1024, 4, 1, False, 16),    # 16 pair tiles of 16 k-blocks: too little to save
+    (2560, 640, 1024, 3, 1, False, 200),    # 200 tiles of 128 x 64, 16 k-blocks each
+    (128, 16384, 4096, 2, 1, False, 128),   # the skinny shape: 128 tiles on 148 SMs
+    (4000, 3000, 2050, 4, 1, False, 192),   # the ragged shape: 33 k-blocks per tile
     (8192, 16384, 4096, 4, 1, True, 1998),  # 2048 pair tiles = 27 rounds of 74 + 50
     (700, 900, 333, 4, 1, False, 12),       # too few k-blocks to split
     (16384, 1024, 8192, 4, 1, True, 222),   # the tall shape
@@ -263,14 +264,28 @@ def test_plan_splits_only_a_short_last_round(M, N, K, config, dtype, split, full
     from schedule_model import check_schedule
     p = tg.plan(M, N, K, dtype, None, num_sms=148, config=config)
     tiles = p["tiles_m"] * p["tiles_n"]
-    assert (p["split"] > 1) == split and p["full_tiles"] == (full if split else tiles)
+    assert (p["split"] > 1) == split and p["full_tiles"] == full
     parts = check_schedule(p, 148, K)
     if split:
         slabs = p["num_slots"] * p["cluster_ctas"]
         assert p["workspace_bytes"] >= slabs * 128 * p["block_n"] * 4
-        assert parts <= 254  # the arrival count is 8 bits
+        assert parts <= 3 and p["tail_units"] <= 2 * (tiles - full)  # at most two units per tile on average
     else:
         assert p["workspace_bytes"] == 0 or p["pad_a"] or p["pad_b"]
+    # forcing the split takes it wherever the last round is partial and K is long enough
+    f = tg.plan(M, N, K, dtype, None, num_sms=148, config=config, force_split=True)
+    units = 148 // f["cluster_ctas"]
+    assert (f["split"] > 1) == (tiles % units != 0 and -(-K // 64) >= 8)
+    check_schedule(f, 148, K)
+    # and no_split never does
+    n = tg.plan(M, N, K, dtype, None, num_sms=148, config=config, no_split=True)
+    assert n["split"] == 1 and n["full_tiles"] == tiles and n["tail_units"] == 0
+
+
+def test_split_options_are_validated():
+    for bad in (tg.Options(force_split=2), tg.Options(force_split=1, no_split=1), tg.Options(raster_group=-1)):
+        st, _ = tg.tl_gemm_plan(P, P, 0, P, 64, 64, 64, 0, 0, 148, bad)
+        assert st == tg.Status.INVALID_ARG
 
 
 def test_host_fault_hook_is_valid_and_changes_no_plan():
@@ -422,9 +437,10 @@ def test_split_schedule_covers_every_k_block_once():
 
     @settings(max_examples=600, deadline=None)
     @given(M=st.integers(1, 9000), N=st.integers(1, 9000), K=st.integers(1, 20000),
-           config=st.integers(0, tg.tl_num_configs()), sms=st.sampled_from([148, 132, 20, 8, 2]))
-    def check(M, N, K, config, sms):
-        s, p = tg.tl_gemm_plan(P, P, 0, P, M, N, K, 1, 0, sms, tg.Options(config=config))
+           config=st.integers(0, tg.tl_num_configs()), sms=st.sampled_from([148, 132, 20, 8, 2]),
+           force=st.booleans())
+    def check(M, N, K, config, sms, force):
+        s, p = tg.tl_gemm_plan(P, P, 0, P, M, N, K, 1, 0, sms, tg.Options(config=config, force_split=int(force)))
         assert s == 0
         if p.tiles_m * p.tiles_n <= 20000:
             if check_schedule(p.as_dict(), sms, K) > 1:

@@ -73,7 +73,9 @@ def test_checked_kernel_no_invariant_fires(M, N, K, config, dt, epi, bt, f32):
     out = torch.empty((M, N), dtype=torch.float32 if f32 else (torch.float16 if dt == wl.F16 else torch.bfloat16),
                       device="cuda")
     stream = torch.cuda.current_stream().cuda_stream
-    opt = tg.Options(config=config, b_layout=int(bt), c_float32=int(f32))
+    # the split tail taken wherever the last round is partial: its slots and
+    # arrival words are among the checked invariants
+    opt = tg.Options(config=config, b_layout=int(bt), c_float32=int(f32), force_split=int(config != 0))
     st = lib.tl_gemm_ex(dA.data_ptr(), dB.data_ptr(), dbias.data_ptr() if dbias is not None else None,
                         out.data_ptr(), M, N, K, dt, epi, stream or None, ctypes.byref(opt))
     assert st == 0
