@@ -88,6 +88,28 @@ def shapes(which):
     return named + extra
 
 
+def read_table(path=TABLE):
+    """The rows of an existing table as records (shape, config, split, group, TFLOP/s)."""
+    import re
+    rows = []
+    if not os.path.exists(path):
+        return rows
+    pat = re.compile(r'\{(\d+), (\d+), (\d+), (\d+), (\d+), "([^"]+)", (\d+)(?:, (\d+))?\},\s*//\s*([\d.]+) TFLOP/s')
+    for m in pat.finditer(open(path).read()):
+        M, N, K, dt, epi = (int(m.group(i)) for i in range(1, 6))
+        rows.append({"M": M, "N": N, "K": K, "dtype": "f16" if dt == 0 else "bf16", "epi": epi,
+                     "config": m.group(6), "split": int(m.group(7)), "group": int(m.group(8) or 0),
+                     "tflops": float(m.group(9))})
+    return rows
+
+
+def merge_rows(new_rows, old_rows):
+    """The new rows, then the old rows for shapes the new sweep did not time."""
+    key = lambda r: (r["M"], r["N"], r["K"], r["dtype"], r["epi"])  # noqa: E731
+    seen = {key(r) for r in new_rows}
+    return list(new_rows) + [r for r in old_rows if key(r) not in seen]
+
+
 def write_table(best_rows):
     """Write csrc/config_table.inc from the fastest record per shape."""
     lines = ["// Kernel configuration per measured shape: {M, N, K, dtype, epilogue, config, split, raster group}.",
@@ -134,7 +156,7 @@ def main(argv=None):
     a.groups = [int(x) for x in a.groups.split(",")]
     if a.from_jsonl:
         with open(a.from_jsonl) as f:
-            write_table(best_from_records([json.loads(x) for x in f if x.strip()]))
+            write_table(merge_rows(best_from_records([json.loads(x) for x in f if x.strip()]), read_table()))
         return 0
     import torch
     import tensor_core_gemm_tl_b200 as tg
@@ -165,7 +187,7 @@ def main(argv=None):
         del ops
         torch.cuda.empty_cache()
     if a.write:
-        write_table(rows)
+        write_table(merge_rows(rows, read_table()))
     return 0
 
 
