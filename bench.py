@@ -413,6 +413,55 @@ def per_config_entry(w, bench, ms, warm_ms, peaks, clocks):
     return e
 
 
+# The attention forward (the library's next kernel on the tensor cores): the
+# shapes it is measured on, (batch, heads, seq, head_dim, causal), bf16.
+ATTENTION_SHAPES = ((4, 16, 4096, 128, False), (4, 16, 4096, 128, True), (8, 16, 2048, 64, False),
+                    (8, 16, 2048, 64, True))
+
+
+def attention_entries(args, stream, peaks, dist, dev):
+    """tl_attention_fwd timed like the GEMM bursts (a region of back-to-back
+    launches after an idle pause), with PyTorch's scaled_dot_product_attention
+    on the same inputs beside it as context."""
+    import torch
+    import torch.nn.functional as F
+    import tensor_core_gemm_tl_b200 as tg
+    from tensor_core_gemm_tl_b200.compare import attention_flops
+    burst, _ = tensor_peak(peaks, 0.0)
+    out = {}
+    for B, H, S, D, causal in ATTENTION_SHAPES:
+        g = torch.Generator(device=dev).manual_seed(0)
+        q, k, v = (torch.randn(B, H, S, D, device=dev, dtype=torch.bfloat16, generator=g) for _ in range(3))
+        o = torch.empty_like(q)
+        fl = attention_flops(B, H, S, S, D, causal)
+
+        def region(fn):
+            time.sleep(args.rest_s)
+            for _ in range(args.warmup):
+                fn()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            if dist:
+                dist.barrier()
+            torch.cuda.synchronize()
+            t0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            t1.record(stream)
+            torch.cuda.synchronize()
+            return max_over_ranks(t0.elapsed_time(t1) / args.steps, dist, dev)
+
+        ms = region(lambda: tg.attention(q, k, v, causal=causal, out=o, stream=stream))
+        if tg.check_device() != 0:
+            raise RuntimeError("device error in the attention region")
+        ms_sdpa = region(lambda: F.scaled_dot_product_attention(q, k, v, is_causal=causal))
+        tf, tf_sdpa = fl / (ms / 1e3) / 1e12, fl / (ms_sdpa / 1e3) / 1e12
+        out[f"b{B}h{H}s{S}d{D}{'_causal' if causal else ''}_bf16"] = {
+            "ms": round(ms, 5), "tflops": round(tf, 1), "frac": round(tf / burst, 4),
+            "torch_sdpa_tflops": round(tf_sdpa, 1), "of_sdpa": round(tf / tf_sdpa, 3)}
+        del q, k, v, o
+    return out
+
+
 def run_gpu(args, w):
     import torch
     ws, rank, local = dist_env()
@@ -472,6 +521,11 @@ def run_gpu(args, w):
                 b.free()
                 del b
             torch.cuda.empty_cache()
+
+    # ---------------------------------------------------------------- the attention forward, as bursts
+    attention = None
+    if not args.no_attention:
+        attention = attention_entries(args, stream, peaks, dist, dev)
 
     # ---------------------------------------------------------------- end to end through the public API
     # Every step copies its inputs from pinned host memory, runs the GEMM and
@@ -549,6 +603,7 @@ def run_gpu(args, w):
         "gpu_launches": K * head.launches_per_step,
         "clocks": clocks,
         "per_config": per_config,
+        "attention": attention,
         "sustained": sustained,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -608,6 +663,7 @@ def parse(argv=None):
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--no-attention", action="store_true")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be at least 3")

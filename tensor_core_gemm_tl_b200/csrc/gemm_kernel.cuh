@@ -628,6 +628,16 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
                 tail_contributors(w.tail, p, t_first, t_last);
             const bool shared_tile = t_last > t_first;
             const int row0 = tm * CF::TILE_M + static_cast<int>(rank) * CF::BM + q * 32;  // this warp's rows
+            if constexpr (EPI == 1) {
+                // bring this warp's bias columns into L1 while the tile's
+                // products run: the epilogue's bias loads then hit
+                if (p.epi_bias && lane < CHUNKS) {
+                    const int c = half + 2 * (lane >> 1);
+                    const int col = n0 + c * 64 + (lane & 1) * 32;
+                    if (c < CHUNKS && col < p.N)
+                        prefetch_l1(p.bias + col);
+                }
+            }
             if (!wait_bounded<PAIR>(tfull_bar(acc), acc_phase, abort_flag, timeout, ERR_EPILOGUE, peer_abort))
                 break;
             tc_fence_after_sync();
@@ -932,12 +942,14 @@ __global__ void __launch_bounds__(CF::THREADS, 1)
 
 // Zero-padded copy of a rows x cols matrix of 16-bit values (any 2-byte
 // aligned `src`) into dst with a row length of dst_cols (a multiple of 8) and
-// a 16-byte-aligned base.  One warp per row: lane l reads the l-th 16-byte
-// word of the row's aligned span (512 contiguous bytes per warp step), takes
-// the next word from lane l + 1 and shifts the pair into place, so every
-// global access is a whole aligned 16-byte word.  A word is read only when it
-// holds at least one byte of the row (it then lies in memory the row's
-// allocation covers); bytes past `cols` are written as zero.
+// a 16-byte-aligned base.  A warp copies 32 consecutive 16-byte words of one
+// destination row per step (rows x ceil(words / 32) such steps, spread over
+// every warp of the grid, so that thousands of loads are in flight): lane l
+// reads the l-th aligned 16-byte word of the source span, takes the next word
+// from lane l + 1 (lane 31 reads it itself) and shifts the pair into place,
+// so every global access is a whole aligned 16-byte word.  A word is read
+// only when it holds at least one byte of the row (it then lies in memory the
+// row's allocation covers); values past `cols` are written as zero.
 __device__ __forceinline__ uint32_t shift_pair(uint32_t lo, uint32_t hi, uint32_t byte_shift)
 {
     return __funnelshift_r(lo, hi, 8u * byte_shift);
@@ -949,57 +961,58 @@ __global__ void __launch_bounds__(256) pad_copy_kernel(const uint16_t *__restric
 {
     const int lane = threadIdx.x & 31;
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-    const int64_t chunks = dst_cols >> 3;  // 16-byte words of a destination row
-    for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const int64_t chunks = dst_cols >> 3;     // 16-byte words of a destination row
+    const int64_t segs = (chunks + 31) >> 5;  // steps of 32 words per row
+    const int64_t items = rows * segs;
+    for (int64_t it = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); it < items;
+         it += warps) {
+        const int64_t r = it / segs;
+        const int64_t c = ((it - r * segs) << 5) + lane;
         const uintptr_t row_begin = reinterpret_cast<uintptr_t>(src + r * cols);
         const uintptr_t row_end = row_begin + static_cast<uintptr_t>(cols) * 2;
         const uintptr_t base = row_begin & ~static_cast<uintptr_t>(15);
         const uint32_t mis = static_cast<uint32_t>(row_begin - base);  // 0, 2, ..., 14
-        uint4 *drow = reinterpret_cast<uint4 *>(dst + r * dst_cols);
-        for (int64_t c0 = 0; c0 < chunks; c0 += 32) {
-            const int64_t c = c0 + lane;
-            // the aligned word at base + 16 c, if any byte of it is in the row
-            // (also for c == chunks: its first bytes can end chunk c - 1)
-            const uintptr_t wa = base + 16 * static_cast<uintptr_t>(c);
-            uint4 lo = make_uint4(0u, 0u, 0u, 0u);
-            if (wa < row_end)
-                lo = __ldg(reinterpret_cast<const uint4 *>(wa));
-            uint4 hi;
-            hi.x = __shfl_down_sync(0xffffffffu, lo.x, 1);
-            hi.y = __shfl_down_sync(0xffffffffu, lo.y, 1);
-            hi.z = __shfl_down_sync(0xffffffffu, lo.z, 1);
-            hi.w = __shfl_down_sync(0xffffffffu, lo.w, 1);
-            if (lane == 31) {
-                hi = make_uint4(0u, 0u, 0u, 0u);
-                if (mis != 0 && wa + 16 < row_end)
-                    hi = __ldg(reinterpret_cast<const uint4 *>(wa + 16));
-            }
-            if (c >= chunks)
-                continue;
-            // bytes [mis, mis + 16) of lo:hi
-            const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-            const uint32_t q = mis >> 2, b = mis & 3u;
-            uint32_t o[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                // words q + k and q + k + 1 of w, selected without dynamic indexing
-                uint32_t a0 = w[k], a1 = w[k + 1];
-                if (q == 1) { a0 = w[k + 1]; a1 = w[k + 2]; }
-                if (q == 2) { a0 = w[k + 2]; a1 = w[k + 3]; }
-                if (q == 3) { a0 = w[k + 3]; a1 = w[k + 4]; }
-                o[k] = b ? shift_pair(a0, a1, b) : a0;
-            }
-            // zero the values at or past `cols`
-            const int64_t e0 = 8 * c;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                if (e0 + 2 * k >= cols)
-                    o[k] = 0u;
-                else if (e0 + 2 * k + 1 >= cols)
-                    o[k] &= 0xFFFFu;
-            }
-            drow[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        // the aligned word at base + 16 c, if any byte of it is in the row
+        // (also for c == chunks: its first bytes can end chunk c - 1)
+        const uintptr_t wa = base + 16 * static_cast<uintptr_t>(c);
+        uint4 lo = make_uint4(0u, 0u, 0u, 0u);
+        if (wa < row_end)
+            lo = __ldg(reinterpret_cast<const uint4 *>(wa));
+        uint4 hi;
+        hi.x = __shfl_down_sync(0xffffffffu, lo.x, 1);
+        hi.y = __shfl_down_sync(0xffffffffu, lo.y, 1);
+        hi.z = __shfl_down_sync(0xffffffffu, lo.z, 1);
+        hi.w = __shfl_down_sync(0xffffffffu, lo.w, 1);
+        if (lane == 31) {
+            hi = make_uint4(0u, 0u, 0u, 0u);
+            if (mis != 0 && wa + 16 < row_end)
+                hi = __ldg(reinterpret_cast<const uint4 *>(wa + 16));
         }
+        if (c >= chunks)
+            continue;
+        // bytes [mis, mis + 16) of lo:hi
+        const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        const uint32_t q = mis >> 2, b = mis & 3u;
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            // words q + k and q + k + 1 of w, selected without dynamic indexing
+            uint32_t a0 = w[k], a1 = w[k + 1];
+            if (q == 1) { a0 = w[k + 1]; a1 = w[k + 2]; }
+            if (q == 2) { a0 = w[k + 2]; a1 = w[k + 3]; }
+            if (q == 3) { a0 = w[k + 3]; a1 = w[k + 4]; }
+            o[k] = b ? shift_pair(a0, a1, b) : a0;
+        }
+        // zero the values at or past `cols`
+        const int64_t e0 = 8 * c;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (e0 + 2 * k >= cols)
+                o[k] = 0u;
+            else if (e0 + 2 * k + 1 >= cols)
+                o[k] &= 0xFFFFu;
+        }
+        reinterpret_cast<uint4 *>(dst + r * dst_cols)[c] = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
 

@@ -28,7 +28,7 @@ def test_short_bench_run_prints_the_contract_line():
     d = json.loads(lines[0])
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks",
-                "per_config", "sustained"):
+                "per_config", "attention", "sustained"):
         assert key in d, key
     assert d["n_gpus"] == 1 and d["steps"] == steps and d["warmup"] == warmup
     assert d["gpu_launches"] == steps and d["higher_is_better"] is True and d["data"] == "synthetic"
@@ -61,3 +61,8 @@ def test_short_bench_run_prints_the_contract_line():
         assert c["warm_l2_tflops"] > 0
     s = d["sustained"]
     assert s["steps"] >= steps and s["tflops"] > 0
+    # the attention forward beside the GEMMs, each entry self-consistent
+    assert len(d["attention"]) == len(bench.ATTENTION_SHAPES)
+    for name, a in d["attention"].items():
+        assert a["tflops"] > 0 and a["torch_sdpa_tflops"] > 0, name
+        assert abs(a["frac"] - a["tflops"] / float(peaks["bf16_tflops"])) < 1e-3, name
