@@ -80,6 +80,11 @@ CASES = [
     (1, 1, 1, 1, 64),
     (1, 2, 300, 500, 128),
     (1, 4, 512, 512, 64),
+    # head_dim 128 past 256 queries runs on CTA pairs (512 query rows per pair):
+    # ragged query counts, fewer and more keys than queries, several pairs
+    (1, 2, 1000, 777, 128),
+    (2, 1, 513, 1030, 128),
+    (1, 1, 1536, 1536, 128),
 ]
 
 
