@@ -19,7 +19,6 @@
 #include "tl_gemm.h"
 #include "gemm_kernel.cuh"
 #include "attention_kernel.cuh"
-#include "attention_pair_kernel.cuh"
 #include "rowwise_kernels.cuh"
 
 namespace tl {
@@ -722,33 +721,16 @@ AttnEntry make_attn_entry()
 const AttnEntry kAttn64 = make_attn_entry<64>();
 const AttnEntry kAttn128 = make_attn_entry<128>();
 
-// head_dim 128 on CTA pairs: four query tiles per pair (attention_pair_kernel.cuh)
-AttnEntry make_attn_pair_entry()
-{
-    using CF = AttnPairConfig<128>;
-    AttnEntry e;
-    e.smem_bytes = CF::SMEM_BYTES;
-    e.threads = CF::THREADS;
-    e.launch_regs = CF::LAUNCH_REGS;
-    e.tiles_per_cta = CF::TILES;
-    e.fn[0] = attention_pair_fwd_kernel<CF, 0>;
-    e.fn[1] = attention_pair_fwd_kernel<CF, 1>;
-    return e;
-}
-
-const AttnEntry kAttnPair128 = make_attn_pair_entry();
-
-// [BH][S][D] 16-bit tensor as a 3-D map (D innermost), box 64 x box_rows x 1,
+// [BH][S][D] 16-bit tensor as a 3-D map (D innermost), box 64 x 128 x 1,
 // 128-byte swizzle: rows past S read as zero within each (batch, head).
-bool encode_3d_rows(CUtensorMap *map, const void *base, int dtype, int64_t BH, int64_t S, int64_t D,
-                    int box_rows = 128)
+bool encode_3d_rows(CUtensorMap *map, const void *base, int dtype, int64_t BH, int64_t S, int64_t D)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn)
         return false;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(S * D) * 2};
-    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint32_t box[3] = {64, 128, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapDataType dt = dtype == TL_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     return fn(map, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -775,17 +757,10 @@ tl_status attention_validate(const void *Q, const void *K, const void *V, void *
     const int64_t grid_x = causal ? batch * heads : ceil_div(seq_q, 256);
     if (grid_y > 65535 || grid_x > 0x7FFFFFFFll || batch * heads > 0x7FFFFFFFll || seq_k > 0x7FFFFFFFll)
         return TL_ERR_UNSUPPORTED;
-    if (causal && head_dim == 128 && 2 * batch * heads > 0x7FFFFFFFll)
-        return TL_ERR_UNSUPPORTED;  // the CTA-pair kernel puts two CTAs per head along x
     if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || (lse && !aligned(lse, 4)))
         return TL_ERR_MISALIGNED;
     return TL_OK;
 }
-
-// Head_dim 128 runs on CTA pairs (four 128-row query tiles per pair, 512
-// rows) unless the queries fill at most one pair tile, where the single-CTA
-// kernel (two tiles, 256 rows per CTA) wastes less.
-bool attention_uses_pair(int64_t seq_q, int64_t head_dim) { return head_dim == 128 && seq_q > 256; }
 
 tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, float *lse, int64_t batch,
                          int64_t heads, int64_t seq_q, int64_t seq_k, int64_t head_dim, int dtype, int causal,
@@ -800,8 +775,7 @@ tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, f
         return st;
     if (d->cc_major != 10)
         return TL_ERR_UNSUPPORTED;
-    const bool pair = attention_uses_pair(seq_q, head_dim);
-    const AttnEntry &e = pair ? kAttnPair128 : head_dim == 64 ? kAttn64 : kAttn128;
+    const AttnEntry &e = head_dim == 64 ? kAttn64 : kAttn128;
     AttnFn fn = e.fn[dtype];
     {
         // the kernel moves registers between warpgroups; that only fits if
@@ -816,10 +790,7 @@ tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, f
         return st;
     const int64_t BH = batch * heads;
     CUtensorMap tq, tk, tv;
-    // the pair kernel's CTAs each load half of a K block (64 keys) and half of
-    // a V block's head columns (all 128 keys)
-    if (!encode_3d_rows(&tq, Q, dtype, BH, seq_q, head_dim) ||
-        !encode_3d_rows(&tk, K, dtype, BH, seq_k, head_dim, pair ? 64 : 128) ||
+    if (!encode_3d_rows(&tq, Q, dtype, BH, seq_q, head_dim) || !encode_3d_rows(&tk, K, dtype, BH, seq_k, head_dim) ||
         !encode_3d_rows(&tv, V, dtype, BH, seq_k, head_dim))
         return TL_ERR_CUDA;
     AttnParams ap{};
@@ -835,15 +806,13 @@ tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, f
     ap.timeout_ns = kDefaultTimeoutNs;
 
     cudaLaunchConfig_t cfg{};
-    cudaLaunchAttribute attr[2];
-    // blocks start x fastest.  Non-causal: query blocks along x (the CTAs
+    cudaLaunchAttribute attr[1];
+    // blocks start x fastest.  Non-causal: query-tile pairs along x (the CTAs
     // running together share a head's K and V in L2).  Causal: heads along x,
-    // query blocks along y reversed in the kernel, so every head's heaviest
-    // block starts before any lighter one.  A pair kernel's two CTAs are
-    // neighbours along x.
-    const unsigned qblocks = static_cast<unsigned>(pair ? ceil_div(seq_q, 512) : ceil_div(ap.num_qtiles, e.tiles_per_cta));
-    const unsigned cw = pair ? 2u : 1u;
-    cfg.gridDim = causal ? dim3(static_cast<unsigned>(BH) * cw, qblocks, 1) : dim3(qblocks * cw, static_cast<unsigned>(BH), 1);
+    // pairs along y reversed in the kernel, so every head's heaviest pair
+    // starts before any lighter one.
+    const unsigned pairs = static_cast<unsigned>(ceil_div(ap.num_qtiles, e.tiles_per_cta));
+    cfg.gridDim = causal ? dim3(static_cast<unsigned>(BH), pairs, 1) : dim3(pairs, static_cast<unsigned>(BH), 1);
     cfg.blockDim = dim3(static_cast<unsigned>(e.threads), 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(e.smem_bytes);
     cfg.stream = stream;
@@ -851,13 +820,6 @@ tl_status attention_impl(const void *Q, const void *K, const void *V, void *O, f
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (pair) {
-        attr[1].id = cudaLaunchAttributeClusterDimension;
-        attr[1].val.clusterDim.x = 2;
-        attr[1].val.clusterDim.y = 1;
-        attr[1].val.clusterDim.z = 1;
-        cfg.numAttrs = 2;
-    }
     if (cudaLaunchKernelEx(&cfg, fn, tq, tk, tv, ap) != cudaSuccess)
         return TL_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ERR_CUDA;
