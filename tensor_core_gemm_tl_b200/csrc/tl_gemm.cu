@@ -495,9 +495,8 @@ tl_status max_active_clusters(DeviceState *d, KernelFn fn, const cudaLaunchConfi
 tl_status launch_pad(const void *src, int64_t rows, int64_t cols, void *dst, int64_t dst_cols, int num_sms,
                      cudaStream_t stream)
 {
-    // a warp per 32 destination words of a row, eight warps per block
-    const int64_t items = rows * ceil_div(dst_cols / 8, 32);
-    int64_t blocks = ceil_div(items, 8);
+    const int64_t work = rows * (dst_cols / 8);  // 16-byte destination words
+    int64_t blocks = ceil_div(work, 256);
     const int64_t cap = static_cast<int64_t>(num_sms) * 16;
     if (blocks > cap)
         blocks = cap;
