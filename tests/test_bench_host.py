@@ -116,3 +116,35 @@ def test_attention_flop_count_closed_forms():
     Sq, Sk = 1000, 300  # rows past Sk - 1 see all Sk keys
     kept = Sk * (Sk + 1) // 2 + (Sq - Sk) * Sk
     assert attention_flops(B, H, Sq, Sk, D, True) == 4 * B * H * D * kept
+
+
+def test_peak_follows_the_timed_region_length():
+    """A region shorter than a second is a burst (burst peak); a longer one
+    runs power-capped (sustained peak)."""
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6500.0}
+    assert bench.tensor_peak(peaks, 0.015) == (1600.0, "bf16_tflops")
+    assert bench.tensor_peak(peaks, 0.999) == (1600.0, "bf16_tflops")
+    assert bench.tensor_peak(peaks, 1.0) == (1400.0, "bf16_tflops_sustained")
+    assert bench.tensor_peak({"bf16_tflops": 1600.0, "hbm_gbs": 6500.0}, 5.0)[0] == 1600.0
+
+
+def test_bound_of_each_benchmark_configuration():
+    """Roofline class per configuration: launch latency for 256^3, HBM for
+    the 128-row skinny shape, the tensor pipe for the rest."""
+    wl = bench.wl
+    got = {n: bench.bound_of(wl.WORKLOADS[n]) for n in bench.PER_CONFIG}
+    for n, b in got.items():
+        w = wl.WORKLOADS[n]
+        expect = "latency" if w.M == 256 else ("hbm" if w.M == 128 else "tensor")
+        assert b == expect, (n, b)
+
+
+def test_oracle_sample_is_the_same_for_both_cpu_figures():
+    """cpu_baseline and the reference arm time the same row sample: a fixed
+    number of multiply-adds, rows drawn without replacement."""
+    wl = bench.wl
+    for n in bench.PER_CONFIG:
+        w = wl.WORKLOADS[n]
+        r1, r2 = bench.oracle_sample_rows(w), bench.oracle_sample_rows(w)
+        assert (r1 == r2).all() and len(set(r1.tolist())) == len(r1) and r1.max() < w.M
+        assert len(r1) == max(1, min(w.M, round(bench.ORACLE_SAMPLE_MACS / (w.N * w.K))))
