@@ -350,7 +350,7 @@ class GemmBench:
         self.bias = None
 
 
-def timed_region(bench, stream, steps, warmup, ramp_s, rotate=True, sampler=None, dist=None):
+def timed_region(gb, stream, steps, warmup, ramp_s, rotate=True, sampler=None, dist=None):
     """Run an untimed clock ramp and `warmup` steps, then time exactly `steps`
     steps between two events on `stream` (barrier and synchronize on both
     sides).  Returns the region's milliseconds on this rank."""
@@ -359,14 +359,14 @@ def timed_region(bench, stream, steps, warmup, ramp_s, rotate=True, sampler=None
     i = 0
     while time.time() < t_end:
         for _ in range(5):
-            bench.step(i, stream, rotate)
+            gb.step(i, stream, rotate)
             i += 1
         torch.cuda.synchronize()
     for j in range(warmup):
-        bench.step(j, stream, rotate)
+        gb.step(j, stream, rotate)
     torch.cuda.synchronize()
-    if bench.tg.check_device() != 0:
-        raise RuntimeError(f"device error during the warm-up of {bench.w.name}")
+    if gb.tg.check_device() != 0:
+        raise RuntimeError(f"device error during the warm-up of {gb.w.name}")
     # Events only at the two ends of the region: an event between launches
     # would serialise them and hide the overlap of one kernel's set-up with the
     # previous kernel's tail.
@@ -378,13 +378,13 @@ def timed_region(bench, stream, steps, warmup, ramp_s, rotate=True, sampler=None
     with ctx:
         t0.record(stream)
         for j in range(steps):
-            bench.step(j, stream, rotate)
+            gb.step(j, stream, rotate)
         t1.record(stream)
         torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    if bench.tg.check_device() != 0:
-        raise RuntimeError(f"device error in the timed region of {bench.w.name}")
+    if gb.tg.check_device() != 0:
+        raise RuntimeError(f"device error in the timed region of {gb.w.name}")
     return t0.elapsed_time(t1)
 
 
@@ -396,7 +396,7 @@ class _NullCtx:
         return False
 
 
-def per_config_entry(w, bench, ms, warm_ms, peaks, clocks):
+def per_config_entry(w, gb, ms, warm_ms, peaks, clocks):
     tflops = w.flops / (ms / 1e3) / 1e12
     gbs = w.min_bytes() / (ms / 1e3) / 1e9
     peak, peak_name = tensor_peak(peaks, 0.0)
@@ -405,8 +405,9 @@ def per_config_entry(w, bench, ms, warm_ms, peaks, clocks):
     e = {"ms": round(ms, 5), "tflops": round(tflops, 2), "frac": round(tflops / peak, 4),
          "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4), "bound": bound,
          "warm_l2_tflops": round(w.flops / (warm_ms / 1e3) / 1e12, 2),
-         "kernel_config": bench.plan["config_name"], "split": bench.plan["split"],
-         "launches_per_step": bench.launches_per_step, "sm_mhz": clocks["sm_mhz"],
+         "kernel_config": gb.plan["config_name"], "split": gb.plan["split"],
+         "raster_group": gb.plan["raster_group"],
+         "launches_per_step": gb.launches_per_step, "sm_mhz": clocks["sm_mhz"],
          "reasons": clocks["reasons"]}
     # the roofline fraction of the bound that applies
     e["roofline_frac"] = e["frac_hbm"] if bound == "hbm" else e["frac"]
@@ -596,7 +597,7 @@ def run_gpu(args, w):
         "impl": "tl_gemm",
         "config": common_config(w, args.seed, ws),
         "kernel": {"config": head.plan["config_name"], "grid": head.plan["grid"], "split": head.plan["split"],
-                   "accumulate": "f32"},
+                   "raster_group": head.plan["raster_group"], "accumulate": "f32"},
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps, "streams": nstreams},

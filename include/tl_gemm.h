@@ -20,9 +20,11 @@
  * The result is rounded once, to nearest even, from float32 to the input
  * dtype (or kept as float32 with tl_gemm_ex's c_float32 option).  The library
  * also holds the tutorial's adjacent kernels: tl_attention_fwd,
- * tl_softmax_rows and tl_vector_add.  Sums are accumulated in float32 on the tensor cores; the order of
- * the sum is fixed by the kernel configuration, so two calls with the same
- * configuration give bit-identical results.
+ * tl_softmax_rows and tl_vector_add.  Sums are accumulated in float32 on the
+ * tensor cores; the order of the sum is fixed by the kernel configuration and
+ * the work split (tl_gemm_plan), so two calls with the same plan give
+ * bit-identical results (the raster group changes only which tiles run
+ * together).
  *
  * All calls are host functions.  None of them allocates memory that outlives
  * the call; a call that must re-lay out an operand, or whose last round of
@@ -47,7 +49,10 @@
 extern "C" {
 #endif
 
-#define TL_VERSION 1002 /* major * 1000 + minor */
+/* major * 1000 + minor.  2.0: tl_gemm_options gained raster_group and
+ * force_split, and tl_plan gained tail_units, num_slots and raster_group; both
+ * structs grew, so callers built against 1.x must be rebuilt.               */
+#define TL_VERSION 2000
 
 #if defined(__GNUC__)
 #define TL_API __attribute__((visibility("default")))
