@@ -149,6 +149,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--rest-s", type=float, default=0.5, help="idle time before each timed region")
     ap.add_argument("--groups", default="0", help="comma-separated raster groups to try (0: the library's choice)")
+    ap.add_argument("--configs", default=None, help="comma-separated 1-based configurations to try (default: all)")
     ap.add_argument("--shapes", default="named", choices=["named", "all"])
     ap.add_argument("--only", default=None, help="comma-separated workload names")
     ap.add_argument("--from-jsonl", default=None, help="write the table from recorded sweep output")
@@ -170,7 +171,7 @@ def main(argv=None):
     for w in todo:
         ops = Operands(w)
         best = None
-        for k in range(1, tg.tl_num_configs() + 1):
+        for k in ([int(x) for x in a.configs.split(",")] if a.configs else range(1, tg.tl_num_configs() + 1)):
             p = tg.plan(w.M, w.N, w.K, w.dtype, ops.epi, num_sms=sms, config=k, force_split=True)
             for split in ((1, 0) if p["split"] > 1 else (0,)):
                 for group in a.groups:
