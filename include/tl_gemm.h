@@ -106,7 +106,8 @@ typedef void *tl_stream;
  * Layout requirements: every pointer must be aligned to 2 bytes.  Nothing
  * else is required.  When a row stride of A or B is not a multiple of 16
  * bytes (K or N not a multiple of 8) or its base is not 16-byte aligned, the
- * call first copies that operand into a zero-padded temporary; when C's rows
+ * call first copies that operand into a zero-padded temporary with rows of a
+ * whole number of 128-byte lines (64 elements); when C's rows
  * are not 16-byte aligned the epilogue stores element by element instead of
  * through the tensor-memory-access unit.  Both are slower than the aligned
  * path but give the same numbers.

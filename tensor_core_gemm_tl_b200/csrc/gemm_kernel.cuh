@@ -949,6 +949,11 @@ __global__ void __launch_bounds__(256) pad_copy_kernel(const uint16_t *__restric
                                                        int64_t cols, uint16_t *__restrict__ dst,
                                                        int64_t dst_cols)
 {
+    // launched as a programmatic dependent: src may be the previous kernel's
+    // output and dst may still be read by it, so wait for that kernel first;
+    // the GEMM that reads dst waits for this kernel in turn
+    grid_dependency_wait();
+    grid_launch_dependents();
     const int64_t chunks_per_row = dst_cols >> 3;
     const int64_t total = rows * chunks_per_row;
     for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;

@@ -112,14 +112,14 @@ def test_plan_unaligned_k_pads_A_only():
     M, N, K = 4000, 3000, 2050
     p = tg.plan(M, N, K, tg.TL_BF16, "bias_gelu", num_sms=148)
     assert p["pad_a"] == 1 and p["pad_b"] == 0 and p["direct_store"] == 0
-    assert p["workspace_bytes"] == ((M * 2056 * 2 + 255) // 256) * 256
+    assert p["workspace_bytes"] == ((M * 2112 * 2 + 255) // 256) * 256  # rows of whole 128-byte lines
 
 
 def test_plan_unaligned_n_pads_B_and_stores_directly():
     M, N, K = 300, 1001, 64
     p = tg.plan(M, N, K, tg.TL_F16, None, num_sms=148)
     assert p["pad_a"] == 0 and p["pad_b"] == 1 and p["direct_store"] == 1
-    assert p["workspace_bytes"] == ((K * 1008 * 2 + 255) // 256) * 256
+    assert p["workspace_bytes"] == ((K * 1024 * 2 + 255) // 256) * 256
 
 
 def test_plan_misaligned_bases():
@@ -415,10 +415,10 @@ def test_plan_is_total_and_consistent_for_any_shape():
         assert bool(p.direct_store) == (f32 or N % 8 != 0)  # base pointers here are 256-byte aligned
         need = 0
         if p.pad_a:
-            need += M * ((K + 7) // 8 * 8) * 2
+            need += M * ((K + 63) // 64 * 64) * 2
         if p.pad_b:
             rows, cols = (N, K) if bt else (K, N)
-            need += rows * ((cols + 7) // 8 * 8) * 2
+            need += rows * ((cols + 63) // 64 * 64) * 2
         assert p.workspace_bytes >= need
 
     check()

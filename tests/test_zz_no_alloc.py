@@ -94,7 +94,7 @@ def test_noalloc_matches_tl_gemm_on_two_calls_in_a_row(M, N, K, dt, epi, kind):
 
 def test_noalloc_refuses_work_beyond_its_scratch_and_enqueues_nothing():
     import tensor_core_gemm_tl_b200 as tg
-    M, N, K = 20000, 64, 2050  # A padded to 20000 x 2056 x 2 bytes > 64 MiB
+    M, N, K = 20000, 64, 2050  # A padded to 20000 x 2112 x 2 bytes > 64 MiB
     st, plan = tg.tl_gemm_plan(256, 256, 0, 256, M, N, K, wl.BF16, wl.EPI_NONE, 148)
     assert st == 0 and plan.workspace_bytes > SCRATCH_BYTES
     A, B, _ = wl.make_inputs(wl.custom("big", M, N, K, wl.BF16, wl.EPI_NONE), 1)
