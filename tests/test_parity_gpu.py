@@ -152,6 +152,26 @@ def test_unaligned_bases(offsets):
     compare(C, ref, dt, accumulation_bound(A, B, bias, dt, epi, ref))
 
 
+@pytest.mark.parametrize("M,N,K,offsets", [
+    (333, 1002, 1030, (0, 0, 0, 0)),   # K and N even: both copies read 4-byte words
+    (333, 1002, 1030, (2, 2, 0, 0)),   # bases 4 bytes past alignment: still 4-byte words
+    (333, 1002, 1030, (1, 1, 0, 0)),   # bases 2 bytes past alignment: 2-byte values
+    (333, 1001, 1031, (0, 0, 0, 0)),   # K and N odd: 2-byte values
+])
+def test_padded_copies_both_load_paths_vs_oracle(M, N, K, offsets):
+    """The zero-padded copies of A and B read 4-byte words where every source
+    word is 4-byte aligned and 2-byte values otherwise; both paths, for both
+    operands, against the oracle."""
+    m = tg()
+    ptrs = tuple(256 + 2 * o for o in offsets)
+    p = m.plan(M, N, K, wl.BF16, "bias_gelu", ptrs=ptrs)
+    assert p["pad_a"] == 1 and p["pad_b"] == 1
+    A, B, bias = inputs(M, N, K, wl.BF16, wl.EPI_BIAS_GELU, seed=M + N + K + sum(offsets))
+    ref = oracle.gemm(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU)
+    C = run_library(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU, offsets=offsets)
+    compare(C, ref, wl.BF16, accumulation_bound(A, B, bias, wl.BF16, wl.EPI_BIAS_GELU, ref))
+
+
 def test_deterministic_bitwise():
     M, N, K = 1024, 768, 1000
     A, B, bias = inputs(M, N, K, wl.BF16, wl.EPI_BIAS_GELU, seed=42)
