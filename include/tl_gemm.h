@@ -244,7 +244,9 @@ typedef struct {
                              stage without issuing the copy, so the MMA warp's
                              bounded wait runs out and the kernel drains what
                              it issued and returns with TL_ERR_DEVICE_TIMEOUT
-                             recorded (bit 1 of the detail word); 2 makes
+                             recorded (bit 1 of the detail word; the copy and
+                             epilogue warps then wait up to 2 x timeout_ns, so
+                             the MMA warp's wait is the one that runs out); 2 makes
                              the host treat the encoding of A's tensor map as
                              failed: the call returns TL_ERR_CUDA and the GEMM
                              kernel is not launched (padding copies the shape
